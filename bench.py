@@ -1,0 +1,420 @@
+"""Benchmark of the attention hot path: one step = KV append (RoPE of K at global frames + ring
+write) + attention forward (RoPE of Q fused, masked online softmax on tcgen05) over one seeded
+synthetic batch, on every GPU of one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID] [--impl reference]
+
+Prints one JSON line on rank 0. For N > 1 launch with torch.distributed.run: each rank runs
+its own independent step (weak scaling, no data-path collective); the step time is the max over
+ranks. ``--impl reference`` times the fp64 CPU oracle on the host cores instead (bounded sample
+of the same workload per step). Default workload: the Wan2.1-1.3B-shaped bidirectional denoise
+step (21 x 30 x 52 tokens, 12 heads, head_dim 128, dense).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "attention TFLOP/s (unmasked) & % of B200 BF16 peak; RoPE/KV-append GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+MASK_NAMES = {0: "dense", 1: "block-causal", 2: "radial", 3: "block-causal+radial"}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+ATTN_SRC = os.path.join(ROOT, "video_diffusion_transformer_vdit_b200", "csrc", "attn_fwd.cu")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def config_of(w, extra=None):
+    c = {"workload": w.name, "frames_x_grid": f"{w.q_frames}x{w.grid_h}x{w.grid_w}",
+         "q_tokens": w.q_tokens, "kv_tokens": w.kv_tokens, "heads": w.heads,
+         "head_dim": w.head_dim, "mask": MASK_NAMES[w.mask_kind], "q_start_frame": w.q_start,
+         "batch": 1}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------------------ oracle arm
+
+def oracle_sample(w, budget_s: float = 10.0, pilot_rows: int = 16):
+    """Times the oracle on a bounded sample of the workload: the KV appends of one step for all
+    heads, then masked attention for a sample of query rows (all heads). Returns (TFLOP/s in the
+    metric's units, seconds, sample description)."""
+    import oracle
+
+    og = oracle.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, *w.bands, w.theta)
+    om = oracle.Mask(block_causal=bool(w.mask_kind & 1), radial=bool(w.mask_kind & 2),
+                     chunk_frames=w.chunk_frames, w0=w.w0, gamma_shift=w.gamma_shift, lam=w.lam)
+    ft = w.frame_tokens
+    n_kv = w.kv_stream_frames * ft
+    k = synth.bf16_bits_to_f64(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "k"))
+    v = synth.bf16_bits_to_f64(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "v"))
+    first, last = w.window()
+    kpos, kvalid = oracle.cache_positions(w.capacity_frames, first, last, w.grid_h, w.grid_w)
+    qpos_all = oracle.positions(w.q_tokens, w.grid_h, w.grid_w, w.q_start)
+    qbits = synth.qkv_bf16(w.id, w.q_tokens, w.heads, w.head_dim, "q")
+
+    def run(rows):
+        t0 = time.perf_counter()
+        kc = np.zeros((w.heads, w.kv_tokens, w.head_dim))
+        vc = np.zeros_like(kc)
+        for s, n in w.appends:
+            off = (s - w.kv_stream_first_frame) * ft
+            oracle.kv_append(kc, vc, w.capacity_frames, og, k[off:off + n * ft], v[off:off + n * ft], s, n)
+        qp = tuple(p[rows] for p in qpos_all)
+        q = oracle.rope3d(synth.bf16_bits_to_f64(qbits[rows]), qp, og)
+        m = oracle.mask_rows(qp, kpos, kvalid, om)
+        oracle.attention(q, kc.transpose(1, 0, 2), vc.transpose(1, 0, 2), m, w.scale)
+        dt = time.perf_counter() - t0
+        return dt, int(m.sum())
+
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(w.q_tokens, pilot_rows, replace=False))
+    dt, _ = run(rows)
+    n_rows = int(min(w.q_tokens, max(pilot_rows, pilot_rows * budget_s / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(w.q_tokens, n_rows, replace=False))
+    dt, kept = run(rows)
+    flops = 4.0 * w.head_dim * w.heads * kept
+    desc = (f"oracle (fp64 C, OpenMP) KV appends of the step for all {w.heads} heads + RoPE/mask/"
+            f"two-pass attention of {n_rows} random query rows x {w.heads} heads against all "
+            f"{w.kv_tokens} keys; TFLOP/s counts 4*d per kept pair of the sample")
+    return flops / dt / 1e12, dt, desc
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    cores = os.cpu_count()
+    times, vals = [], []
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        val, dt, desc = oracle_sample(w, budget_s=budget)
+        if i >= args.warmup:
+            times.append(dt)
+            vals.append(val)
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic N(0,1), seeded SplitMix64 + Box-Muller, bf16-rounded",
+            "config": config_of(w, {"parallelism": "host cores (OpenMP)"}),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+                power.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def traffic_per_launch(w):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on this
+    workload from the current kernel source (else None)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, None
+    kv = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if ":" in line:
+                a, b = line.split(":", 1)
+                kv[a.strip()] = b.strip()
+    with open(ATTN_SRC, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if kv.get("source_sha256") != sha or kv.get("workload_id") != str(w.id):
+        return None, "kernel changed since the ncu capture" if kv.get("source_sha256") != sha else None
+    try:
+        return float(kv["dram_bytes_per_launch"]), kv.get("note")
+    except (KeyError, ValueError):
+        return None, None
+
+
+def run_gpu(args, w):
+    import video_diffusion_transformer_vdit_b200 as vdit
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = vdit.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, w.bands, w.theta)
+    m = vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+    ft = w.frame_tokens
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    n_kv = w.kv_stream_frames * ft
+    q_h = bf16(synth.qkv_bf16(w.id, w.q_tokens, w.heads, w.head_dim, "q"))
+    k_h = bf16(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "k"))
+    v_h = bf16(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "v"))
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    cache = vdit.KVCache(g, w.capacity_frames, device=dev)
+    # history before the timed append (the earlier chunks of a causal rollout)
+    s_last, n_last = w.appends[-1]
+    for s, n in w.appends[:-1]:
+        off = (s - w.kv_stream_first_frame) * ft
+        cache.append(k[off:off + n * ft], v[off:off + n * ft], s)
+    off_last = (s_last - w.kv_stream_first_frame) * ft
+    k_step, v_step = k[off_last:off_last + n_last * ft], v[off_last:off_last + n_last * ft]
+    cache.append(k_step, v_step, s_last)
+    t_plan = time.perf_counter()
+    plan = vdit.Plan(g, m, w.q_start, w.q_frames, cache=cache)
+    t_plan = time.perf_counter() - t_plan
+    o = torch.empty_like(q)
+    flops = plan.flops()
+    stream = torch.cuda.current_stream()
+    append_bytes = 4 * k_step.numel() * 2  # read K, V; write K', V (bf16)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        vdit.kv_append(cache.k, cache.v, g, w.capacity_frames, k_step, v_step, s_last)
+        if evs:
+            evs[1].record(stream)
+        vdit.attn_forward(plan, q, cache, out=o, scale=w.scale)
+        if evs:
+            evs[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / args.steps
+    attn_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps))
+    app_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
+
+    status = vdit.get_status()
+
+    # standalone RoPE (the C-ABI call on Q, out of place) for its GB/s
+    y = torch.empty_like(q)
+    for _ in range(3):
+        vdit.rope3d_apply(q, g, w.q_start, out=y)
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_rope = 20
+    r0.record(stream)
+    for _ in range(n_rope):
+        vdit.rope3d_apply(q, g, w.q_start, out=y)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    rope_ms = r0.elapsed_time(r1) / n_rope
+    rope_bytes = 2 * q.numel() * 2
+
+    # end to end through the public API: pinned host inputs -> device, step, output -> host
+    q_p, k_p, v_p = q_h.pin_memory(), k_h[off_last:off_last + n_last * ft].pin_memory(), \
+        v_h[off_last:off_last + n_last * ft].pin_memory()
+    o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_step), torch.empty_like(v_step)
+
+    def e2e_step():
+        q_d.copy_(q_p, non_blocking=True)
+        k_d.copy_(k_p, non_blocking=True)
+        v_d.copy_(v_p, non_blocking=True)
+        vdit.kv_append(cache.k, cache.v, g, w.capacity_frames, k_d, v_d, s_last)
+        vdit.attn_forward(plan, q_d, cache, out=o, scale=w.scale)
+        o_p.copy_(o, non_blocking=True)
+
+    n_e2e = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = (q_p.numel() + k_p.numel() + v_p.numel()) * 2
+    d2h = o_p.numel() * 2
+
+    if rank == 0:
+        pk, src = peaks()
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        traffic, tnote = traffic_per_launch(w)
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            val, dt, desc = oracle_sample(w, budget_s=args.cpu_budget)
+            cpu = {"value": val, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                   "sample": desc, "seconds": dt}
+        info = plan.info
+        line = {
+            "metric": METRIC,
+            "value": world * flops / (ms_step * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic N(0,1), seeded SplitMix64 + Box-Muller, bf16-rounded",
+            "config": config_of(w, {
+                "parallelism": f"{world} independent replicas (no collective)",
+                "l2": "inputs larger than L2: %.0f MB touched per step (Q, K/V chunk, caches, O)"
+                      % ((q.numel() * 2 * 2 + append_bytes + cache.k.numel() * 4) / 1e6),
+                "step": "kv_append(newest chunk) + attn_forward (RoPE of Q fused); plan built "
+                        "once per geometry outside the timed region (%.1f ms host)" % (1e3 * t_plan),
+                "tiles": info["tiles"], "full_tiles": info["full_tiles"],
+                "kept_fraction": info["kept_pairs"] / (w.q_tokens * w.kv_tokens)}),
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_kind": f"bf16 dense, sustained ({src})",
+                         "frac_of_burst_peak": achieved / pk["bf16_tflops"],
+                         "traffic": traffic, "traffic_note": tnote,
+                         "algorithmic": "4*head_dim FLOP per kept (query, key, head): %.4g per launch" % flops},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+            "kernels": {
+                "attn_fwd_ms": attn_ms, "attn_fwd_tflops": achieved,
+                "kv_append_ms": app_ms, "kv_append_gbs": append_bytes / (app_ms * 1e-3) / 1e9,
+                "kv_append_frac_hbm": append_bytes / (app_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "rope3d_apply_ms": rope_ms, "rope3d_apply_gbs": rope_bytes / (rope_ms * 1e-3) / 1e9,
+                "rope3d_apply_frac_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "hbm_peak_gbs": pk["hbm_gbs"]},
+            "status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

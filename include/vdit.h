@@ -1,0 +1,178 @@
+/*
+ * vdit.h -- C ABI of libvdit: spatio-temporal self-attention over the latent tokens of a
+ * video diffusion transformer (frames x grid_h x grid_w patches), on one NVIDIA B200 (sm_100a).
+ *
+ * The library computes, for each head,
+ *     o_i = sum_j softmax_j( (R(p_i) q_i) . (R(p_j) k_j) * scale  restricted to mask_ij ) v_j
+ * where R(p) is a 3-D rotary embedding at token position p = (t, h, w) and mask is dense,
+ * block-causal over chunks of latent frames, radial (distance-decayed), or block-causal AND
+ * radial. Passages each call follows:
+ *
+ *   [CRoPE] "Accelerating Video Generation Inference with Sequential-Parallel 3D Positional
+ *           Encoding Using a Global Time Index": section 2.B (global time index
+ *           t_global = t_local + s, s = the chunk's start frame, so no rank or chunk asks another
+ *           for its positions), section 2.A (KV cache of past chunks), section 2.C (RoPE
+ *           frequencies precomputed into contiguous tables; QKV projection and RoPE fused).
+ *   [TR]    "Timeripple: Accelerating vDiTs by Understanding the Spatio-Temporal Correlations
+ *           in Latent Space", Metodologia 1 (RoPE channels form a temporal and two spatial groups).
+ *   [DR]    "DynamicRad: Content-Adaptive Sparse Attention for Long Video Diffusion", section 2
+ *           (radial window whose width decays with temporal distance by a factor gamma;
+ *           long-range factor lambda; static-ratio mode: a fixed, content-free mask).
+ *   [WF]    Wave Forcing / WaveRT news item (block-causal attention over chunks of latent frames,
+ *           frame count divisible by 3; per-layer K/V cache refreshed chunk by chunk).
+ *
+ * Conventions shared by every call
+ *   - Tensors are bf16, contiguous, in device memory, 16-byte aligned.
+ *   - Token order inside a clip or chunk: frame-major, then patch row h, then column w; token n
+ *     of a chunk starting at global frame s has t = s + n / (grid_h*grid_w), h and w local.
+ *   - Q, K, V, O: [tokens, heads, head_dim].
+ *   - KV cache: two buffers [heads, capacity_frames * grid_h * grid_w, head_dim]; global frame f
+ *     lives in frame slot f mod capacity_frames (a ring holding the newest capacity_frames).
+ *     The caller owns the buffers; zero them once before first use so that never-written slots
+ *     hold finite values (they are masked out, but 0 * NaN would still poison O).
+ *   - RoPE: head_dim splits into bands band_t, band_h, band_w (channels in that order from 0);
+ *     each band is a 1-D rotary embedding over adjacent channel pairs (2j, 2j+1) turned by
+ *     pos * theta^(-2j / band). Wan2.1 shapes: 44/42/42 at head_dim 128, 24/20/20 at 64.
+ *   - Every call is asynchronous on the caller's CUDA stream (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream) except vdit_attn_plan, vdit_plan_info and vdit_plan_export,
+ *     which are host-only, and vdit_get_status, which synchronises the device.
+ *   - Errors: each call returns VDIT_OK (0) or a negative VDIT_ERR_* code and never throws;
+ *     vdit_last_error() gives a thread-local message for the last failure on this thread.
+ *     Argument checks happen before any launch, so a rejected call has no effect.
+ */
+#ifndef VDIT_H
+#define VDIT_H
+
+#if defined(__GNUC__)
+#define VDIT_API __attribute__((visibility("default")))
+#else
+#define VDIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    VDIT_OK = 0,
+    VDIT_ERR_INVALID_ARG = -1,  /* null pointer, size out of range, inconsistent geometry     */
+    VDIT_ERR_UNSUPPORTED = -2,  /* valid request this build does not implement (head_dim,...) */
+    VDIT_ERR_MISALIGNED = -3,   /* a tensor pointer is not 16-byte aligned                    */
+    VDIT_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (message has the reason)  */
+    VDIT_ERR_TIMEOUT = -5,      /* a bounded wait inside a kernel gave up (vdit_get_status)    */
+    VDIT_ERR_NOT_UPLOADED = -6  /* vdit_attn_forward on a plan without vdit_plan_upload        */
+};
+
+/* Mask kinds (bit set). */
+#define VDIT_MASK_DENSE 0
+#define VDIT_MASK_BLOCK_CAUSAL 1
+#define VDIT_MASK_RADIAL 2
+
+#define VDIT_TILE 128         /* query and key tile edge of the schedule and of the kernel   */
+#define VDIT_MAX_FRAME 16383  /* largest global frame index the RoPE tables cover           */
+#define VDIT_MAX_GRID 1024    /* largest grid_h and grid_w                                  */
+#define VDIT_MAX_DT 1023      /* largest |t_q - t_k| a plan may contain                     */
+
+/* Token grid, head layout and RoPE bands. heads >= 1; head_dim 64 or 128; bands even, > 0,
+ * band_t + band_h + band_w == head_dim; theta > 1. */
+typedef struct vdit_geom {
+    int grid_h;   /* patch rows per latent frame (Wan2.1 480p: 30) */
+    int grid_w;   /* patch columns per latent frame (Wan2.1 480p: 52) */
+    int heads;
+    int head_dim;
+    int band_t, band_h, band_w;
+    double theta; /* RoPE base, 10000 */
+} vdit_geom;
+
+/* Mask predicate for a query at (t_q, h_q, w_q) and a key at (t_k, h_k, w_k), global frames:
+ *   BLOCK_CAUSAL ([WF]): kept iff floor(t_k / chunk_frames) <= floor(t_q / chunk_frames).
+ *   RADIAL ([DR] sec. 2, static-ratio mode): with dt = |t_q - t_k| and
+ *     d = max(|h_q - h_k|, |w_q - w_k|) (Chebyshev patch distance), kept iff
+ *     (lambda > 0 and dt mod lambda == 0) or d <= w0 * 2^(-gamma_shift * dt).
+ *   Both bits: AND of the two. 0: dense. Keys in never-written cache slots are never kept. */
+typedef struct vdit_mask {
+    int kind;          /* VDIT_MASK_* bits */
+    int chunk_frames;  /* >= 1 when BLOCK_CAUSAL (Wan2.1 causal decode: 3) */
+    long long w0;      /* >= 0 when RADIAL (52 on a 30 x 52 grid) */
+    int gamma_shift;   /* >= 0; gamma = 2^-gamma_shift (1 -> gamma = 1/2) */
+    int lambda;        /* >= 0; 0 disables the long-range frames (8) */
+} vdit_mask;
+
+/* Opaque attention schedule: the non-empty 128 x 128 (query x key) tiles of the mask. */
+typedef struct vdit_plan vdit_plan;
+
+typedef struct vdit_plan_info_t {
+    int q_tokens;        /* query tokens = q_frames * grid_h * grid_w */
+    int kv_tokens;       /* key slots = capacity_frames * grid_h * grid_w */
+    int q_tiles, kv_tiles;
+    int tiles;           /* listed (non-empty) tiles */
+    int full_tiles;      /* listed tiles that are complete and wholly kept */
+    long long kept_pairs;/* kept (query, key) pairs per head */
+    int uploaded;        /* 1 after vdit_plan_upload */
+} vdit_plan_info_t;
+
+/* 3-D RoPE ([CRoPE] 2.B, [TR] Metodologia 1) of n_tokens consecutive tokens of one chunk whose
+ * first token is at global frame start_frame, local patch (0, 0):
+ *   y[n, head, :] = R(start_frame + n / (grid_h*grid_w), (n / grid_w) mod grid_h, n mod grid_w)
+ *                   x[n, head, :].
+ * x, y: device bf16 [n_tokens, heads, head_dim]; y == x (in place) is allowed, other overlap is
+ * not. Math in fp32 with cos/sin from fp64-built tables, result rounded to bf16 (nearest-even).
+ * n_tokens == 0 is a no-op. The first call per device and band set builds the tables
+ * (allocates, synchronous); later calls only launch. start_frame + frames <= VDIT_MAX_FRAME + 1. */
+VDIT_API int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int start_frame,
+                      long long n_tokens, void* stream);
+
+/* KV-cache append ([CRoPE] 2.A; [WF] cache refresh): for frames start_frame .. start_frame +
+ * n_frames - 1 of one chunk, rotates K at its global positions (as vdit_rope3d_apply) and writes
+ * K' and V (unchanged, bit-exact) into frame slot f mod capacity_frames of the caches.
+ * k, v: device bf16 [n_frames * grid_h * grid_w, heads, head_dim]; k_cache, v_cache: device bf16
+ * [heads, capacity_frames * grid_h * grid_w, head_dim], must not overlap k or v.
+ * 1 <= n_frames <= capacity_frames. Window bookkeeping (which frames the cache holds) is the
+ * caller's: it passes that window to vdit_attn_plan. */
+VDIT_API int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache, int capacity_frames,
+                   const void* k, const void* v, int start_frame, int n_frames, void* stream);
+
+/* Tile schedule (host only; [DR] sec. 2 and [WF] masks): queries are q_frames frames starting at
+ * global frame q_start_frame; keys are the capacity_frames-frame ring cache holding global frames
+ * kv_first_frame .. kv_last_frame (at most capacity_frames of them; other slots empty).
+ * Lists, per 128-query tile in ascending order, the 128-key tiles (ascending) that contain a kept
+ * pair, each flagged full iff it is complete and wholly kept. Built exactly from the rectangle
+ * geometry of the tiles (integer arithmetic only), so it is identical to the tile list of the
+ * explicit per-pair mask. *out receives a new plan owned by the caller (vdit_plan_destroy). */
+VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask* m,
+                   int q_start_frame, int q_frames,
+                   int capacity_frames, int kv_first_frame, int kv_last_frame);
+
+/* Copies the plan's schedule and tables to the current device (allocates; the copy is ordered on
+ * stream). Idempotent. Required before vdit_attn_forward. */
+VDIT_API int vdit_plan_upload(vdit_plan* p, void* stream);
+
+VDIT_API int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info);
+
+/* Host copy of the schedule: row_ptr [q_tiles + 1], col_idx [tiles], full [tiles] (0/1). */
+VDIT_API int vdit_plan_export(const vdit_plan* p, int* row_ptr, int* col_idx, unsigned char* full);
+
+VDIT_API void vdit_plan_destroy(vdit_plan* p);
+
+/* Attention forward over an uploaded plan. q: UNROTATED queries, device bf16
+ * [q_tokens, heads, head_dim] (RoPE at the plan's query positions is applied while the Q tile is
+ * staged into shared memory, [CRoPE] 2.C fusion). k_cache: rotated keys, v_cache: values, in the
+ * ring layout above. o: device bf16 [q_tokens, heads, head_dim]. lse: optional device fp32
+ * [heads, q_tokens] (natural-log sum of exp of the kept scaled scores) or NULL. scale > 0
+ * (1/sqrt(head_dim) for the Wan2.1 shapes). Rows with no kept key get o = 0, lse = -inf.
+ * head_dim must be 128 for this kernel (VDIT_ERR_UNSUPPORTED otherwise). */
+VDIT_API int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
+                      void* o, float* lse, float scale, void* stream);
+
+/* Reads and clears the current device's kernel status word: *status = VDIT_OK, or
+ * VDIT_ERR_TIMEOUT when a bounded wait in a kernel gave up since the last read. Synchronises the
+ * device. */
+VDIT_API int vdit_get_status(int* status);
+
+/* Message of the last failed call on this thread ("" if none). Valid until the next call. */
+VDIT_API const char* vdit_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VDIT_H */

@@ -81,6 +81,7 @@ void vo_rope3d(const double *x, double *y, long n_tokens, int heads, int head_di
                const int *t, const int *h, const int *w,
                int band_t, int band_h, int band_w, double theta)
 {
+    #pragma omp parallel for schedule(static)
     for (long n = 0; n < n_tokens; ++n) {
         for (int hh = 0; hh < heads; ++hh) {
             const double *xv = x + (n * heads + hh) * (long)head_dim;

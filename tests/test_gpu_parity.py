@@ -1,0 +1,191 @@
+"""GPU parity: libvdit's CUDA kernels (through the C ABI) against the fp64 oracle on the same
+seeded bf16 inputs. Bit-exact where the operation is a copy or an integer decision (V in the
+cache, the tile schedule); within the bf16 rounding bound for RoPE; max-abs 2e-2 and relative RMS
+1e-2 for attention (bf16 inputs, fp32 accumulation)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import video_diffusion_transformer_vdit_b200 as vdit
+from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS, Workload
+
+from _parity import (assert_close, dev, f64, geom, inputs, mask, ogeom, rope_tolerance,
+                     run_oracle, run_product)
+
+pytestmark = pytest.mark.gpu
+
+
+# ----------------------------------------------------------------------------- RoPE
+
+@pytest.mark.parametrize("wid,start", [(1, 0), (1, 3), (2, 0), (5, 396)])
+def test_rope3d_apply_parity(wid, start):
+    w = WORKLOADS[wid]
+    n = w.q_tokens if wid != 2 else 3 * w.frame_tokens + 77  # ragged token count
+    bits = synth.qkv_bf16(w.id, n, w.heads, w.head_dim, "q")
+    x = dev(bits)
+    y = vdit.rope3d_apply(x, geom(w), start)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(wid)
+    rows = np.unique(np.r_[rng.integers(0, n, 1500), np.arange(n - 40, n), np.arange(0, 40)])
+    pos = oracle.positions(n, w.grid_h, w.grid_w, start)
+    x64 = synth.bf16_bits_to_f64(bits[rows])
+    ref = oracle.rope3d(x64, tuple(p[rows] for p in pos), ogeom(w))
+    got = f64(y)[rows]
+    assert np.all(np.abs(got - ref) <= rope_tolerance(ref, x64))
+
+
+def test_rope3d_apply_in_place_matches_out_of_place():
+    w = WORKLOADS[1]
+    bits = synth.qkv_bf16(9, 5 * w.frame_tokens + 3, w.heads, w.head_dim, "k")
+    a = vdit.rope3d_apply(dev(bits), geom(w), 7)
+    x = dev(bits)
+    vdit.rope3d_apply(x, geom(w), 7, out=x)
+    torch.cuda.synchronize()
+    assert torch.equal(a, x)
+
+
+# ----------------------------------------------------------------------------- KV append
+
+def test_kv_append_ring_parity_small():
+    w = Workload(90, "ring", grid_h=3, grid_w=5, heads=3, head_dim=128, bands=(44, 42, 42),
+                 mask_kind=0, q_start=12, q_frames=3, capacity_frames=7,
+                 appends=tuple((s, 3) for s in range(0, 15, 3)), kv_stream_first_frame=0)
+    _, k, v = inputs(w)
+    _, _, cache, _ = run_product(w, synth.qkv_bf16(90, w.q_tokens, 3, 128, "q"), k, v, lse=False)
+    og = ogeom(w)
+    kc = np.zeros((3, w.kv_tokens, 128))
+    vc = np.zeros_like(kc)
+    ft = w.frame_tokens
+    for s, n in w.appends:
+        oracle.kv_append(kc, vc, 7, og, synth.bf16_bits_to_f64(k[s * ft:(s + n) * ft]),
+                         synth.bf16_bits_to_f64(v[s * ft:(s + n) * ft]), s, n)
+    assert np.array_equal(f64(cache.v), vc)  # V is a bit-exact copy
+    kx = np.zeros_like(kc)
+    for f in range(8, 15):  # unrotated source of each held frame, for the bound
+        slot = f % 7
+        kx[:, slot * ft:(slot + 1) * ft] = synth.bf16_bits_to_f64(k[f * ft:(f + 1) * ft]).transpose(1, 0, 2)
+    got = f64(cache.k)
+    assert np.all(np.abs(got - kc) <= rope_tolerance(kc, kx))
+    assert (cache.first_frame, cache.last_frame) == (8, 14)
+
+
+def test_kv_append_parity_long_rollout_sampled():
+    w = WORKLOADS[5]
+    q, k, v = inputs(w)
+    _, _, cache, _ = run_product(w, q, k, v, lse=False)
+    hs = [0, 17, 39]
+    og = ogeom(w, len(hs))
+    ft = w.frame_tokens
+    kc = np.zeros((3, w.kv_tokens, 128))
+    vc = np.zeros_like(kc)
+    for s, n in w.appends:
+        off = (s - 378) * ft
+        oracle.kv_append(kc, vc, 21, og, synth.bf16_bits_to_f64(k[off:off + n * ft][:, hs]),
+                         synth.bf16_bits_to_f64(v[off:off + n * ft][:, hs]), s, n)
+    rng = np.random.default_rng(3)
+    toks = np.unique(np.r_[rng.integers(0, w.kv_tokens, 3000), np.arange(w.kv_tokens - 60, w.kv_tokens)])
+    gk = f64(cache.k[hs][:, toks])
+    gv = f64(cache.v[hs][:, toks])
+    assert np.array_equal(gv, vc[:, toks])
+    # unrotated source values for the bound: slot s holds frame 378 + s here (378 = 18 * 21)
+    src = synth.bf16_bits_to_f64(k[toks][:, hs]).transpose(1, 0, 2)
+    assert np.all(np.abs(gk - kc[:, toks]) <= rope_tolerance(kc[:, toks], src))
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _full_check(w, q_scale=1.0):
+    q, k, v = inputs(w, q_scale)
+    o, lse, _, _ = run_product(w, q, k, v)
+    rows = np.arange(w.q_tokens)
+    ro, rl = run_oracle(w, q, k, v, rows, range(w.heads))
+    assert_close(f64(o), ro)
+    assert np.max(np.abs(lse.cpu().numpy() - rl)) < 2e-2
+    assert vdit.get_status() == vdit.OK
+
+
+def test_attention_tiny_workload_full():
+    _full_check(WORKLOADS[1])
+
+
+def _medium(kind, q_start, q_frames, cap, appends, first_stream=0, d=128, wid=91, heads=2):
+    return Workload(wid, "medium", grid_h=6, grid_w=10, heads=heads, head_dim=d,
+                    bands=(44, 42, 42) if d == 128 else (24, 20, 20), mask_kind=kind,
+                    q_start=q_start, q_frames=q_frames, capacity_frames=cap, appends=appends,
+                    kv_stream_first_frame=first_stream, chunk_frames=3, w0=4, gamma_shift=1, lam=4)
+
+
+MEDIUM = {
+    # 9 frames x 60 tokens = 540 = 4 x 128 + 28: several tiles and a ragged tail
+    "dense": _medium(0, 0, 9, 9, ((0, 9),)),
+    "causal": _medium(1, 3, 6, 9, ((0, 3), (3, 3), (6, 3))),
+    "radial_ring_wrap": _medium(2, 9, 3, 8, tuple((s, 3) for s in range(0, 12, 3)) + ((12, 1),)),
+    "causal_radial": _medium(3, 6, 3, 9, tuple((s, 3) for s in range(0, 9, 3))),
+    "partial_fill": _medium(1, 3, 3, 12, ((0, 3), (3, 3))),
+    "d64_radial": _medium(2, 0, 7, 7, ((0, 7),), d=64, wid=92, heads=3),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MEDIUM))
+def test_attention_medium_full(name):
+    _full_check(MEDIUM[name])
+
+
+def test_attention_sharp_softmax():
+    # Q scaled by 4: logits of standard deviation ~4 and a peaked softmax (|o| ~ 1), where the
+    # relative-RMS bound is the binding one. The kernel multiplies bf16 operands, so the rotated
+    # q and k carry a relative rounding of up to 2^-9 per element; on 128-term dot products with
+    # |q_i k_i| * scale ~ 0.35 that moves a logit by ~0.015 typically (a few times that at the
+    # tail), i.e. a softmax weight by a few percent, so single outputs near 1 can move by several
+    # 1e-2. Bound: max-abs 0.1 (5x the dense bound), relative RMS 1e-2 unchanged.
+    w = MEDIUM["causal_radial"]
+    q, k, v = inputs(w, 4.0)
+    o, lse, _, _ = run_product(w, q, k, v)
+    ro, rl = run_oracle(w, q, k, v, np.arange(w.q_tokens), range(w.heads))
+    assert_close(f64(o), ro, max_abs=0.1, rel_rms=1e-2)
+    assert np.max(np.abs(lse.cpu().numpy() - rl)) < 5e-2
+
+
+@pytest.mark.parametrize("wid", [2, 3, 4, 5])
+def test_attention_full_size_sampled(wid):
+    w = WORKLOADS[wid]
+    q, k, v = inputs(w)
+    o, lse, _, plan = run_product(w, q, k, v)
+    rng = np.random.default_rng(wid)
+    last_tile = np.arange((w.q_tokens - 1) // 128 * 128, w.q_tokens)
+    rows = np.unique(np.r_[np.arange(0, 64), rng.integers(0, w.q_tokens, 96), last_tile])
+    hs = [0, w.heads // 2, w.heads - 1]
+    ro, rl = run_oracle(w, q, k, v, rows, hs)
+    assert_close(f64(o[rows][:, hs]), ro)
+    assert np.max(np.abs(lse[hs][:, rows].cpu().numpy() - rl)) < 2e-2
+    # every output row is finite and the kernel reported no timeout
+    assert torch.isfinite(o).all()
+    assert vdit.get_status() == vdit.OK
+
+
+def test_attention_is_deterministic():
+    w = MEDIUM["causal_radial"]
+    q, k, v = inputs(w)
+    o1, l1, cache, plan = run_product(w, q, k, v)
+    o2 = vdit.attn_forward(plan, dev(q), cache, scale=w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("q_start,q_frames", [(2, 2), (0, 1)])
+def test_attention_rows_without_keys(q_start, q_frames):
+    # block-causal, cache holds only frame 3 (chunk 1): query frames of chunk 0 see no key
+    # (o = 0, lse = -inf); with q_start=0, q_frames=1 the plan lists no tile at all
+    w = _medium(1, q_start, q_frames, 4, ((3, 1),), first_stream=3, wid=93)
+    q, k, v = inputs(w)
+    o, lse, _, plan = run_product(w, q, k, v)
+    ro, rl = run_oracle(w, q, k, v, np.arange(w.q_tokens), range(w.heads))
+    assert_close(f64(o), ro)
+    gl = lse.cpu().numpy()
+    assert np.array_equal(np.isinf(gl), np.isinf(rl))
+    fin = np.isfinite(rl)
+    assert np.max(np.abs(gl[fin] - rl[fin]), initial=0.0) < 2e-2
+    if q_frames == 1:
+        assert plan.info["tiles"] == 0 and not o.float().abs().sum().item()

@@ -1,0 +1,124 @@
+"""Host-side checks of libvdit that need no GPU: the C ABI loads and exports every declared
+symbol, the tile schedule is bit-identical to the oracle's explicit-mask tile list, and bad
+arguments are rejected before any device work."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+import video_diffusion_transformer_vdit_b200 as vdit
+from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS
+
+
+def test_library_exports_every_declared_symbol():
+    names = vdit.declared_symbols()
+    assert len(names) >= 10
+    L = vdit.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    # the ctypes prototypes cover the same set
+    for n in names:
+        assert getattr(L, n).argtypes is not None or n == "vdit_last_error", n
+
+
+def _geom(w):
+    return vdit.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, w.bands, w.theta)
+
+
+def _mask(w):
+    return vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+
+
+def _oracle_tiles(grid_h, grid_w, q_start, q_frames, cap, first, last, mask_kind, chunk, w0, g, lam):
+    qpos = oracle.positions(q_frames * grid_h * grid_w, grid_h, grid_w, q_start)
+    kpos, kvalid = oracle.cache_positions(cap, first, last, grid_h, grid_w)
+    m = oracle.Mask(block_causal=bool(mask_kind & 1), radial=bool(mask_kind & 2),
+                    chunk_frames=chunk, w0=w0, gamma_shift=g, lam=lam)
+    return oracle.tiles(qpos, kpos, kvalid, m)
+
+
+def _compare(plan, ref):
+    rp, ci, fu = plan.export()
+    orp, oci, ofu, kept = ref
+    assert np.array_equal(rp.numpy(), orp)
+    assert np.array_equal(ci.numpy(), oci)
+    assert np.array_equal(fu.numpy(), ofu)
+    assert plan.info["kept_pairs"] == kept
+    assert plan.info["full_tiles"] == int(ofu.sum())
+
+
+@pytest.mark.parametrize("wid", sorted(WORKLOADS))
+def test_plan_bit_exact_vs_oracle_workloads(wid):
+    w = WORKLOADS[wid]
+    first, last = w.window()
+    plan = vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                     kv_first_frame=first, kv_last_frame=last, upload=False)
+    ref = _oracle_tiles(w.grid_h, w.grid_w, w.q_start, w.q_frames, w.capacity_frames, first, last,
+                        w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+    _compare(plan, ref)
+
+
+def test_plan_counts_of_the_wan_workloads():
+    # non-empty / full tile counts and kept fractions of the four full-size workloads
+    exp = {2: (65536, 65025), 3: (9472, 9180), 4: (30326, 7190), 5: (3998, 1134), 1: (4, 0)}
+    for wid, (tiles, full) in exp.items():
+        w = WORKLOADS[wid]
+        first, last = w.window()
+        info = vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames,
+                         capacity_frames=w.capacity_frames, kv_first_frame=first,
+                         kv_last_frame=last, upload=False).info
+        assert (info["tiles"], info["full_tiles"]) == (tiles, full), wid
+
+
+def test_plan_bit_exact_vs_oracle_random_geometries():
+    rng = np.random.default_rng(7)
+    for _ in range(40):
+        gh, gw = int(rng.integers(1, 9)), int(rng.integers(1, 40))
+        cap = int(rng.integers(1, 12))
+        last = int(rng.integers(0, 40))
+        first = max(0, last - int(rng.integers(0, cap)))
+        q_frames = int(rng.integers(1, 6))
+        q_start = int(rng.integers(max(0, last - 8), last + 3))
+        kind = int(rng.integers(0, 4))
+        chunk = int(rng.integers(1, 5))
+        w0 = int(rng.integers(0, 60))
+        gs = int(rng.integers(0, 3))
+        lam = int(rng.integers(0, 6))
+        g = vdit.Geometry(gh, gw, 1, 64, (24, 20, 20))
+        plan = vdit.Plan(g, vdit.Mask(kind, chunk, w0, gs, lam), q_start, q_frames,
+                         capacity_frames=cap, kv_first_frame=first, kv_last_frame=last, upload=False)
+        ref = _oracle_tiles(gh, gw, q_start, q_frames, cap, first, last, kind, chunk, w0, gs, lam)
+        _compare(plan, ref)
+
+
+def test_plan_rejects_bad_arguments():
+    L = vdit.lib()
+    g = vdit.Geometry(30, 52, 12, 128, (44, 42, 42)).c()
+    m = vdit.Mask.block_causal(3).c()
+    h = ctypes.c_void_p()
+    assert L.vdit_attn_plan(ctypes.byref(h), ctypes.byref(g), ctypes.byref(m), 0, 3, 21, 5, 2) == vdit.ERR_INVALID_ARG
+    assert L.vdit_attn_plan(ctypes.byref(h), ctypes.byref(g), ctypes.byref(m), 0, 3, 2, 0, 5) == vdit.ERR_INVALID_ARG
+    assert b"window" in L.vdit_last_error()
+    bad = vdit.Geometry(30, 52, 12, 96, (32, 32, 32)).c()
+    assert L.vdit_attn_plan(ctypes.byref(h), ctypes.byref(bad), ctypes.byref(m), 0, 3, 21, 0, 20) == vdit.ERR_UNSUPPORTED
+    odd = vdit.Geometry(30, 52, 12, 128, (43, 43, 42)).c()
+    assert L.vdit_attn_plan(ctypes.byref(h), ctypes.byref(odd), ctypes.byref(m), 0, 3, 21, 0, 20) == vdit.ERR_INVALID_ARG
+    far = vdit.Mask.radial().c()
+    assert L.vdit_attn_plan(ctypes.byref(h), ctypes.byref(g), ctypes.byref(far), 5000, 3, 21, 0, 20) == vdit.ERR_UNSUPPORTED
+
+
+def test_calls_reject_null_and_misaligned_pointers_before_device_work():
+    L = vdit.lib()
+    g = vdit.Geometry(30, 52, 12, 128, (44, 42, 42)).c()
+    assert L.vdit_rope3d_apply(ctypes.byref(g), None, None, 0, 10, None) == vdit.ERR_INVALID_ARG
+    assert L.vdit_rope3d_apply(ctypes.byref(g), ctypes.c_void_p(8), ctypes.c_void_p(16), 0, 10, None) == vdit.ERR_MISALIGNED
+    assert L.vdit_rope3d_apply(ctypes.byref(g), None, None, 0, 0, None) == vdit.OK  # empty is a no-op
+    assert L.vdit_kv_append(ctypes.byref(g), ctypes.c_void_p(16), ctypes.c_void_p(32), 21,
+                            ctypes.c_void_p(48), ctypes.c_void_p(64), 0, 22, None) == vdit.ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    m = vdit.Mask().c()
+    assert L.vdit_attn_plan(ctypes.byref(h), ctypes.byref(g), ctypes.byref(m), 0, 21, 21, 0, 20) == vdit.OK
+    assert L.vdit_attn_forward(h, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                               ctypes.c_void_p(16), None, ctypes.c_float(0.1), None) == vdit.ERR_NOT_UPLOADED
+    L.vdit_plan_destroy(h)

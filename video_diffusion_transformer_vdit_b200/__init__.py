@@ -1,0 +1,303 @@
+"""Python binding of libvdit: B200 (sm_100a) spatio-temporal attention for video DiTs.
+
+Argument marshalling only: every step runs in libvdit's CUDA kernels through its C ABI
+(include/vdit.h). PyTorch supplies device memory and the current CUDA stream. There is no CPU
+fallback: without the built library every call raises.
+
+    import video_diffusion_transformer_vdit_b200 as vdit
+    g = vdit.Geometry(grid_h=30, grid_w=52, heads=12, head_dim=128, bands=(44, 42, 42))
+    cache = vdit.KVCache(g, capacity_frames=21, device="cuda")
+    cache.append(k_chunk, v_chunk, start_frame=18)          # RoPE(K) at global frames + ring write
+    plan = vdit.Plan(g, vdit.Mask.block_causal(3), q_start_frame=18, q_frames=3, cache=cache)
+    o = vdit.attn_forward(plan, q_chunk, cache)              # RoPE(Q) fused into the Q load
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvdit.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "vdit.h")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_MISALIGNED = -3
+ERR_CUDA = -4
+ERR_TIMEOUT = -5
+ERR_NOT_UPLOADED = -6
+
+MASK_DENSE = 0
+MASK_BLOCK_CAUSAL = 1
+MASK_RADIAL = 2
+TILE = 128
+
+
+class VditError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libvdit error {code}: {msg}")
+        self.code = code
+
+
+class _Geom(ctypes.Structure):
+    _fields_ = [("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("band_t", ctypes.c_int), ("band_h", ctypes.c_int),
+                ("band_w", ctypes.c_int), ("theta", ctypes.c_double)]
+
+
+class _Mask(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("chunk_frames", ctypes.c_int), ("w0", ctypes.c_longlong),
+                ("gamma_shift", ctypes.c_int), ("lambda_", ctypes.c_int)]
+
+
+class _PlanInfo(ctypes.Structure):
+    _fields_ = [("q_tokens", ctypes.c_int), ("kv_tokens", ctypes.c_int), ("q_tiles", ctypes.c_int),
+                ("kv_tiles", ctypes.c_int), ("tiles", ctypes.c_int), ("full_tiles", ctypes.c_int),
+                ("kept_pairs", ctypes.c_longlong), ("uploaded", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libvdit.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run "
+                               "`python -m video_diffusion_transformer_vdit_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+        gp, mp = ctypes.POINTER(_Geom), ctypes.POINTER(_Mask)
+        L.vdit_rope3d_apply.argtypes = [gp, P, P, I, LL, P]
+        L.vdit_kv_append.argtypes = [gp, P, P, I, P, P, I, I, P]
+        L.vdit_attn_plan.argtypes = [ctypes.POINTER(P), gp, mp, I, I, I, I, I]
+        L.vdit_plan_upload.argtypes = [P, P]
+        L.vdit_plan_info.argtypes = [P, ctypes.POINTER(_PlanInfo)]
+        L.vdit_plan_export.argtypes = [P, P, P, P]
+        L.vdit_plan_destroy.argtypes = [P]
+        L.vdit_plan_destroy.restype = None
+        L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
+        L.vdit_get_status.argtypes = [ctypes.POINTER(I)]
+        L.vdit_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> list:
+    """Names of the functions include/vdit.h declares (for export checks)."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"VDIT_API\s+[\w\s\*]+?\b(vdit_\w+)\s*\(", text)
+
+
+def _check(rc: int) -> None:
+    if rc != OK:
+        raise VditError(rc, lib().vdit_last_error().decode())
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor, name: str) -> ctypes.c_void_p:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+@dataclass(frozen=True)
+class Geometry:
+    """grid_h x grid_w patches per latent frame, heads x head_dim, RoPE bands (t, h, w)."""
+    grid_h: int
+    grid_w: int
+    heads: int
+    head_dim: int
+    bands: Tuple[int, int, int]
+    theta: float = 10000.0
+
+    @property
+    def frame_tokens(self) -> int:
+        return self.grid_h * self.grid_w
+
+    def c(self) -> _Geom:
+        return _Geom(self.grid_h, self.grid_w, self.heads, self.head_dim, *self.bands,
+                     float(self.theta))
+
+
+@dataclass(frozen=True)
+class Mask:
+    """Mask kind bits (MASK_BLOCK_CAUSAL | MASK_RADIAL) and parameters."""
+    kind: int = MASK_DENSE
+    chunk_frames: int = 3
+    w0: int = 52
+    gamma_shift: int = 1
+    lam: int = 8
+
+    @staticmethod
+    def dense() -> "Mask":
+        return Mask(MASK_DENSE)
+
+    @staticmethod
+    def block_causal(chunk_frames: int = 3) -> "Mask":
+        return Mask(MASK_BLOCK_CAUSAL, chunk_frames=chunk_frames)
+
+    @staticmethod
+    def radial(w0: int = 52, gamma_shift: int = 1, lam: int = 8, chunk_frames: Optional[int] = None) -> "Mask":
+        kind = MASK_RADIAL | (MASK_BLOCK_CAUSAL if chunk_frames else 0)
+        return Mask(kind, chunk_frames=chunk_frames or 3, w0=w0, gamma_shift=gamma_shift, lam=lam)
+
+    def c(self) -> _Mask:
+        return _Mask(self.kind, self.chunk_frames, self.w0, self.gamma_shift, self.lam)
+
+
+def rope3d_apply(x: torch.Tensor, g: Geometry, start_frame: int,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """3-D RoPE of x [n_tokens, heads, head_dim] (bf16, CUDA) whose first token is at global
+    frame start_frame. out=x rotates in place."""
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or x.shape[1:] != (g.heads, g.head_dim):
+        raise ValueError("x must be bf16 [n_tokens, heads, head_dim]")
+    y = torch.empty_like(x) if out is None else out
+    gc = g.c()
+    _check(lib().vdit_rope3d_apply(ctypes.byref(gc), _dev_ptr(x, "x"), _dev_ptr(y, "out"),
+                                   int(start_frame), x.shape[0], _stream(stream)))
+    return y
+
+
+def kv_append(k_cache: torch.Tensor, v_cache: torch.Tensor, g: Geometry, capacity_frames: int,
+              k: torch.Tensor, v: torch.Tensor, start_frame: int, stream=None) -> None:
+    """Rotate K at its global frames and write K', V into ring slots f mod capacity_frames."""
+    ft = g.frame_tokens
+    if k.shape != v.shape or k.shape[0] % ft or k.shape[1:] != (g.heads, g.head_dim):
+        raise ValueError("k, v must be [n_frames * frame_tokens, heads, head_dim]")
+    for t in (k, v, k_cache, v_cache):
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bf16")
+    gc = g.c()
+    _check(lib().vdit_kv_append(ctypes.byref(gc), _dev_ptr(k_cache, "k_cache"),
+                                _dev_ptr(v_cache, "v_cache"), int(capacity_frames),
+                                _dev_ptr(k, "k"), _dev_ptr(v, "v"), int(start_frame),
+                                k.shape[0] // ft, _stream(stream)))
+
+
+class KVCache:
+    """Ring KV cache [heads, capacity_frames * frame_tokens, head_dim] (bf16, zero-filled) plus
+    the bookkeeping of which global frames it holds."""
+
+    def __init__(self, g: Geometry, capacity_frames: int, device="cuda"):
+        self.g = g
+        self.capacity_frames = capacity_frames
+        shape = (g.heads, capacity_frames * g.frame_tokens, g.head_dim)
+        self.k = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.first_frame: Optional[int] = None
+        self.last_frame: Optional[int] = None
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, start_frame: int, stream=None) -> None:
+        n = k.shape[0] // self.g.frame_tokens
+        if self.last_frame is not None:
+            if start_frame > self.last_frame + 1:
+                raise ValueError("append would leave a gap of frames")
+            if start_frame < self.first_frame:
+                raise ValueError("frame older than the cache window")
+        kv_append(self.k, self.v, self.g, self.capacity_frames, k, v, start_frame, stream)
+        last = start_frame + n - 1
+        self.last_frame = last if self.last_frame is None else max(self.last_frame, last)
+        first = start_frame if self.first_frame is None else self.first_frame
+        self.first_frame = max(first, self.last_frame - self.capacity_frames + 1)
+
+
+class Plan:
+    """Tile schedule of the mask for q_frames query frames from q_start_frame against the frames
+    a ring cache holds (host-built, exact); uploaded to the current device on construction unless
+    upload=False."""
+
+    def __init__(self, g: Geometry, mask: Mask, q_start_frame: int, q_frames: int,
+                 cache: Optional[KVCache] = None, capacity_frames: Optional[int] = None,
+                 kv_first_frame: Optional[int] = None, kv_last_frame: Optional[int] = None,
+                 upload: bool = True, stream=None):
+        if cache is not None:
+            capacity_frames, kv_first_frame, kv_last_frame = (
+                cache.capacity_frames, cache.first_frame, cache.last_frame)
+        self.g, self.mask = g, mask
+        self.q_start_frame, self.q_frames = q_start_frame, q_frames
+        self._h = ctypes.c_void_p()
+        gc, mc = g.c(), mask.c()
+        _check(lib().vdit_attn_plan(ctypes.byref(self._h), ctypes.byref(gc), ctypes.byref(mc),
+                                    int(q_start_frame), int(q_frames), int(capacity_frames),
+                                    int(kv_first_frame), int(kv_last_frame)))
+        if upload:
+            self.upload(stream)
+
+    def upload(self, stream=None) -> None:
+        _check(lib().vdit_plan_upload(self._h, _stream(stream)))
+
+    @property
+    def info(self) -> dict:
+        i = _PlanInfo()
+        _check(lib().vdit_plan_info(self._h, ctypes.byref(i)))
+        return {f: getattr(i, f) for f, _ in _PlanInfo._fields_}
+
+    def export(self):
+        """(row_ptr, col_idx, full) as CPU int32 / int32 / uint8 tensors."""
+        inf = self.info
+        rp = torch.zeros(inf["q_tiles"] + 1, dtype=torch.int32)
+        ci = torch.zeros(max(1, inf["tiles"]), dtype=torch.int32)
+        fu = torch.zeros(max(1, inf["tiles"]), dtype=torch.uint8)
+        _check(lib().vdit_plan_export(self._h, ctypes.c_void_p(rp.data_ptr()),
+                                      ctypes.c_void_p(ci.data_ptr()), ctypes.c_void_p(fu.data_ptr())))
+        n = inf["tiles"]
+        return rp, ci[:n], fu[:n]
+
+    def flops(self) -> float:
+        """Unmasked-entry FLOPs of one forward: 4 * head_dim per kept (query, key, head)."""
+        return 4.0 * self.g.head_dim * self.g.heads * self.info["kept_pairs"]
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.vdit_plan_destroy(h)
+            self._h = ctypes.c_void_p()
+
+
+def attn_forward(plan: Plan, q: torch.Tensor, cache: Optional[KVCache] = None,
+                 k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 scale: Optional[float] = None, stream=None) -> torch.Tensor:
+    """o = masked softmax(RoPE(q) . K'^T * scale) V over the plan; q is unrotated."""
+    if cache is not None:
+        k_cache, v_cache = cache.k, cache.v
+    g = plan.g
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[1:] != (g.heads, g.head_dim):
+        raise ValueError("q must be bf16 [q_tokens, heads, head_dim]")
+    if q.shape[0] != plan.info["q_tokens"]:
+        raise ValueError("q has a different token count than the plan")
+    o = torch.empty_like(q) if out is None else out
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.head_dim)
+    lse_ptr = ctypes.c_void_p(0)
+    if lse is not None:
+        if lse.dtype != torch.float32 or lse.shape != (g.heads, q.shape[0]) or not lse.is_contiguous():
+            raise ValueError("lse must be fp32 [heads, q_tokens]")
+        lse_ptr = ctypes.c_void_p(lse.data_ptr())
+    _check(lib().vdit_attn_forward(plan._h, _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                                   _dev_ptr(v_cache, "v_cache"), _dev_ptr(o, "out"), lse_ptr,
+                                   float(scale), _stream(stream)))
+    return o
+
+
+def get_status() -> int:
+    """Reads and clears the device status word (OK or ERR_TIMEOUT); synchronises the device."""
+    s = ctypes.c_int(0)
+    _check(lib().vdit_get_status(ctypes.byref(s)))
+    return s.value

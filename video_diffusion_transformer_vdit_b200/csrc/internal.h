@@ -1,0 +1,56 @@
+// Internal helpers shared by the libvdit translation units (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "vdit.h"
+
+namespace vdit {
+
+// Records msg as this thread's last error and returns code.
+int fail(int code, const std::string& msg);
+// Maps a cudaError_t (as int) to VDIT_ERR_CUDA with the CUDA message, or VDIT_OK.
+int cuda_check(int err, const char* what);
+
+// Validates a geometry (bands, head_dim, grid); returns VDIT_OK or an error already recorded.
+int check_geom(const vdit_geom* g);
+
+// Device RoPE tables for one band set on the current device: float2 (cos, sin) rows
+//   t: (VDIT_MAX_FRAME + 1) x band_t/2, h: VDIT_MAX_GRID x band_h/2, w: VDIT_MAX_GRID x band_w/2,
+// built once in fp64 on the host ([CRoPE] 2.C: precomputed contiguous tables, no per-call host
+// work). Returned pointers stay valid until process exit.
+struct RopeTables {
+    const void* t;  // float2*
+    const void* h;
+    const void* w;
+};
+int get_rope_tables(const vdit_geom* g, RopeTables* out);
+
+}  // namespace vdit
+
+// Plan object (host schedule + optional device copy).
+struct vdit_plan {
+    vdit_geom g;
+    vdit_mask m;
+    int q_start, q_frames, cap_frames, kv_first, kv_last;
+    int q_tokens, kv_tokens, n_qt, n_kt;
+    int n_full;
+    int dt_max;  // largest |t_q - t_k| over query frames x held key frames
+    long long kept_pairs;
+    std::vector<int> row_ptr, col_idx;
+    std::vector<unsigned char> full;
+    std::vector<int> slot_frame;  // global frame held by each frame slot, -1 if empty
+    std::vector<int> radius;      // per dt in [0, dt_max]: largest kept Chebyshev distance
+    std::vector<int> qtile_order; // q-tiles sorted by descending tile count (longest first)
+    // device copy
+    int device = -1;
+    void* d_buf = nullptr;
+    const int* d_row_ptr = nullptr;
+    const int* d_col_idx = nullptr;
+    const unsigned char* d_full = nullptr;
+    const int* d_slot_frame = nullptr;
+    const int* d_radius = nullptr;
+    const int* d_qtile_order = nullptr;
+};

@@ -1,0 +1,304 @@
+// Host side of libvdit: error reporting, geometry checks and the tile schedule (vdit_attn_plan).
+//
+// The schedule lists, per 128-query tile, the 128-key tiles holding at least one kept pair of the
+// block-causal / radial mask ("DynamicRad: Content-Adaptive Sparse Attention for Long Video
+// Diffusion", section 2; Wave Forcing / WaveRT news item: block-causal chunks), each flagged full
+// when complete and wholly kept. It is derived without touching individual pairs: a tile's token
+// range splits into row segments (constant frame and patch row h, a contiguous run of columns w),
+// and for two segments every predicate term is either constant (validity, causal chunk order,
+// |dt|, |dh|) or a function of |w_q - w_k| over two integer intervals, whose minimum and maximum
+// are closed forms. Cost is O(tiles x segment pairs) instead of O(tokens^2).
+#include <algorithm>
+#include <climits>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace {
+thread_local std::string g_last_error;
+}
+
+namespace vdit {
+
+int fail(int code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+int cuda_check(int err, const char* what) {
+    if (err == 0) return VDIT_OK;
+    return fail(VDIT_ERR_CUDA, std::string(what) + ": " +
+                                   cudaGetErrorString(static_cast<cudaError_t>(err)));
+}
+
+int check_geom(const vdit_geom* g) {
+    if (!g) return fail(VDIT_ERR_INVALID_ARG, "geometry is NULL");
+    if (g->grid_h < 1 || g->grid_w < 1 || g->grid_h > VDIT_MAX_GRID || g->grid_w > VDIT_MAX_GRID)
+        return fail(VDIT_ERR_INVALID_ARG, "grid_h/grid_w must be in [1, VDIT_MAX_GRID]");
+    if (g->heads < 1) return fail(VDIT_ERR_INVALID_ARG, "heads must be >= 1");
+    if (g->head_dim != 64 && g->head_dim != 128)
+        return fail(VDIT_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (g->band_t <= 0 || g->band_h <= 0 || g->band_w <= 0 || (g->band_t | g->band_h | g->band_w) & 1)
+        return fail(VDIT_ERR_INVALID_ARG, "RoPE bands must be positive and even");
+    if (g->band_t + g->band_h + g->band_w != g->head_dim)
+        return fail(VDIT_ERR_INVALID_ARG, "RoPE bands must sum to head_dim");
+    if (!(g->theta > 1.0)) return fail(VDIT_ERR_INVALID_ARG, "theta must be > 1");
+    long long ft = (long long)g->grid_h * g->grid_w;
+    if (ft * (VDIT_MAX_FRAME + 1) > INT_MAX / 2)
+        return fail(VDIT_ERR_UNSUPPORTED, "frame too large");
+    return VDIT_OK;
+}
+
+}  // namespace vdit
+
+extern "C" const char* vdit_last_error(void) { return g_last_error.c_str(); }
+
+namespace {
+
+struct Seg {
+    int t;      // global frame (queries) or held frame (keys); -1 = empty slot
+    int h;      // patch row
+    int wlo, whi;  // inclusive column range
+};
+
+// Splits tokens [lo, hi) of a frame-major (frame, h, w) sequence into row segments. frame_of maps
+// the local frame index (queries) or the frame slot (keys) to a global frame.
+template <class F>
+void segments(int lo, int hi, int grid_h, int grid_w, F frame_of, std::vector<Seg>& out) {
+    out.clear();
+    const int ft = grid_h * grid_w;
+    int tok = lo;
+    while (tok < hi) {
+        const int f = tok / ft, rem = tok % ft, h = rem / grid_w, w = rem % grid_w;
+        const int run = std::min(hi - tok, grid_w - w);
+        out.push_back(Seg{frame_of(f), h, w, w + run - 1});
+        tok += run;
+    }
+}
+
+// Radius of the radial window at temporal distance dt: the largest Chebyshev distance d with
+// d <= w0 * 2^(-gamma_shift * dt), i.e. floor(w0 / 2^s), s = gamma_shift * dt; INT_MAX when
+// the whole frame is kept (long-range frame, or no radial term).
+int radius_at(const vdit_mask& m, int dt) {
+    if (!(m.kind & VDIT_MASK_RADIAL)) return INT_MAX;
+    if (m.lambda > 0 && dt % m.lambda == 0) return INT_MAX;
+    const long long s = (long long)m.gamma_shift * dt;
+    const long long r = s >= 63 ? 0 : (m.w0 >> s);
+    return r > INT_MAX ? INT_MAX : (int)r;
+}
+
+// Number of (a, b) in [a0, a1] x [b0, b1] with |a - b| <= r.
+long long pairs_within(int a0, int a1, int b0, int b1, int r) {
+    if (r == INT_MAX) return (long long)(a1 - a0 + 1) * (b1 - b0 + 1);
+    long long n = 0;
+    for (int a = a0; a <= a1; ++a) {
+        const long long lo = std::max<long long>(b0, (long long)a - r);
+        const long long hi = std::min<long long>(b1, (long long)a + r);
+        if (hi >= lo) n += hi - lo + 1;
+    }
+    return n;
+}
+
+}  // namespace
+
+extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask* m,
+                              int q_start_frame, int q_frames, int capacity_frames,
+                              int kv_first_frame, int kv_last_frame) {
+    using vdit::fail;
+    if (!out) return fail(VDIT_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (!m) return fail(VDIT_ERR_INVALID_ARG, "mask is NULL");
+    if (m->kind & ~(VDIT_MASK_BLOCK_CAUSAL | VDIT_MASK_RADIAL))
+        return fail(VDIT_ERR_INVALID_ARG, "unknown mask kind bits");
+    if ((m->kind & VDIT_MASK_BLOCK_CAUSAL) && m->chunk_frames < 1)
+        return fail(VDIT_ERR_INVALID_ARG, "chunk_frames must be >= 1");
+    if ((m->kind & VDIT_MASK_RADIAL) && (m->w0 < 0 || m->gamma_shift < 0 || m->lambda < 0))
+        return fail(VDIT_ERR_INVALID_ARG, "radial mask needs w0, gamma_shift, lambda >= 0");
+    if (q_start_frame < 0 || q_frames < 1 || q_start_frame + q_frames - 1 > VDIT_MAX_FRAME)
+        return fail(VDIT_ERR_INVALID_ARG, "query frames out of range");
+    if (capacity_frames < 1 || kv_first_frame < 0 || kv_last_frame < kv_first_frame ||
+        kv_last_frame - kv_first_frame + 1 > capacity_frames || kv_last_frame > VDIT_MAX_FRAME)
+        return fail(VDIT_ERR_INVALID_ARG, "KV window must satisfy 0 <= first <= last, "
+                                          "last - first < capacity_frames");
+
+    vdit_plan* p = new (std::nothrow) vdit_plan();
+    if (!p) return fail(VDIT_ERR_INVALID_ARG, "out of host memory");
+    p->g = *g;
+    p->m = *m;
+    p->q_start = q_start_frame;
+    p->q_frames = q_frames;
+    p->cap_frames = capacity_frames;
+    p->kv_first = kv_first_frame;
+    p->kv_last = kv_last_frame;
+    const int ft = g->grid_h * g->grid_w;
+    const long long qtok = (long long)q_frames * ft, ktok = (long long)capacity_frames * ft;
+    if (qtok > INT_MAX / 2 || ktok > INT_MAX / 2) {
+        delete p;
+        return fail(VDIT_ERR_UNSUPPORTED, "too many tokens");
+    }
+    p->q_tokens = (int)qtok;
+    p->kv_tokens = (int)ktok;
+    p->n_qt = (p->q_tokens + VDIT_TILE - 1) / VDIT_TILE;
+    p->n_kt = (p->kv_tokens + VDIT_TILE - 1) / VDIT_TILE;
+
+    p->slot_frame.assign(capacity_frames, -1);
+    for (int f = kv_first_frame; f <= kv_last_frame; ++f) p->slot_frame[f % capacity_frames] = f;
+
+    const int q_last = q_start_frame + q_frames - 1;
+    p->dt_max = std::max(std::abs(q_last - kv_first_frame), std::abs(kv_last_frame - q_start_frame));
+    if (p->dt_max > VDIT_MAX_DT) {
+        delete p;
+        return fail(VDIT_ERR_UNSUPPORTED, "query and key frames further apart than VDIT_MAX_DT");
+    }
+    p->radius.resize(p->dt_max + 1);
+    for (int dt = 0; dt <= p->dt_max; ++dt) p->radius[dt] = radius_at(*m, dt);
+
+    const bool causal = m->kind & VDIT_MASK_BLOCK_CAUSAL;
+    std::vector<std::vector<Seg>> kseg(p->n_kt);
+    for (int kt = 0; kt < p->n_kt; ++kt)
+        segments(kt * VDIT_TILE, std::min(p->kv_tokens, (kt + 1) * VDIT_TILE), g->grid_h,
+                 g->grid_w, [&](int slot) { return p->slot_frame[slot]; }, kseg[kt]);
+    std::vector<Seg> qs;
+    p->row_ptr.assign(p->n_qt + 1, 0);
+    p->kept_pairs = 0;
+    p->n_full = 0;
+    for (int qt = 0; qt < p->n_qt; ++qt) {
+        const int q0 = qt * VDIT_TILE, q1 = std::min(p->q_tokens, q0 + VDIT_TILE);
+        segments(q0, q1, g->grid_h, g->grid_w, [&](int f) { return q_start_frame + f; }, qs);
+        for (int kt = 0; kt < p->n_kt; ++kt) {
+            const int k0 = kt * VDIT_TILE, k1 = std::min(p->kv_tokens, k0 + VDIT_TILE);
+            bool any = false;
+            bool all = (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE);
+            long long kept = 0;
+            for (const Seg& a : qs) {
+                for (const Seg& b : kseg[kt]) {
+                    if (b.t < 0) { all = false; continue; }
+                    if (causal && b.t / m->chunk_frames > a.t / m->chunk_frames) {
+                        all = false;
+                        continue;
+                    }
+                    const int r = p->radius[std::abs(a.t - b.t)];
+                    if (std::abs(a.h - b.h) > r) { all = false; continue; }
+                    const int dmin = std::max(0, std::max(b.wlo - a.whi, a.wlo - b.whi));
+                    const int dmax = std::max(a.whi - b.wlo, b.whi - a.wlo);
+                    if (dmin <= r) {
+                        any = true;
+                        kept += pairs_within(a.wlo, a.whi, b.wlo, b.whi, r);
+                    }
+                    if (dmax > r) all = false;
+                }
+            }
+            p->kept_pairs += kept;
+            if (any) {
+                p->col_idx.push_back(kt);
+                p->full.push_back(all ? 1 : 0);
+                p->n_full += all;
+            }
+        }
+        p->row_ptr[qt + 1] = (int)p->col_idx.size();
+    }
+    // longest rows first: a persistent kernel that takes q-tiles in this order finishes its
+    // longest work items early and fills the tail with short ones
+    p->qtile_order.resize(p->n_qt);
+    for (int i = 0; i < p->n_qt; ++i) p->qtile_order[i] = i;
+    std::stable_sort(p->qtile_order.begin(), p->qtile_order.end(), [&](int a, int b) {
+        return p->row_ptr[a + 1] - p->row_ptr[a] > p->row_ptr[b + 1] - p->row_ptr[b];
+    });
+    *out = p;
+    return VDIT_OK;
+}
+
+extern "C" int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info) {
+    if (!p || !info) return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or info");
+    info->q_tokens = p->q_tokens;
+    info->kv_tokens = p->kv_tokens;
+    info->q_tiles = p->n_qt;
+    info->kv_tiles = p->n_kt;
+    info->tiles = (int)p->col_idx.size();
+    info->full_tiles = p->n_full;
+    info->kept_pairs = p->kept_pairs;
+    info->uploaded = p->d_buf != nullptr;
+    return VDIT_OK;
+}
+
+extern "C" int vdit_plan_export(const vdit_plan* p, int* row_ptr, int* col_idx,
+                                unsigned char* full) {
+    if (!p || !row_ptr || (!p->col_idx.empty() && (!col_idx || !full)))
+        return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or output");
+    std::memcpy(row_ptr, p->row_ptr.data(), sizeof(int) * p->row_ptr.size());
+    if (!p->col_idx.empty()) {
+        std::memcpy(col_idx, p->col_idx.data(), sizeof(int) * p->col_idx.size());
+        std::memcpy(full, p->full.data(), p->full.size());
+    }
+    return VDIT_OK;
+}
+
+extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
+    using vdit::cuda_check;
+    if (!p) return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan");
+    int dev = 0;
+    if (int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    if (p->d_buf) {
+        if (p->device == dev) return VDIT_OK;
+        return vdit::fail(VDIT_ERR_INVALID_ARG, "plan already uploaded to another device");
+    }
+    // one allocation: row_ptr | qtile_order | slot_frame | radius | col_idx | full
+    auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+    const size_t n_rp = sizeof(int) * p->row_ptr.size(), n_qo = sizeof(int) * p->qtile_order.size();
+    const size_t n_sf = sizeof(int) * p->slot_frame.size(), n_ra = sizeof(int) * p->radius.size();
+    const size_t n_ci = sizeof(int) * std::max<size_t>(1, p->col_idx.size());
+    const size_t n_fu = std::max<size_t>(1, p->full.size());
+    const size_t total = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_ci) + up(n_fu);
+    std::vector<unsigned char> host(total, 0);
+    size_t off = 0;
+    auto put = [&](const void* src, size_t n) {
+        size_t at = off;
+        if (n) std::memcpy(host.data() + off, src, n);
+        off += up(n);
+        return at;
+    };
+    const size_t o_rp = put(p->row_ptr.data(), n_rp);
+    const size_t o_qo = put(p->qtile_order.data(), n_qo);
+    const size_t o_sf = put(p->slot_frame.data(), n_sf);
+    const size_t o_ra = put(p->radius.data(), n_ra);
+    const size_t o_ci = put(p->col_idx.data(), sizeof(int) * p->col_idx.size());
+    off = o_ci + up(n_ci);
+    const size_t o_fu = put(p->full.data(), p->full.size());
+    void* d = nullptr;
+    if (int rc = cuda_check(cudaMalloc(&d, total), "cudaMalloc(plan)")) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int rc = cuda_check(cudaMemcpyAsync(d, host.data(), total, cudaMemcpyHostToDevice, s),
+                            "cudaMemcpyAsync(plan)")) {
+        cudaFree(d);
+        return rc;
+    }
+    // a pageable source is staged before cudaMemcpyAsync returns, so `host` may go now
+    unsigned char* b = static_cast<unsigned char*>(d);
+    p->device = dev;
+    p->d_buf = d;
+    p->d_row_ptr = reinterpret_cast<const int*>(b + o_rp);
+    p->d_qtile_order = reinterpret_cast<const int*>(b + o_qo);
+    p->d_slot_frame = reinterpret_cast<const int*>(b + o_sf);
+    p->d_radius = reinterpret_cast<const int*>(b + o_ra);
+    p->d_col_idx = reinterpret_cast<const int*>(b + o_ci);
+    p->d_full = b + o_fu;
+    (void)o_fu;
+    return VDIT_OK;
+}
+
+extern "C" void vdit_plan_destroy(vdit_plan* p) {
+    if (!p) return;
+    if (p->d_buf) {
+        int cur = 0;
+        cudaGetDevice(&cur);
+        cudaSetDevice(p->device);
+        cudaFree(p->d_buf);
+        cudaSetDevice(cur);
+    }
+    delete p;
+}

@@ -1,0 +1,284 @@
+// 3-D RoPE with a global time index and the KV-cache append (libvdit, sm_100a).
+//
+// "Accelerating Video Generation Inference with Sequential-Parallel 3D Positional Encoding Using
+// a Global Time Index": section 2.B gives each chunk its own temporal positions from its start
+// frame (t = s + local frame) so no gather of the sequence is needed before RoPE; section 2.C
+// precomputes the rotary frequencies into contiguous tables; section 2.A keeps a KV cache of
+// past chunks. "Timeripple" (Metodologia 1) splits the channels into a temporal group and two
+// spatial groups.
+//
+// Both kernels are HBM streams: every (token, head) row is 16-byte-vector read once and written
+// once; a warp owns a run of consecutive tokens, so the token's (t, h, w) is advanced
+// incrementally instead of divided out per element, and the 32 lanes sweep the token's
+// heads x head_dim/8 16-byte chunks (fully coalesced). Each 32-bit word of a chunk is one RoPE
+// pair (channel 2j in the low half, 2j+1 in the high half), rotated in fp32 with a (cos, sin)
+// pair read from the tables (L1/L2 resident) and rounded to bf16 nearest-even.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace vdit {
+
+namespace {
+std::mutex g_tab_mu;
+std::map<std::tuple<int, int, int, int, uint64_t>, RopeTables> g_tabs;
+}  // namespace
+
+int get_rope_tables(const vdit_geom* g, RopeTables* out) {
+    int dev = 0;
+    if (int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    uint64_t tbits;
+    std::memcpy(&tbits, &g->theta, sizeof tbits);
+    auto key = std::make_tuple(dev, g->band_t, g->band_h, g->band_w, tbits);
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    auto it = g_tabs.find(key);
+    if (it != g_tabs.end()) {
+        *out = it->second;
+        return VDIT_OK;
+    }
+    const int bt2 = g->band_t / 2, bh2 = g->band_h / 2, bw2 = g->band_w / 2;
+    const size_t nt = (size_t)(VDIT_MAX_FRAME + 1) * bt2, nh = (size_t)VDIT_MAX_GRID * bh2,
+                 nw = (size_t)VDIT_MAX_GRID * bw2;
+    std::vector<float2> host(nt + nh + nw);
+    auto fill = [&](float2* dst, int rows, int width) {
+        for (int p = 0; p < rows; ++p)
+            for (int j = 0; j < width / 2; ++j) {
+                const double omega = std::pow(g->theta, -2.0 * j / width);
+                const double a = (double)p * omega;
+                dst[(size_t)p * (width / 2) + j] = make_float2((float)std::cos(a), (float)std::sin(a));
+            }
+    };
+    fill(host.data(), VDIT_MAX_FRAME + 1, g->band_t);
+    fill(host.data() + nt, VDIT_MAX_GRID, g->band_h);
+    fill(host.data() + nt + nh, VDIT_MAX_GRID, g->band_w);
+    void* d = nullptr;
+    if (int rc = cuda_check(cudaMalloc(&d, host.size() * sizeof(float2)), "cudaMalloc(rope tables)"))
+        return rc;
+    if (int rc = cuda_check(cudaMemcpy(d, host.data(), host.size() * sizeof(float2),
+                                       cudaMemcpyHostToDevice), "cudaMemcpy(rope tables)")) {
+        cudaFree(d);
+        return rc;
+    }
+    RopeTables t;
+    t.t = d;
+    t.h = static_cast<float2*>(d) + nt;
+    t.w = static_cast<float2*>(d) + nt + nh;
+    g_tabs[key] = t;
+    *out = t;
+    return VDIT_OK;
+}
+
+}  // namespace vdit
+
+namespace {
+
+struct StreamArgs {
+    const uint4* x;     // rope: input; append: K chunk
+    uint4* y;           // rope: output; append: K cache
+    const uint4* v;     // append: V chunk
+    uint4* vc;          // append: V cache
+    long long n_tokens;
+    int cpr_log2;       // log2(head_dim / 8): 16-byte chunks per head row
+    int cpt;            // chunks per token = heads * head_dim / 8
+    int grid_h, grid_w;
+    int start_frame;
+    int cap_frames;     // append: ring capacity in frames
+    long long cap_tok;  // append: capacity_frames * grid_h * grid_w
+    const float2* tt;
+    const float2* th;
+    const float2* tw;
+    int bt2, bh2, bw2;  // pairs per band
+};
+
+// Rotates the four RoPE pairs of one 16-byte chunk (pairs pp0 .. pp0+3) at position (t, h, w).
+__device__ __forceinline__ uint4 rotate_chunk(uint4 in, int pp0, int t, int h, int w,
+                                              const StreamArgs& a) {
+    uint32_t word[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int pp = pp0 + i;
+        float2 cs;
+        if (pp < a.bt2)
+            cs = __ldg(a.tt + (size_t)t * a.bt2 + pp);
+        else if (pp < a.bt2 + a.bh2)
+            cs = __ldg(a.th + h * a.bh2 + (pp - a.bt2));
+        else
+            cs = __ldg(a.tw + w * a.bw2 + (pp - a.bt2 - a.bh2));
+        __nv_bfloat162 b;
+        memcpy(&b, &word[i], 4);
+        const float2 xv = __bfloat1622float2(b);
+        const float y0 = fmaf(xv.x, cs.x, -xv.y * cs.y);
+        const float y1 = fmaf(xv.x, cs.y, xv.y * cs.x);
+        b = __floats2bfloat162_rn(y0, y1);
+        memcpy(&word[i], &b, 4);
+    }
+    return make_uint4(word[0], word[1], word[2], word[3]);
+}
+
+constexpr int kUnroll = 4;
+
+// APPEND = false: y[tok] = RoPE(x[tok]).  APPEND = true: K' = RoPE(k) and V go to the ring slot.
+template <bool APPEND>
+__global__ void __launch_bounds__(256) rope_stream_kernel(StreamArgs a) {
+    const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+    const long long gw = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    const long long per = (a.n_tokens + warps - 1) / warps;
+    long long tok = gw * per;
+    const long long end = tok + per < a.n_tokens ? tok + per : a.n_tokens;
+    if (tok >= end) return;
+    const int ft = a.grid_h * a.grid_w;
+    int f = (int)(tok / ft);
+    int rem = (int)(tok - (long long)f * ft);
+    int h = rem / a.grid_w, w = rem - h * a.grid_w;
+    const int cpr_mask = (1 << a.cpr_log2) - 1;
+    for (; tok < end; ++tok) {
+        const int t = a.start_frame + f;
+        const long long src0 = tok * a.cpt;
+        long long dst_tok = 0;
+        if (APPEND) dst_tok = (long long)(t % a.cap_frames) * ft + rem;
+        for (int k0 = 0; k0 < a.cpt; k0 += 32 * kUnroll) {
+            uint4 xin[kUnroll], vin[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int k = k0 + u * 32 + lane;
+                if (k < a.cpt) {
+                    xin[u] = __ldcs(a.x + src0 + k);
+                    if (APPEND) vin[u] = __ldcs(a.v + src0 + k);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int k = k0 + u * 32 + lane;
+                if (k < a.cpt) {
+                    const int c8 = k & cpr_mask;
+                    const uint4 r = rotate_chunk(xin[u], c8 * 4, t, h, w, a);
+                    if (APPEND) {
+                        const int head = k >> a.cpr_log2;
+                        const long long d = (((long long)head * a.cap_tok + dst_tok) << a.cpr_log2) + c8;
+                        __stcs(a.y + d, r);
+                        __stcs(a.vc + d, vin[u]);
+                    } else {
+                        __stcs(a.y + src0 + k, r);
+                    }
+                }
+            }
+        }
+        // advance (f, h, w) to the next token
+        ++rem;
+        if (++w == a.grid_w) {
+            w = 0;
+            if (++h == a.grid_h) {
+                h = 0;
+                rem = 0;
+                ++f;
+            }
+        }
+    }
+}
+
+int launch_stream(bool append, StreamArgs& a, cudaStream_t s) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long max_warps = (long long)sms * 64;  // 8 blocks x 8 warps per SM resident
+    long long warps = a.n_tokens < max_warps ? a.n_tokens : max_warps;
+    const int blocks = (int)((warps + 7) / 8);
+    if (append)
+        rope_stream_kernel<true><<<blocks, 256, 0, s>>>(a);
+    else
+        rope_stream_kernel<false><<<blocks, 256, 0, s>>>(a);
+    return vdit::cuda_check(cudaGetLastError(), "rope kernel launch");
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int fill_common(const vdit_geom* g, StreamArgs& a) {
+    vdit::RopeTables tabs;
+    if (int rc = vdit::get_rope_tables(g, &tabs)) return rc;
+    a.tt = static_cast<const float2*>(tabs.t);
+    a.th = static_cast<const float2*>(tabs.h);
+    a.tw = static_cast<const float2*>(tabs.w);
+    a.bt2 = g->band_t / 2;
+    a.bh2 = g->band_h / 2;
+    a.bw2 = g->band_w / 2;
+    a.cpr_log2 = g->head_dim == 128 ? 4 : 3;
+    a.cpt = g->heads * (g->head_dim / 8);
+    a.grid_h = g->grid_h;
+    a.grid_w = g->grid_w;
+    return VDIT_OK;
+}
+
+}  // namespace
+
+extern "C" int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int start_frame,
+                                 long long n_tokens, void* stream) {
+    using vdit::fail;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (n_tokens < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens < 0");
+    if (n_tokens == 0) return VDIT_OK;
+    if (!x || !y) return fail(VDIT_ERR_INVALID_ARG, "x or y is NULL");
+    if (!aligned16(x) || !aligned16(y)) return fail(VDIT_ERR_MISALIGNED, "x/y not 16-byte aligned");
+    const long long ft = (long long)g->grid_h * g->grid_w;
+    const long long frames = (n_tokens + ft - 1) / ft;
+    if (start_frame < 0 || start_frame + frames - 1 > VDIT_MAX_FRAME)
+        return fail(VDIT_ERR_INVALID_ARG, "frames outside [0, VDIT_MAX_FRAME]");
+    const long long row_bytes = (long long)g->heads * g->head_dim * 2;
+    const char* xb = static_cast<const char*>(x);
+    char* yb = static_cast<char*>(y);
+    if (xb != yb && xb < yb + n_tokens * row_bytes && yb < xb + n_tokens * row_bytes)
+        return fail(VDIT_ERR_INVALID_ARG, "x and y overlap without being identical");
+    StreamArgs a{};
+    if (int rc = fill_common(g, a)) return rc;
+    a.x = static_cast<const uint4*>(x);
+    a.y = static_cast<uint4*>(y);
+    a.n_tokens = n_tokens;
+    a.start_frame = start_frame;
+    return launch_stream(false, a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
+                              int capacity_frames, const void* k, const void* v, int start_frame,
+                              int n_frames, void* stream) {
+    using vdit::fail;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (!k_cache || !v_cache || !k || !v) return fail(VDIT_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+        return fail(VDIT_ERR_MISALIGNED, "tensor not 16-byte aligned");
+    if (capacity_frames < 1 || n_frames < 1 || n_frames > capacity_frames)
+        return fail(VDIT_ERR_INVALID_ARG, "need 1 <= n_frames <= capacity_frames");
+    if (start_frame < 0 || start_frame + n_frames - 1 > VDIT_MAX_FRAME)
+        return fail(VDIT_ERR_INVALID_ARG, "frames outside [0, VDIT_MAX_FRAME]");
+    const long long ft = (long long)g->grid_h * g->grid_w;
+    const long long row = (long long)g->heads * g->head_dim * 2;
+    const long long chunk_bytes = ft * n_frames * row, cache_bytes = ft * capacity_frames * row;
+    auto overlap = [](const void* a, long long na, const void* b, long long nb) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        return x < y + nb && y < x + na;
+    };
+    if (overlap(k_cache, cache_bytes, v_cache, cache_bytes) ||
+        overlap(k_cache, cache_bytes, k, chunk_bytes) || overlap(k_cache, cache_bytes, v, chunk_bytes) ||
+        overlap(v_cache, cache_bytes, k, chunk_bytes) || overlap(v_cache, cache_bytes, v, chunk_bytes))
+        return fail(VDIT_ERR_INVALID_ARG, "caches overlap each other or the chunk");
+    StreamArgs a{};
+    if (int rc = fill_common(g, a)) return rc;
+    a.x = static_cast<const uint4*>(k);
+    a.v = static_cast<const uint4*>(v);
+    a.y = static_cast<uint4*>(k_cache);
+    a.vc = static_cast<uint4*>(v_cache);
+    a.n_tokens = ft * n_frames;
+    a.start_frame = start_frame;
+    a.cap_frames = capacity_frames;
+    a.cap_tok = ft * capacity_frames;
+    return launch_stream(true, a, static_cast<cudaStream_t>(stream));
+}
