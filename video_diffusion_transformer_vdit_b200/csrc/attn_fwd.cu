@@ -1,26 +1,35 @@
 // Masked spatio-temporal attention forward on tcgen05 tensor cores (libvdit, sm_100a).
 //
 // Computes o = softmax(R(p_q) q . R(p_k) k * scale, restricted to the mask) v for every
-// (query tile, head) of a plan: the O(N^2) step of full spatio-temporal attention ("Accelerating
+// (query block, head) of a plan: the O(N^2) step of full spatio-temporal attention ("Accelerating
 // Video Generation Inference with Sequential-Parallel 3D Positional Encoding Using a Global Time
 // Index", section 1) over the block-causal / radial tile schedule ("DynamicRad", section 2;
 // Wave Forcing / WaveRT block-causal chunks). Only the tiles the plan lists are visited; a tile
 // flagged full skips the per-pair predicate.
 //
-// One CTA = one 128-row query tile of one head; 8 warps:
-//   warp 0      producer: TMA (cp.async.bulk.tensor, SWIZZLE_128B) of the K and V tiles from the
-//               head-major cache into a 2-stage ring, and the key-position table of partial tiles;
-//   warp 1      TMEM allocator and MMA issuer (one thread): S = Q K^T into TMEM columns [0,128),
-//               O += P V into columns [128,256), kind::f16 bf16 x bf16 -> fp32, M = N = 128;
-//   warps 2-3   help stage Q, then idle;
-//   warps 4-7   softmax: thread r owns query row r (TMEM lane r): tcgen05.ld of its S row, mask,
-//               online softmax in fp32 (log2 domain, lazy rescale of O only when the running max
-//               grows by more than 2^8), P as bf16 into shared memory (K-major, 128B swizzle) for
-//               the PV MMA, epilogue (O / l -> bf16, staged through shared memory so the global
-//               stores are 256-byte coalesced rows; natural-log LSE).
+// One CTA = two 128-row query tiles (Q0, Q1) of one head, sharing every K/V tile it loads;
+// 12 warps (3 warpgroups):
+//   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query row r (TMEM lane r);
+//               tcgen05.ld of its S row, mask, online softmax in fp32 (log2 domain; O is rescaled
+//               in TMEM only when the running max grows by more than 2^8), P written back as
+//               bf16 into the S columns of TMEM (tcgen05.st), epilogue (O / l -> bf16, staged
+//               through shared memory for 256-byte coalesced row stores; natural-log LSE);
+//   warp 8      producer: TMA (cp.async.bulk.tensor, SWIZZLE_128B) of K and V tiles from the
+//               head-major cache into 2-stage rings, plus the key-position table of partial tiles;
+//   warp 9      TMEM allocator (512 columns) and single-thread MMA issuer (warps 10-11 idle), kind::f16 bf16 x bf16
+//               -> fp32, M = 128:  S_h = Q_h K^T (SS, N = 128) into columns [128h, 128h + 128);
+//               O_h += P_h V (TS: P from TMEM, V the MN-major smem operand) into [256 + 128h, ..).
+//               Issue order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1), so each softmax
+//               group works while the tensor core runs the other group's two MMAs.
 // Q is read from global memory, rotated (3-D RoPE at the plan's query positions, fp32 math on
 // fp64-built tables) and written straight into the swizzled K-major layout the MMA reads: the
 // RoPE of Q is fused into the Q load.
+//
+// Ordering facts relied on: tcgen05.commit signals when every earlier tcgen05 operation of the
+// issuing thread has completed, so when softmax h sees S_h(j+1) complete, PV_h(j) (issued before
+// it) has completed too: O_h is stable for a rescale and P_h(j)'s columns may be overwritten.
+// tcgen05.mma operations of one thread execute in issue order, so S_h(j+1) (which overwrites the
+// TMEM columns holding P_h(j)) runs after PV_h(j) has read them.
 //
 // Every mbarrier wait is bounded (globaltimer): on expiry the thread raises the CTA abort flag
 // and the device status word (VDIT_ERR_TIMEOUT), every role leaves its loop, in-flight TMA and
@@ -41,10 +50,18 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kStages = 2;
-constexpr int kThreads = 256;
+constexpr int kQTiles = 2;                       // query tiles per CTA (one softmax group each)
+constexpr int kSoftmaxThreads = 128 * kQTiles;
+constexpr int kWarpTMA = 8, kWarpMMA = 9;     // warps 10-11 complete the third warpgroup
+constexpr int kThreads = 384;
+// Register split (setmaxnreg, per warpgroup): launched at 168 per thread (3 warps per SM
+// sub-partition, 16384 registers each); the two softmax groups grow to 216 and the producer /
+// MMA group shrinks to 72: 2 * 128 * 216 + 128 * 72 = 64512 = 384 * 168. (No call may sit
+// inside a setmaxnreg region: the bounded wait is inlined.)
+constexpr int kRegsSoftmax = 216, kRegsOther = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * 168, "register split");
 constexpr uint32_t kSlabBytes = kTile * 64 * 2;  // 16 KiB: 128 rows x 128 B (one swizzle width)
-constexpr uint32_t kPBytes = kTile * kTile * 2;  // P tile: 128 queries x 128 keys, bf16
-constexpr uint32_t kTmemCols = 256;              // S: columns [0,128), O: [128, 128 + D)
+constexpr uint32_t kTmemCols = 512;              // S0/P0, S1/P1, O0, O1: 128 columns each
 constexpr float kRescaleTau = 8.0f;              // rescale O only when the max grows by > 2^8
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -52,33 +69,32 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 enum {
     B_KFULL = 0, B_KEMPTY = B_KFULL + kStages, B_VFULL = B_KEMPTY + kStages,
     B_VEMPTY = B_VFULL + kStages, B_IFULL = B_VEMPTY + kStages, B_IEMPTY = B_IFULL + kStages,
-    B_SFULL = B_IEMPTY + kStages, B_SFREE, B_PFULL, B_ODONE, B_DRAIN, B_COUNT
+    B_SFULL = B_IEMPTY + kStages, B_PFULL = B_SFULL + kQTiles, B_ODONE = B_PFULL + kQTiles,
+    B_DRAIN = B_ODONE + kQTiles, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier area too small");
-constexpr uint32_t kKinfoBytes = 16 + kTile * 16;  // header (tile, full) + 128 x int4
+constexpr uint32_t kKinfoBytes = 16 + kTile * 16;  // header (tile, flags) + 128 x int4
 
 // Shared-memory map for head_dim D (offsets from a 1024-byte aligned base).
 template <int D>
 struct Layout {
     static constexpr int kSlabs = D / 64;
     static constexpr uint32_t kTileBytes = kTile * D * 2;  // one Q, K or V tile
-    static constexpr uint32_t OFF_Q = 0;
-    static constexpr uint32_t OFF_K = OFF_Q + kTileBytes;
+    static constexpr uint32_t OFF_Q = 0;                   // kQTiles tiles
+    static constexpr uint32_t OFF_K = OFF_Q + kQTiles * kTileBytes;
     static constexpr uint32_t OFF_V = OFF_K + kStages * kTileBytes;
-    static constexpr uint32_t OFF_P = OFF_V + kStages * kTileBytes;
-    static constexpr uint32_t OFF_BAR = OFF_P + kPBytes;
+    static constexpr uint32_t OFF_BAR = OFF_V + kStages * kTileBytes;
     static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 32;  // [0] tmem base, [1] abort flag
     static constexpr uint32_t OFF_KINFO = OFF_MISC + 64;
     static constexpr uint32_t OFF_RAD = OFF_KINFO + kStages * kKinfoBytes;
     static constexpr uint32_t kSmemBytes = OFF_RAD + (VDIT_MAX_DT + 1) * 4 + 1024;  // + align slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-    static_assert(kTile * D * 2 <= kPBytes, "O staging must fit in the P buffer");
 };
 
 struct AttnArgs {
-    const int* row_ptr;
-    const int* col_idx;
-    const unsigned char* full;
+    const int* u_row_ptr;  // per block of two q-tiles: union key-tile list
+    const int* u_col;
+    const unsigned char* u_flags;
     const int* slot_frame;
     const int* radius;
     const uint4* q;
@@ -130,7 +146,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Waits for the phase of `bar` with the given parity. Gives up (returns false) after
 // kWaitLimitNs, or as soon as another thread of the CTA has given up.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int* status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -270,6 +286,17 @@ __device__ __forceinline__ uint4 rope_chunk(uint4 in, int pp0, int t, int h, int
     return make_uint4(word[0], word[1], word[2], word[3]);
 }
 
+// O += A B with A read from TMEM (M = 128 lanes, 16-bit elements packed two per column).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // ------------------------------------------------------------------------------ the kernel
 
 template <int D>
@@ -278,24 +305,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
     using L = Layout<D>;
     constexpr uint32_t kTileBytes = L::kTileBytes;
-    constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, OFF_P = L::OFF_P;
-    constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC, OFF_KINFO = L::OFF_KINFO;
-    constexpr uint32_t OFF_RAD = L::OFF_RAD;
     constexpr int kC16 = D / 8;  // 16-byte chunks per head row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + OFF_BAR;
-    auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
-    int* rad_s = reinterpret_cast<int*>(smem + OFF_RAD);
+    auto BAR = [&](int i) { return sbase + L::OFF_BAR + 8u * (uint32_t)i; };
+    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    int* rad_s = reinterpret_cast<int*>(smem + L::OFF_RAD);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, head = blockIdx.y;
-    const int t_begin = __ldg(a.row_ptr + qt);
-    const int n_tiles = __ldg(a.row_ptr + qt + 1) - t_begin;
+    const int qb = blockIdx.x, head = blockIdx.y;
+    const int u_begin = __ldg(a.u_row_ptr + qb);
+    const int n_ent = __ldg(a.u_row_ptr + qb + 1) - u_begin;
     const int ft = a.grid_h * a.grid_w;
 
     if (threadIdx.x == 0) {
@@ -305,79 +328,235 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(B_VFULL + s), 1);
             mbar_init(BAR(B_VEMPTY + s), 1);
             mbar_init(BAR(B_IFULL + s), 1);
-            mbar_init(BAR(B_IEMPTY + s), 128);
+            mbar_init(BAR(B_IEMPTY + s), kSoftmaxThreads);
         }
-        mbar_init(BAR(B_SFULL), 1);
-        mbar_init(BAR(B_SFREE), 128);
-        mbar_init(BAR(B_PFULL), 128);
-        mbar_init(BAR(B_ODONE), 1);
+        for (int h = 0; h < kQTiles; ++h) {
+            mbar_init(BAR(B_SFULL + h), 1);
+            mbar_init(BAR(B_PFULL + h), 128);
+            mbar_init(BAR(B_ODONE + h), 1);
+        }
         mbar_init(BAR(B_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
+    if (warp == kWarpMMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         sbase + OFF_MISC),
+                         sbase + L::OFF_MISC),
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // radius table and the rotated Q tile (all 256 threads)
+    // radius table and the two rotated Q tiles (all threads)
     for (int i = threadIdx.x; i <= a.dt_max; i += kThreads) rad_s[i] = __ldg(a.radius + i);
-    {
-        const int q0 = qt * kTile;
-#pragma unroll 2
-        for (int i = 0; i < (kTile * kC16) / kThreads; ++i) {
-            const int idx = threadIdx.x + i * kThreads;
-            const int r = idx / kC16, c16 = idx % kC16;
-            const int qi = q0 + r;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (qi < a.q_tokens) {
-                const int f = qi / ft, rem = qi - f * ft;
-                const int hh = rem / a.grid_w, ww = rem - hh * a.grid_w;
-                const uint4 x = __ldg(a.q + ((size_t)qi * a.heads + head) * kC16 + c16);
-                v = rope_chunk(x, c16 * 4, a.q_start + f, hh, ww, a);
-            }
-            *reinterpret_cast<uint4*>(smem + OFF_Q + sw128_offset(r, c16)) = v;
+    for (int idx = threadIdx.x; idx < kQTiles * kTile * kC16; idx += kThreads) {
+        const int h = idx / (kTile * kC16), rem = idx - h * (kTile * kC16);
+        const int r = rem / kC16, c16 = rem - r * kC16;
+        const int qi = (qb * kQTiles + h) * kTile + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (qi < a.q_tokens) {
+            const int f = qi / ft, rm = qi - f * ft;
+            const int hh = rm / a.grid_w, ww = rm - hh * a.grid_w;
+            const uint4 x = __ldg(a.q + ((size_t)qi * a.heads + head) * kC16 + c16);
+            v = rope_chunk(x, c16 * 4, a.q_start + f, hh, ww, a);
         }
-        fence_proxy_async_smem();
+        *reinterpret_cast<uint4*>(smem + L::OFF_Q + h * kTileBytes + sw128_offset(r, c16)) = v;
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
 
-    if (warp == 0) {
+    if (warp < 4 * kQTiles) {
+        // ------------------------------------------------------------------ softmax (group h)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        const int h = warp >> 2;
+        const int row = threadIdx.x & 127;  // TMEM lane == query row within the tile
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + 128u * h + lane_base;
+        const uint32_t t_o = tmem + 256u + 128u * h + lane_base;
+        const uint32_t f_in = h ? 4u : 1u, f_full = h ? 8u : 2u;
+        const int qi = (qb * kQTiles + h) * kTile + row;
+        const int qf = qi / ft, qrem = qi - qf * ft;
+        const int tq = a.q_start + qf, hq = qrem / a.grid_w, wq = qrem - hq * a.grid_w;
+        const int cq = a.causal ? tq / a.chunk_frames : 0x7fffffff;
+        const float c = a.scale_log2;
+        float m = -INFINITY, l = 0.f;  // running max (raw score units) and sum
+        int cnt = 0;
+        bool ok = true;
+        for (int j = 0; j < n_ent; ++j) {
+            const int s = j % kStages;
+            if (!warp_wait(BAR(B_IFULL + s), (j / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+            const uint8_t* info = smem + L::OFF_KINFO + s * kKinfoBytes;
+            const uint32_t flags = (uint32_t)reinterpret_cast<const int*>(info)[1];
+            if (!(flags & f_in)) {
+                mbar_arrive(BAR(B_IEMPTY + s));
+                continue;
+            }
+            if (!warp_wait(BAR(B_SFULL + h), cnt & 1, abort_flag, a.status)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[128];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(t_s + q4 * 32, sr + q4 * 32);
+            tmem_ld_wait(sr);
+            reg_touch32(sr + 32);
+            reg_touch32(sr + 64);
+            reg_touch32(sr + 96);
+            float* sv = reinterpret_cast<float*>(sr);
+            if (!(flags & f_full)) {
+                const int4* ki = reinterpret_cast<const int4*>(info + 16);
+#pragma unroll
+                for (int jj = 0; jj < 128; ++jj) {
+                    const int4 e = ki[jj];
+                    int dt = abs(tq - e.x);
+                    dt = dt > a.dt_max ? a.dt_max : dt;
+                    const int cheb = max(abs(hq - e.y), abs(wq - e.z));
+                    const bool keep = (e.x >= 0) & (e.w <= cq) & (cheb <= rad_s[dt]);
+                    sv[jj] = keep ? sv[jj] : -INFINITY;
+                }
+            }
+            mbar_arrive(BAR(B_IEMPTY + s));
+            // row max with 8 independent chains
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+            for (int jj = 8; jj < 128; ++jj) mx[jj & 7] = fmaxf(mx[jj & 7], sv[jj]);
+            const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_new = fmaxf(m, m_tile);
+            const bool resc = (m_new - m) * c > kRescaleTau;
+            float alpha = 1.f;
+            if (resc) {
+                alpha = fast_exp2((m - m_new) * c);
+                m = m_new;
+            }
+            const float mc = (m == -INFINITY) ? 0.f : m * c;
+            // O_h is stable here: PV_h of the previous tile completed before S_h of this one
+            if (cnt > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                for (int q4 = 0; q4 < D / 32; ++q4) {
+                    uint32_t orow[32];
+                    tmem_ld32(t_o + q4 * 32, orow);
+                    tmem_ld_wait(orow);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                    tmem_st32(t_o + q4 * 32, orow);
+                }
+            }
+            // P = 2^(s*c - m*c) as bf16 pairs into the S columns [0, 64) of this lane
+            float rs[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rs[i] = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = fast_exp2(fmaf(sv[64 * half + 2 * i], c, -mc));
+                    const float p1 = fast_exp2(fmaf(sv[64 * half + 2 * i + 1], c, -mc));
+                    rs[i & 7] += p0 + p1;
+                    __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
+                    memcpy(&pk[i], &b, 4);
+                }
+                tmem_st32(t_s + 32 * half, pk);
+            }
+            tmem_st_wait();
+            l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+            tc_fence_before();
+            mbar_arrive(BAR(B_PFULL + h));
+            ++cnt;
+        }
+        if (ok && cnt > 0) {
+            if (!warp_wait(BAR(B_ODONE + h), 0, abort_flag, a.status)) ok = false;
+        }
+        // every thread of the group reaches this barrier (aborted or not); any failure skips
+        // the epilogue of the whole group
+        int any_fail;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t"
+            "setp.eq.u32 p, %1, 0;\n\t"
+            "bar.red.or.pred q, %2, 128, p;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(any_fail)
+            : "r"((uint32_t)ok), "r"(1 + h)
+            : "memory");
+        if (!any_fail) {
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            uint8_t* stage = smem + L::OFF_Q + h * kTileBytes;  // Q_h is no longer read
+#pragma unroll 1
+            for (int q4 = 0; q4 < D / 32; ++q4) {
+                uint32_t orow[32];
+                if (cnt > 0) {
+                    tmem_ld32(t_o + q4 * 32, orow);
+                    tmem_ld_wait(orow);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) orow[i] = 0u;
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t wds[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(
+                            __uint_as_float(orow[g * 8 + 2 * e]) * inv_l,
+                            __uint_as_float(orow[g * 8 + 2 * e + 1]) * inv_l);
+                        memcpy(&wds[e], &b, 4);
+                    }
+                    const int chunk = q4 * 4 + g;
+                    *reinterpret_cast<uint4*>(stage + row * (D * 2) + ((chunk ^ (row & 7)) << 4)) =
+                        make_uint4(wds[0], wds[1], wds[2], wds[3]);
+                }
+            }
+            if (a.lse && qi < a.q_tokens)
+                a.lse[(size_t)head * a.q_tokens + qi] =
+                    l > 0.f ? (m * c + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            asm volatile("bar.sync %0, 128;" ::"r"(3 + h) : "memory");
+            const int q0 = (qb * kQTiles + h) * kTile;
+#pragma unroll 4
+            for (int i = 0; i < kC16; ++i) {
+                const int r = i * (128 / kC16) + row / kC16, chunk = row % kC16;
+                if (q0 + r < a.q_tokens) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(stage + r * (D * 2) +
+                                                                    ((chunk ^ (r & 7)) << 4));
+                    __stcs(a.o + ((size_t)(q0 + r) * a.heads + head) * kC16 + chunk, v);
+                }
+            }
+        }
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    }
+    if (warp == kWarpTMA) {
         // ------------------------------------------------------------------ producer
         int issued = 0;
-        for (int it = 0; it < n_tiles; ++it) {
+        for (int it = 0; it < n_ent; ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) - 1) & 1u;
-            const int kt = __ldg(a.col_idx + t_begin + it);
-            const int full = __ldg(a.full + t_begin + it);
+            const int kt = __ldg(a.u_col + u_begin + it);
+            const int flags = __ldg(a.u_flags + u_begin + it);
             if (it >= kStages && !warp_wait(BAR(B_KEMPTY + s), ph, abort_flag, a.status)) break;
             if (lane == 0) {
                 mbar_expect_tx(BAR(B_KFULL + s), kTileBytes);
-                const uint32_t dst = sbase + OFF_K + s * kTileBytes;
+                const uint32_t dst = sbase + L::OFF_K + s * kTileBytes;
 #pragma unroll
                 for (int sl = 0; sl < L::kSlabs; ++sl)
                     tma_load_3d(dst + sl * kSlabBytes, &tmap_k, BAR(B_KFULL + s), 64 * sl, kt * kTile, head);
             }
-            // key positions of a partial tile (one int4 per key: frame, h, w, causal chunk)
-            if (it >= kStages && !warp_wait(BAR(B_IEMPTY + s), ph, abort_flag, a.status)) {
-                issued = it * 2 + 1;
-                break;
-            }
-            uint8_t* info = smem + OFF_KINFO + s * kKinfoBytes;
+            issued = it * 2 + 1;
+            if (it >= kStages && !warp_wait(BAR(B_IEMPTY + s), ph, abort_flag, a.status)) break;
+            uint8_t* info = smem + L::OFF_KINFO + s * kKinfoBytes;
             if (lane == 0) {
                 reinterpret_cast<int*>(info)[0] = kt;
-                reinterpret_cast<int*>(info)[1] = full;
+                reinterpret_cast<int*>(info)[1] = flags;
             }
-            if (!full) {
+            const bool partial = ((flags & 1) && !(flags & 2)) || ((flags & 4) && !(flags & 8));
+            if (partial) {
                 int4* ki = reinterpret_cast<int4*>(info + 16);
-                for (int j = lane; j < kTile; j += 32) {
-                    const int key = kt * kTile + j;
+                for (int jj = lane; jj < kTile; jj += 32) {
+                    const int key = kt * kTile + jj;
                     int4 e = make_int4(-1, 0, 0, 0x7fffffff);
                     if (key < a.kv_tokens) {
                         const int slot = key / ft, rem = key - slot * ft;
@@ -387,18 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       (tk >= 0 && a.causal) ? tk / a.chunk_frames : 0);
                         if (tk < 0) e.w = 0x7fffffff;
                     }
-                    ki[j] = e;
+                    ki[jj] = e;
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(B_IFULL + s));
-            if (it >= kStages && !warp_wait(BAR(B_VEMPTY + s), ph, abort_flag, a.status)) {
-                issued = it * 2 + 1;
-                break;
-            }
+            if (it >= kStages && !warp_wait(BAR(B_VEMPTY + s), ph, abort_flag, a.status)) break;
             if (lane == 0) {
                 mbar_expect_tx(BAR(B_VFULL + s), kTileBytes);
-                const uint32_t dst = sbase + OFF_V + s * kTileBytes;
+                const uint32_t dst = sbase + L::OFF_V + s * kTileBytes;
 #pragma unroll
                 for (int sl = 0; sl < L::kSlabs; ++sl)
                     tma_load_3d(dst + sl * kSlabBytes, &tmap_v, BAR(B_VFULL + s), 64 * sl, kt * kTile, head);
@@ -408,64 +584,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // drain: every TMA this warp issued must have landed before the CTA may exit
         if (*abort_flag) {
-            for (int j = (issued - 2 * kStages > 0 ? issued - 2 * kStages : 0); j < issued; ++j) {
-                const int it = j >> 1, s = it % kStages;
+            for (int jn = (issued - 2 * kStages > 0 ? issued - 2 * kStages : 0); jn < issued; ++jn) {
+                const int it = jn >> 1, s = it % kStages;
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                const int b = (j & 1) ? B_VFULL + s : B_KFULL + s;
-                // a landed load completes the phase; give up only on the time limit
+                const int b = (jn & 1) ? B_VFULL + s : B_KFULL + s;
                 const uint64_t t0 = globaltimer();
                 while (!mbar_try_wait(BAR(b), ph) && globaltimer() - t0 < kWaitLimitNs) {
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kWarpMMA) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0 && n_ent > 0) {
             constexpr uint32_t idesc_qk = instr_desc(kTile, 0), idesc_pv = instr_desc(D, 1);
-            const uint32_t q_addr = sbase + OFF_Q, p_addr = sbase + OFF_P;
-            auto issue_qk = [&](int s) {
-                const uint32_t k_addr = sbase + OFF_K + s * kTileBytes;
+            auto issue_s = [&](int h, int s) {
+                const uint32_t q_addr = sbase + L::OFF_Q + h * kTileBytes;
+                const uint32_t k_addr = sbase + L::OFF_K + s * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    tc_mma(tmem_s, smem_desc_sw128(q_addr + off, 16, 1024),
+                    tc_mma(tmem + 128u * h, smem_desc_sw128(q_addr + off, 16, 1024),
                            smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0);
                 }
+                tc_commit(BAR(B_SFULL + h));
             };
+            auto issue_pv = [&](int h, int s, bool acc) {
+                const uint32_t v_addr = sbase + L::OFF_V + s * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    tc_mma_ts(tmem + 256u + 128u * h, tmem + 128u * h + 8u * kk,
+                              smem_desc_sw128(v_addr + kk * 16 * 128, kSlabBytes, 1024), idesc_pv,
+                              (acc || kk > 0) ? 1u : 0u);
+            };
+            const unsigned char* fl = a.u_flags + u_begin;
             bool ok = wait_bounded(BAR(B_KFULL + 0), 0, abort_flag, a.status);
             if (ok) {
+                const int f0 = __ldg(fl);
                 tc_fence_after();
-                issue_qk(0);
-                tc_commit(BAR(B_SFULL));
+                if (f0 & 1) issue_s(0, 0);
+                if (f0 & 4) issue_s(1, 0);
                 tc_commit(BAR(B_KEMPTY + 0));
             }
-            for (int it = 0; ok && it < n_tiles; ++it) {
-                const int s = it % kStages;
-                if (it + 1 < n_tiles) {
-                    const int s1 = (it + 1) % kStages;
-                    if (!wait_bounded(BAR(B_KFULL + s1), ((it + 1) / kStages) & 1, abort_flag, a.status) ||
-                        !wait_bounded(BAR(B_SFREE), it & 1, abort_flag, a.status))
-                        break;
-                    tc_fence_after();
-                    issue_qk(s1);
-                    tc_commit(BAR(B_SFULL));
-                    tc_commit(BAR(B_KEMPTY + s1));
-                }
-                if (!wait_bounded(BAR(B_PFULL), it & 1, abort_flag, a.status) ||
-                    !wait_bounded(BAR(B_VFULL + s), (it / kStages) & 1, abort_flag, a.status))
-                    break;
-                tc_fence_after();
-                const uint32_t v_addr = sbase + OFF_V + s * kTileBytes;
+            int npv[2] = {0, 0};
+            for (int j = 0; ok && j < n_ent; ++j) {
+                const int s = j % kStages, s1 = (j + 1) % kStages;
+                const int f = __ldg(fl + j);
+                const int fn = j + 1 < n_ent ? __ldg(fl + j + 1) : 0;
+                if (!wait_bounded(BAR(B_VFULL + s), (j / kStages) & 1, abort_flag, a.status)) break;
+                bool k_ready = false;
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint32_t poff = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    tc_mma(tmem_o, smem_desc_sw128(p_addr + poff, 16, 1024),
-                           smem_desc_sw128(v_addr + kk * 16 * 128, kSlabBytes, 1024), idesc_pv,
-                           (it > 0 || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < kQTiles; ++h) {
+                    if (f & (h ? 4 : 1)) {
+                        if (!wait_bounded(BAR(B_PFULL + h), npv[h] & 1, abort_flag, a.status)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(h, s, npv[h] > 0);
+                        ++npv[h];
+                    }
+                    if (fn & (h ? 4 : 1)) {
+                        if (!k_ready) {
+                            if (!wait_bounded(BAR(B_KFULL + s1), ((j + 1) / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+                            tc_fence_after();
+                            k_ready = true;
+                        }
+                        issue_s(h, s1);
+                    }
                 }
-                tc_commit(BAR(B_ODONE));
+                if (!ok) break;
                 tc_commit(BAR(B_VEMPTY + s));
+                if (j + 1 < n_ent) tc_commit(BAR(B_KEMPTY + s1));
             }
+            for (int h = 0; h < kQTiles; ++h)
+                if (npv[h] > 0) tc_commit(BAR(B_ODONE + h));
         }
         if (lane == 0) {
             // drain: all MMAs issued by this thread complete before TMEM is released
@@ -475,161 +664,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------------ softmax
-        const int row = threadIdx.x - 128;  // TMEM lane == query row within the tile
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const int qi = qt * kTile + row;
-        const int qf = qi / ft, qrem = qi - qf * ft;
-        const int tq = a.q_start + qf, hq = qrem / a.grid_w, wq = qrem - (qrem / a.grid_w) * a.grid_w;
-        const int cq = a.causal ? tq / a.chunk_frames : 0x7fffffff;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int it = 0; it < n_tiles; ++it) {
-            const int s = it % kStages;
-            if (!warp_wait(BAR(B_SFULL), it & 1, abort_flag, a.status)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr + c * 32);
-            tmem_ld_wait(sr);
-            reg_touch32(sr + 32);
-            reg_touch32(sr + 64);
-            reg_touch32(sr + 96);
-            tc_fence_before();
-            mbar_arrive(BAR(B_SFREE));
-            float sv[128];
-#pragma unroll
-            for (int j = 0; j < 128; ++j) sv[j] = __uint_as_float(sr[j]) * a.scale_log2;
-
-            if (!warp_wait(BAR(B_IFULL + s), (it / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
-            const uint8_t* info = smem + OFF_KINFO + s * kKinfoBytes;
-            const int full = reinterpret_cast<const int*>(info)[1];
-            if (!full) {
-                const int4* ki = reinterpret_cast<const int4*>(info + 16);
-#pragma unroll
-                for (int j = 0; j < 128; ++j) {
-                    const int4 e = ki[j];
-                    int dt = abs(tq - e.x);
-                    dt = dt > a.dt_max ? a.dt_max : dt;
-                    const int cheb = max(abs(hq - e.y), abs(wq - e.z));
-                    const bool keep = (e.x >= 0) & (e.w <= cq) & (cheb <= rad_s[dt]);
-                    sv[j] = keep ? sv[j] : -INFINITY;
-                }
-            }
-            mbar_arrive(BAR(B_IEMPTY + s));
-
-            float mx = sv[0];
-#pragma unroll
-            for (int j = 1; j < 128; ++j) mx = fmaxf(mx, sv[j]);
-            const float m_new = fmaxf(m, mx);
-            const bool resc = m_new > m + kRescaleTau;
-            float alpha = 1.f;
-            if (resc) {
-                alpha = fast_exp2(m - m_new);
-                m = m_new;
-            }
-            const float m_use = (m == -INFINITY) ? 0.f : m;
-            float rs = 0.f;
-            uint32_t pk[64];
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float p0 = fast_exp2(sv[2 * j] - m_use), p1 = fast_exp2(sv[2 * j + 1] - m_use);
-                rs += p0 + p1;
-                __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-                memcpy(&pk[j], &b, 4);
-            }
-            l = l * alpha + rs;
-
-            // PV of the previous tile must be done before O is rescaled or P is overwritten
-            if (it > 0) {
-                if (!warp_wait(BAR(B_ODONE), (it - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t orow[32];
-                        tmem_ld32(tmem_o + lane_base + c * 32, orow);
-                        tmem_ld_wait(orow);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            orow[j] = __float_as_uint(__uint_as_float(orow[j]) * alpha);
-                        tmem_st32(tmem_o + lane_base + c * 32, orow);
-                    }
-                    tmem_st_wait();
-                }
-            }
-#pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16)
-                *reinterpret_cast<uint4*>(smem + OFF_P + sw128_offset(row, c16)) =
-                    make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(BAR(B_PFULL));
-        }
-        if (ok && n_tiles > 0) {
-            if (!warp_wait(BAR(B_ODONE), (n_tiles - 1) & 1, abort_flag, a.status)) ok = false;
-        }
-        // every softmax thread reaches this barrier (aborted or not); any failure skips the
-        // epilogue for the whole warpgroup
-        int any_fail;
-        asm volatile(
-            "{\n\t.reg .pred p, q;\n\t"
-            "setp.eq.u32 p, %1, 0;\n\t"
-            "bar.red.or.pred q, 1, 128, p;\n\t"
-            "selp.u32 %0, 1, 0, q;\n\t}"
-            : "=r"(any_fail)
-            : "r"((uint32_t)ok)
-            : "memory");
-        if (!any_fail) {
-            tc_fence_after();
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            uint8_t* stage = smem + OFF_P;  // P is no longer needed: stage O rows here
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t orow[32];
-                if (n_tiles > 0) {
-                    tmem_ld32(tmem_o + lane_base + c * 32, orow);
-                    tmem_ld_wait(orow);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) orow[j] = 0u;
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t wds[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(
-                            __uint_as_float(orow[q4 * 8 + 2 * e]) * inv_l,
-                            __uint_as_float(orow[q4 * 8 + 2 * e + 1]) * inv_l);
-                        memcpy(&wds[e], &b, 4);
-                    }
-                    const int chunk = c * 4 + q4;
-                    *reinterpret_cast<uint4*>(stage + row * (D * 2) + ((chunk ^ (row & 7)) << 4)) =
-                        make_uint4(wds[0], wds[1], wds[2], wds[3]);
-                }
-            }
-            if (a.lse && qi < a.q_tokens)
-                a.lse[(size_t)head * a.q_tokens + qi] =
-                    l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-            const int t = threadIdx.x - 128;
-#pragma unroll 4
-            for (int i = 0; i < kC16; ++i) {
-                const int r = i * (128 / kC16) + t / kC16, chunk = t % kC16;
-                const int qr = qt * kTile + r;
-                if (qr < a.q_tokens) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((chunk ^ (r & 7)) << 4));
-                    __stcs(a.o + ((size_t)qr * a.heads + head) * kC16 + chunk, v);
-                }
-            }
-        }
     }
     // ---------------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMMA) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(kTmemCols)
@@ -713,9 +752,9 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     if (!status) return fail(VDIT_ERR_CUDA, "cannot resolve status word");
 
     AttnArgs a{};
-    a.row_ptr = p->d_row_ptr;
-    a.col_idx = p->d_col_idx;
-    a.full = p->d_full;
+    a.u_row_ptr = p->d_u_row_ptr;
+    a.u_col = p->d_u_col;
+    a.u_flags = p->d_u_flags;
     a.slot_frame = p->d_slot_frame;
     a.radius = p->d_radius;
     a.q = static_cast<const uint4*>(q);
@@ -738,7 +777,7 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.chunk_frames = a.causal ? p->m.chunk_frames : 1;
     a.dt_max = p->dt_max;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    dim3 grid(p->n_qt, p->g.heads);
+    dim3 grid(p->n_qb, p->g.heads);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128)
         attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);

@@ -202,6 +202,24 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
         }
         p->row_ptr[qt + 1] = (int)p->col_idx.size();
     }
+    // union lists of q-tile pairs
+    p->n_qb = (p->n_qt + 1) / 2;
+    p->u_row_ptr.assign(p->n_qb + 1, 0);
+    for (int b = 0; b < p->n_qb; ++b) {
+        const int t0 = 2 * b, t1 = 2 * b + 1;
+        int i = p->row_ptr[t0], ie = p->row_ptr[t0 + 1];
+        int k = t1 < p->n_qt ? p->row_ptr[t1] : 0, ke = t1 < p->n_qt ? p->row_ptr[t1 + 1] : 0;
+        while (i < ie || k < ke) {
+            const int ci = i < ie ? p->col_idx[i] : INT_MAX, ck = k < ke ? p->col_idx[k] : INT_MAX;
+            const int c = std::min(ci, ck);
+            unsigned char f = 0;
+            if (ci == c) { f |= 1 | (p->full[i] ? 2 : 0); ++i; }
+            if (ck == c) { f |= 4 | (p->full[k] ? 8 : 0); ++k; }
+            p->u_col.push_back(c);
+            p->u_flags.push_back(f);
+        }
+        p->u_row_ptr[b + 1] = (int)p->u_col.size();
+    }
     // longest rows first: a persistent kernel that takes q-tiles in this order finishes its
     // longest work items early and fills the tail with short ones
     p->qtile_order.resize(p->n_qt);
@@ -247,13 +265,18 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
         if (p->device == dev) return VDIT_OK;
         return vdit::fail(VDIT_ERR_INVALID_ARG, "plan already uploaded to another device");
     }
-    // one allocation: row_ptr | qtile_order | slot_frame | radius | col_idx | full
+    // one allocation: row_ptr | qtile_order | slot_frame | radius | u_row_ptr | col_idx | full |
+    // u_col | u_flags
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     const size_t n_rp = sizeof(int) * p->row_ptr.size(), n_qo = sizeof(int) * p->qtile_order.size();
     const size_t n_sf = sizeof(int) * p->slot_frame.size(), n_ra = sizeof(int) * p->radius.size();
+    const size_t n_urp = sizeof(int) * p->u_row_ptr.size();
     const size_t n_ci = sizeof(int) * std::max<size_t>(1, p->col_idx.size());
     const size_t n_fu = std::max<size_t>(1, p->full.size());
-    const size_t total = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_ci) + up(n_fu);
+    const size_t n_uc = sizeof(int) * std::max<size_t>(1, p->u_col.size());
+    const size_t n_uf = std::max<size_t>(1, p->u_flags.size());
+    const size_t total = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_urp) + up(n_ci) +
+                         up(n_fu) + up(n_uc) + up(n_uf);
     std::vector<unsigned char> host(total, 0);
     size_t off = 0;
     auto put = [&](const void* src, size_t n) {
@@ -266,9 +289,16 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t o_qo = put(p->qtile_order.data(), n_qo);
     const size_t o_sf = put(p->slot_frame.data(), n_sf);
     const size_t o_ra = put(p->radius.data(), n_ra);
+    const size_t o_urp = put(p->u_row_ptr.data(), n_urp);
     const size_t o_ci = put(p->col_idx.data(), sizeof(int) * p->col_idx.size());
     off = o_ci + up(n_ci);
     const size_t o_fu = put(p->full.data(), p->full.size());
+    off = o_fu + up(n_fu);
+    const size_t o_uc = put(p->u_col.data(), sizeof(int) * p->u_col.size());
+    off = o_uc + up(n_uc);
+    const size_t o_uf = put(p->u_flags.data(), p->u_flags.size());
+    off = o_uf + up(n_uf);
+    if (off != total) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
     void* d = nullptr;
     if (int rc = cuda_check(cudaMalloc(&d, total), "cudaMalloc(plan)")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -287,7 +317,9 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     p->d_radius = reinterpret_cast<const int*>(b + o_ra);
     p->d_col_idx = reinterpret_cast<const int*>(b + o_ci);
     p->d_full = b + o_fu;
-    (void)o_fu;
+    p->d_u_row_ptr = reinterpret_cast<const int*>(b + o_urp);
+    p->d_u_col = reinterpret_cast<const int*>(b + o_uc);
+    p->d_u_flags = b + o_uf;
     return VDIT_OK;
 }
 
