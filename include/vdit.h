@@ -109,6 +109,8 @@ typedef struct vdit_plan_info_t {
     int full_tiles;      /* listed tiles that are complete and wholly kept */
     long long kept_pairs;/* kept (query, key) pairs per head */
     int uploaded;        /* 1 after vdit_plan_upload */
+    int kv_splits;       /* key-range pieces per (query block, head), set by vdit_plan_upload */
+    long long workspace_bytes; /* device scratch the plan holds for kv_splits > 1 */
 } vdit_plan_info_t;
 
 /* 3-D RoPE ([CRoPE] 2.B, [TR] Metodologia 1) of n_tokens consecutive tokens of one chunk whose
@@ -144,7 +146,12 @@ VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask
                    int capacity_frames, int kv_first_frame, int kv_last_frame);
 
 /* Copies the plan's schedule and tables to the current device (allocates; the copy is ordered on
- * stream). Idempotent. Required before vdit_attn_forward. */
+ * stream). Idempotent. Required before vdit_attn_forward. It also fixes the key-range split of
+ * the forward pass from the device's SM count: when the (query block, head) units alone would
+ * leave most of a wave of SMs idle, each unit's key tiles are cut into kv_splits pieces whose
+ * normalised fp32 partial outputs and log-sum-exps go to a scratch workspace held by the plan
+ * and are merged by a second kernel. Forward calls that share one plan must therefore not run
+ * concurrently on different streams. */
 VDIT_API int vdit_plan_upload(vdit_plan* p, void* stream);
 
 VDIT_API int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info);

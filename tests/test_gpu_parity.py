@@ -125,6 +125,14 @@ MEDIUM = {
     "causal_radial": _medium(3, 6, 3, 9, tuple((s, 3) for s in range(0, 9, 3))),
     "partial_fill": _medium(1, 3, 3, 12, ((0, 3), (3, 3))),
     "d64_radial": _medium(2, 0, 7, 7, ((0, 7),), d=64, wid=92, heads=3),
+    # 3-wide grid: a 128-key tile spans more than 32 row segments, so partial tiles take the
+    # per-key predicate path instead of the per-segment intervals
+    "narrow_grid_causal_radial": Workload(94, "narrow", grid_h=7, grid_w=3, heads=2, head_dim=128,
+                                          bands=(44, 42, 42), mask_kind=3, q_start=9, q_frames=6,
+                                          capacity_frames=16,
+                                          appends=tuple((s, 3) for s in range(0, 15, 3)),
+                                          kv_stream_first_frame=0, chunk_frames=3, w0=4,
+                                          gamma_shift=1, lam=4),
 }
 
 

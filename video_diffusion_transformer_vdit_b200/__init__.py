@@ -60,7 +60,8 @@ class _Mask(ctypes.Structure):
 class _PlanInfo(ctypes.Structure):
     _fields_ = [("q_tokens", ctypes.c_int), ("kv_tokens", ctypes.c_int), ("q_tiles", ctypes.c_int),
                 ("kv_tiles", ctypes.c_int), ("tiles", ctypes.c_int), ("full_tiles", ctypes.c_int),
-                ("kept_pairs", ctypes.c_longlong), ("uploaded", ctypes.c_int)]
+                ("kept_pairs", ctypes.c_longlong), ("uploaded", ctypes.c_int),
+                ("kv_splits", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong)]
 
 
 _lib = None

@@ -34,6 +34,7 @@
 // Every mbarrier wait is bounded (globaltimer): on expiry the thread raises the CTA abort flag
 // and the device status word (VDIT_ERR_TIMEOUT), every role leaves its loop, in-flight TMA and
 // MMA work is drained (again bounded) and TMEM is freed before the CTA exits.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -73,7 +74,12 @@ enum {
     B_DRAIN = B_ODONE + kQTiles, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier area too small");
-constexpr uint32_t kKinfoBytes = 16 + kTile * 16;  // header (tile, flags) + 128 x int4
+// Key-position table of a partial tile, one per K stage: a 16-byte header {tile, flags, nseg}
+// and either nseg row segments (nseg >= 0; consecutive keys of one frame slot and patch row,
+// int4 {k0 | len << 8 | h << 16, frame, causal chunk, first w}) or, when the tile holds more
+// than kMaxSeg segments (very narrow grids), one int4 {frame, h, w, chunk} per key (nseg = -1).
+constexpr int kMaxSeg = 32;
+constexpr uint32_t kKinfoBytes = 16 + kTile * 16;
 
 // Shared-memory map for head_dim D (offsets from a 1024-byte aligned base).
 template <int D>
@@ -95,6 +101,10 @@ struct AttnArgs {
     const int* u_row_ptr;  // per block of two q-tiles: union key-tile list
     const int* u_col;
     const unsigned char* u_flags;
+    const int* unit_order; // q-blocks, longest list first
+    float* ws_o;           // split > 1: normalised partial O [split][q_tokens][heads][D]
+    float* ws_lse;         // split > 1: partial log2-sum-exp [split][heads][q_tokens]
+    int n_qb, n_split;
     const int* slot_frame;
     const int* radius;
     const uint4* q;
@@ -316,9 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* rad_s = reinterpret_cast<int*>(smem + L::OFF_RAD);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = blockIdx.x, head = blockIdx.y;
-    const int u_begin = __ldg(a.u_row_ptr + qb);
-    const int n_ent = __ldg(a.u_row_ptr + qb + 1) - u_begin;
+    // work unit: q-block (longest lists first), head, and the piece `sp` of its key tiles
+    const int sp = blockIdx.x / a.n_qb, head = blockIdx.y;
+    const int qb = __ldg(a.unit_order + (blockIdx.x - sp * a.n_qb));
+    const int u_first = __ldg(a.u_row_ptr + qb);
+    const int n_all = __ldg(a.u_row_ptr + qb + 1) - u_first;
+    const int e0 = (int)((long long)n_all * sp / a.n_split);
+    const int u_begin = u_first + e0;
+    const int n_ent = (int)((long long)n_all * (sp + 1) / a.n_split) - e0;
     const int ft = a.grid_h * a.grid_w;
 
     if (threadIdx.x == 0) {
@@ -404,16 +419,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             reg_touch32(sr + 96);
             float* sv = reinterpret_cast<float*>(sr);
             if (!(flags & f_full)) {
+                const int nseg = reinterpret_cast<const int*>(info)[2];
                 const int4* ki = reinterpret_cast<const int4*>(info + 16);
+                uint32_t mw[4] = {0u, 0u, 0u, 0u};  // keep bit per key of the tile
+                if (nseg >= 0) {
+                    // kept keys of this row: one contiguous run per segment
+                    for (int sg = 0; sg < nseg; ++sg) {
+                        const int4 e = ki[sg];
+                        const int k0 = e.x & 0xff, len = (e.x >> 8) & 0xff, hk = e.x >> 16;
+                        if (e.y < 0 || e.z > cq) continue;
+                        const int dt = min(abs(tq - e.y), a.dt_max);
+                        const int r = min(rad_s[dt], 1 << 20);
+                        if (abs(hq - hk) > r) continue;
+                        const int lo = max(e.w, wq - r) - e.w + k0;
+                        const int hi = min(e.w + len - 1, wq + r) - e.w + k0;
 #pragma unroll
-                for (int jj = 0; jj < 128; ++jj) {
-                    const int4 e = ki[jj];
-                    int dt = abs(tq - e.x);
-                    dt = dt > a.dt_max ? a.dt_max : dt;
-                    const int cheb = max(abs(hq - e.y), abs(wq - e.z));
-                    const bool keep = (e.x >= 0) & (e.w <= cq) & (cheb <= rad_s[dt]);
-                    sv[jj] = keep ? sv[jj] : -INFINITY;
+                        for (int wd = 0; wd < 4; ++wd) {
+                            const int a0 = max(lo - 32 * wd, 0), b0 = min(hi - 32 * wd, 31);
+                            if (a0 <= b0) mw[wd] |= (0xffffffffu >> (31 - b0)) & (0xffffffffu << a0);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int wd = 0; wd < 4; ++wd) {
+                        uint32_t m = 0u;
+#pragma unroll 1
+                        for (int b = 0; b < 32; ++b) {
+                            const int4 e = ki[32 * wd + b];
+                            const int dt = min(abs(tq - e.x), a.dt_max);
+                            const int cheb = max(abs(hq - e.y), abs(wq - e.z));
+                            const bool keep = (e.x >= 0) & (e.w <= cq) & (cheb <= rad_s[dt]);
+                            m |= (uint32_t)keep << b;
+                        }
+                        mw[wd] = m;
+                    }
                 }
+#pragma unroll
+                for (int jj = 0; jj < 128; ++jj)
+                    sv[jj] = ((mw[jj >> 5] >> (jj & 31)) & 1u) ? sv[jj] : -INFINITY;
             }
             mbar_arrive(BAR(B_IEMPTY + s));
             // row max with 8 independent chains
@@ -482,7 +525,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             : "=r"(any_fail)
             : "r"((uint32_t)ok), "r"(1 + h)
             : "memory");
-        if (!any_fail) {
+        if (!any_fail && a.n_split > 1) {
+            // partial result of this key piece: O / l in fp32 and log2(sum) for the merge
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            float4* dst = reinterpret_cast<float4*>(
+                a.ws_o + (((size_t)sp * a.q_tokens + (qi < a.q_tokens ? qi : 0)) * a.heads + head) * D);
+#pragma unroll 1
+            for (int q4 = 0; q4 < D / 32; ++q4) {
+                uint32_t orow[32];
+                if (cnt > 0) {
+                    tmem_ld32(t_o + q4 * 32, orow);
+                    tmem_ld_wait(orow);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) orow[i] = 0u;
+                }
+                if (qi < a.q_tokens) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        dst[q4 * 8 + g] = make_float4(__uint_as_float(orow[4 * g]) * inv_l,
+                                                      __uint_as_float(orow[4 * g + 1]) * inv_l,
+                                                      __uint_as_float(orow[4 * g + 2]) * inv_l,
+                                                      __uint_as_float(orow[4 * g + 3]) * inv_l);
+                }
+            }
+            if (qi < a.q_tokens)
+                a.ws_lse[((size_t)sp * a.heads + head) * a.q_tokens + qi] =
+                    l > 0.f ? m * c + log2f(l) : -INFINITY;
+        } else if (!any_fail) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             uint8_t* stage = smem + L::OFF_Q + h * kTileBytes;  // Q_h is no longer read
@@ -555,18 +626,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool partial = ((flags & 1) && !(flags & 2)) || ((flags & 4) && !(flags & 8));
             if (partial) {
                 int4* ki = reinterpret_cast<int4*>(info + 16);
-                for (int jj = lane; jj < kTile; jj += 32) {
-                    const int key = kt * kTile + jj;
-                    int4 e = make_int4(-1, 0, 0, 0x7fffffff);
-                    if (key < a.kv_tokens) {
+                // row segments of the tile (lane 0 walks them; a 30 x 52 grid gives at most 4)
+                int nseg = 0;
+                if (lane == 0) {
+                    int k = 0;
+                    const int key0 = kt * kTile;
+                    while (k < kTile && key0 + k < a.kv_tokens) {
+                        if (nseg == kMaxSeg) { nseg = -1; break; }
+                        const int key = key0 + k;
                         const int slot = key / ft, rem = key - slot * ft;
-                        const int hh = rem / a.grid_w;
+                        const int hh = rem / a.grid_w, ww = rem - hh * a.grid_w;
+                        const int len = min(min(a.grid_w - ww, kTile - k), a.kv_tokens - key);
                         const int tk = __ldg(a.slot_frame + slot);
-                        e = make_int4(tk, hh, rem - hh * a.grid_w,
-                                      (tk >= 0 && a.causal) ? tk / a.chunk_frames : 0);
-                        if (tk < 0) e.w = 0x7fffffff;
+                        const int ch = tk < 0 ? 0x7fffffff : (a.causal ? tk / a.chunk_frames : 0);
+                        ki[nseg++] = make_int4(k | (len << 8) | (hh << 16), tk, ch, ww);
+                        k += len;
                     }
-                    ki[jj] = e;
+                    reinterpret_cast<int*>(info)[2] = nseg;
+                }
+                nseg = __shfl_sync(0xffffffffu, nseg, 0);
+                if (nseg < 0) {
+                    for (int jj = lane; jj < kTile; jj += 32) {
+                        const int key = kt * kTile + jj;
+                        int4 e = make_int4(-1, 0, 0, 0x7fffffff);
+                        if (key < a.kv_tokens) {
+                            const int slot = key / ft, rem = key - slot * ft;
+                            const int hh = rem / a.grid_w;
+                            const int tk = __ldg(a.slot_frame + slot);
+                            e = make_int4(tk, hh, rem - hh * a.grid_w,
+                                          (tk >= 0 && a.causal) ? tk / a.chunk_frames : 0);
+                            if (tk < 0) e.w = 0x7fffffff;
+                        }
+                        ki[jj] = e;
+                    }
                 }
             }
             __syncwarp();
@@ -676,6 +768,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Merge of the key pieces of every (query, head) row: with piece i holding O_i = (sum over its
+// keys of p v) / l_i and L_i = log2 l_i (in the shared log2 units of the scaled scores),
+//   L = log2 sum_i 2^L_i,   o = sum_i 2^(L_i - L) O_i,   lse = L ln 2.
+// One warp per row; each lane owns D / 32 consecutive channels.
+template <int D>
+__global__ void __launch_bounds__(256) split_combine_kernel(const float* __restrict__ ws_o,
+                                                            const float* __restrict__ ws_lse,
+                                                            int n_split, int q_tokens, int heads,
+                                                            __nv_bfloat16* __restrict__ o,
+                                                            float* __restrict__ lse) {
+    constexpr int kPer = D / 32;
+    const long long rows = (long long)q_tokens * heads;
+    const long long n_warps = (long long)gridDim.x * (blockDim.x / 32);
+    const int lane = threadIdx.x & 31;
+    for (long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; row < rows;
+         row += n_warps) {
+        const int qi = (int)(row / heads), hd = (int)(row - (long long)qi * heads);
+        float lmax = -INFINITY;
+        for (int i = 0; i < n_split; ++i)
+            lmax = fmaxf(lmax, __ldg(ws_lse + ((size_t)i * heads + hd) * q_tokens + qi));
+        float acc[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+        float wsum = 0.f;
+        if (lmax != -INFINITY) {
+            for (int i = 0; i < n_split; ++i) {
+                const float li = __ldg(ws_lse + ((size_t)i * heads + hd) * q_tokens + qi);
+                const float w = exp2f(li - lmax);
+                wsum += w;
+                const float* src = ws_o + (((size_t)i * q_tokens + qi) * heads + hd) * D + lane * kPer;
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, __ldg(src + e), acc[e]);
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        __nv_bfloat16* dst = o + ((size_t)qi * heads + hd) * D + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; e += 2)
+            *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+        if (lse && lane == 0)
+            lse[(size_t)hd * q_tokens + qi] =
+                wsum > 0.f ? (lmax + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+    }
+}
+
 __device__ int g_status = 0;
 
 // ------------------------------------------------------------------------------ host side
@@ -755,6 +892,11 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.u_row_ptr = p->d_u_row_ptr;
     a.u_col = p->d_u_col;
     a.u_flags = p->d_u_flags;
+    a.unit_order = p->d_unit_order;
+    a.ws_o = p->d_ws_o;
+    a.ws_lse = p->d_ws_lse;
+    a.n_qb = p->n_qb;
+    a.n_split = p->n_split;
     a.slot_frame = p->d_slot_frame;
     a.radius = p->d_radius;
     a.q = static_cast<const uint4*>(q);
@@ -777,12 +919,27 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.chunk_frames = a.causal ? p->m.chunk_frames : 1;
     a.dt_max = p->dt_max;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    dim3 grid(p->n_qb, p->g.heads);
+    dim3 grid(p->n_qb * p->n_split, p->g.heads);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128)
         attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
     else
         attn_fwd_kernel<64><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
+    if (p->n_split > 1) {
+        if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
+        int sms = 148;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long rows = (long long)p->q_tokens * p->g.heads;
+        const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)sms * 8);
+        auto* ob = static_cast<__nv_bfloat16*>(o);
+        if (d == 128)
+            split_combine_kernel<128><<<blocks, 256, 0, st>>>(p->d_ws_o, p->d_ws_lse, p->n_split,
+                                                              p->q_tokens, p->g.heads, ob, lse);
+        else
+            split_combine_kernel<64><<<blocks, 256, 0, st>>>(p->d_ws_o, p->d_ws_lse, p->n_split,
+                                                             p->q_tokens, p->g.heads, ob, lse);
+        return vdit::cuda_check(cudaGetLastError(), "split merge launch");
+    }
     return vdit::cuda_check(cudaGetLastError(), "attention kernel launch");
 }
 

@@ -50,6 +50,10 @@ struct vdit_plan {
     int n_qb = 0;
     std::vector<int> u_row_ptr, u_col;
     std::vector<unsigned char> u_flags;
+    std::vector<int> unit_order;  // q-blocks by descending union-list length (longest first)
+    // key-range split of every (q-block, head) unit, chosen at upload from the SM count so the
+    // number of CTAs fills whole waves; > 1 uses the fp32 partial workspace below
+    int n_split = 1;
     // device copy
     int device = -1;
     void* d_buf = nullptr;
@@ -62,4 +66,8 @@ struct vdit_plan {
     const int* d_u_row_ptr = nullptr;
     const int* d_u_col = nullptr;
     const unsigned char* d_u_flags = nullptr;
+    const int* d_unit_order = nullptr;
+    float* d_ws_o = nullptr;    // [n_split][q_tokens][heads][head_dim] normalised partial O
+    float* d_ws_lse = nullptr;  // [n_split][heads][q_tokens] partial log2-sum-exp
+    size_t ws_bytes = 0;
 };

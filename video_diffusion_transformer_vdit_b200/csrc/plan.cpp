@@ -220,6 +220,11 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
         }
         p->u_row_ptr[b + 1] = (int)p->u_col.size();
     }
+    p->unit_order.resize(p->n_qb);
+    for (int i = 0; i < p->n_qb; ++i) p->unit_order[i] = i;
+    std::stable_sort(p->unit_order.begin(), p->unit_order.end(), [&](int a, int b) {
+        return p->u_row_ptr[a + 1] - p->u_row_ptr[a] > p->u_row_ptr[b + 1] - p->u_row_ptr[b];
+    });
     // longest rows first: a persistent kernel that takes q-tiles in this order finishes its
     // longest work items early and fills the tail with short ones
     p->qtile_order.resize(p->n_qt);
@@ -241,6 +246,8 @@ extern "C" int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info) {
     info->full_tiles = p->n_full;
     info->kept_pairs = p->kept_pairs;
     info->uploaded = p->d_buf != nullptr;
+    info->kv_splits = p->n_split;
+    info->workspace_bytes = (long long)p->ws_bytes;
     return VDIT_OK;
 }
 
@@ -265,8 +272,25 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
         if (p->device == dev) return VDIT_OK;
         return vdit::fail(VDIT_ERR_INVALID_ARG, "plan already uploaded to another device");
     }
+    // key-range split: the smallest split count (<= 8, >= 8 key tiles per piece) whose CTA count
+    // fills at least 90% of whole waves, else the best one found
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int max_len = 0;
+    for (int b = 0; b < p->n_qb; ++b) max_len = std::max(max_len, p->u_row_ptr[b + 1] - p->u_row_ptr[b]);
+    const long long units = (long long)p->n_qb * p->g.heads;
+    int best = 1;
+    double best_eff = 0.0;
+    for (int sp = 1; sp <= 8; ++sp) {
+        if (sp > 1 && max_len / sp < 8) break;
+        const long long ctas = units * sp;
+        const double eff = (double)ctas / (double)(((ctas + sms - 1) / sms) * sms);
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = sp; }
+        if (eff >= 0.9) break;
+    }
+    p->n_split = best;
     // one allocation: row_ptr | qtile_order | slot_frame | radius | u_row_ptr | col_idx | full |
-    // u_col | u_flags
+    // u_col | u_flags | unit_order | (split workspace: partial O | partial lse)
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     const size_t n_rp = sizeof(int) * p->row_ptr.size(), n_qo = sizeof(int) * p->qtile_order.size();
     const size_t n_sf = sizeof(int) * p->slot_frame.size(), n_ra = sizeof(int) * p->radius.size();
@@ -275,8 +299,13 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t n_fu = std::max<size_t>(1, p->full.size());
     const size_t n_uc = sizeof(int) * std::max<size_t>(1, p->u_col.size());
     const size_t n_uf = std::max<size_t>(1, p->u_flags.size());
-    const size_t total = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_urp) + up(n_ci) +
-                         up(n_fu) + up(n_uc) + up(n_uf);
+    const size_t n_uo = sizeof(int) * std::max<size_t>(1, p->unit_order.size());
+    const size_t n_wo = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
+                                             p->g.heads * p->g.head_dim : 0;
+    const size_t n_wl = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads * p->q_tokens : 0;
+    const size_t meta = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_urp) + up(n_ci) +
+                        up(n_fu) + up(n_uc) + up(n_uf) + up(n_uo);
+    const size_t total = meta + up(n_wo) + up(n_wl);
     std::vector<unsigned char> host(total, 0);
     size_t off = 0;
     auto put = [&](const void* src, size_t n) {
@@ -298,11 +327,14 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     off = o_uc + up(n_uc);
     const size_t o_uf = put(p->u_flags.data(), p->u_flags.size());
     off = o_uf + up(n_uf);
-    if (off != total) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
+    const size_t o_uo = put(p->unit_order.data(), sizeof(int) * p->unit_order.size());
+    off = o_uo + up(n_uo);
+    if (off != meta) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
+    host.resize(meta);  // the workspace is not initialised: every entry is written before use
     void* d = nullptr;
     if (int rc = cuda_check(cudaMalloc(&d, total), "cudaMalloc(plan)")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (int rc = cuda_check(cudaMemcpyAsync(d, host.data(), total, cudaMemcpyHostToDevice, s),
+    if (int rc = cuda_check(cudaMemcpyAsync(d, host.data(), meta, cudaMemcpyHostToDevice, s),
                             "cudaMemcpyAsync(plan)")) {
         cudaFree(d);
         return rc;
@@ -320,6 +352,12 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     p->d_u_row_ptr = reinterpret_cast<const int*>(b + o_urp);
     p->d_u_col = reinterpret_cast<const int*>(b + o_uc);
     p->d_u_flags = b + o_uf;
+    p->d_unit_order = reinterpret_cast<const int*>(b + o_uo);
+    p->ws_bytes = n_wo + n_wl;
+    if (p->n_split > 1) {
+        p->d_ws_o = reinterpret_cast<float*>(b + meta);
+        p->d_ws_lse = reinterpret_cast<float*>(b + meta + up(n_wo));
+    }
     return VDIT_OK;
 }
 
