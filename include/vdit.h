@@ -171,6 +171,28 @@ VDIT_API void vdit_plan_destroy(vdit_plan* p);
 VDIT_API int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
                       void* o, float* lse, float scale, void* stream);
 
+/* Attention forward that allocates nothing. No passage of the source pages has a counterpart:
+ * this is a service for callers that cannot allocate device memory when they run attention,
+ * for instance code running while another framework owns the GPU's memory through its own
+ * pool (a cudaMalloc would fail or fragment it), or latency-critical loops that must not enter
+ * the allocator or synchronise the device. Same arguments, results and error codes as
+ * vdit_attn_forward; the difference is where the key-split scratch lives: instead of the
+ * workspace that vdit_plan_upload gives the plan, the partial results go to one fixed 32 MiB
+ * device buffer that is part of the library (every GPU that loads the library holds it until
+ * the process exits). A plan whose split needs more than 32 MiB
+ * (kv_splits x q_tokens x heads x (head_dim + 1) x 4 bytes) is rejected with
+ * VDIT_ERR_UNSUPPORTED and a message giving both sizes; plans with kv_splits == 1 need none.
+ * The call itself makes no cudaMalloc / cudaFree or other allocating call: the plan must already
+ * be uploaded, and the RoPE tables for its bands must already exist on the device (any earlier
+ * vdit_kv_append, vdit_rope3d_apply or vdit_attn_forward builds them; otherwise
+ * VDIT_ERR_INVALID_ARG). The first call on each device looks up the buffer's device address
+ * (cudaGetSymbolAddress), so make that first call before any stream capture. All calls share
+ * the buffer and it keeps the last call's contents (nothing in it needs to start at zero): calls
+ * whose kernels may overlap on the GPU, e.g. on two streams of one device, race on it. */
+VDIT_API int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, const void* k_cache,
+                                       const void* v_cache, void* o, float* lse, float scale,
+                                       void* stream);
+
 /* Reads and clears the current device's kernel status word: *status = VDIT_OK, or
  * VDIT_ERR_TIMEOUT when a bounded wait in a kernel gave up since the last read. Synchronises the
  * device. */

@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_destroy.argtypes = [P]
         L.vdit_plan_destroy.restype = None
         L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
+        L.vdit_attn_forward_noalloc.argtypes = [P, P, P, P, P, P, F, P]
         L.vdit_get_status.argtypes = [ctypes.POINTER(I)]
         L.vdit_last_error.restype = ctypes.c_char_p
         _lib = L

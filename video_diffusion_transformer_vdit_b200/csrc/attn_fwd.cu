@@ -39,6 +39,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <string>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -952,5 +953,154 @@ extern "C" int vdit_get_status(int* status) {
     if (int rc = vdit::cuda_check(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)), "clear status"))
         return rc;
     *status = v;
+    return VDIT_OK;
+}
+
+// ------------------------------------------------------------------------------ no-allocation
+// variant of the forward pass
+//
+// Some callers cannot call cudaMalloc at the moment they run attention: code that runs while
+// another framework owns the device's memory through its own pool (a cudaMalloc there fails or
+// fragments that pool), latency-critical loops that must not touch the allocator, and code that
+// must not synchronise the device. vdit_attn_forward takes its key-split scratch from the plan
+// (allocated by vdit_plan_upload); this variant instead writes the partial results into the
+// fixed buffer below, so the call itself allocates nothing.
+//
+// The buffer is a file-scope device array: every GPU that loads this library holds its
+// kNoAllocScratchBytes until the process exits, whether or not the variant is used. In host code
+// its name is only a host-side stand-in, so its device address is resolved with
+// cudaGetSymbolAddress once per device (with that device current) on the variant's first call
+// there; that first call should therefore come before any stream capture. All calls share the
+// buffer and it keeps the last call's contents: every partial entry a call reads is written by
+// the same call first, so nothing has to start at zero, but two calls whose kernels overlap on
+// the GPU (different streams, same device) race on it.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 256;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch_address(int dev, void** out) {
+    if (dev < 0 || dev >= kMaxDevices) return vdit::fail(VDIT_ERR_INVALID_ARG, "device index too large");
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&ptr, g_noalloc_scratch),
+                                      "cudaGetSymbolAddress(no-alloc scratch)"))
+            return rc;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return VDIT_OK;
+}
+}  // namespace
+
+extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, const void* k_cache,
+                                         const void* v_cache, void* o, float* lse, float scale,
+                                         void* stream) {
+    using vdit::fail;
+    if (!p) return fail(VDIT_ERR_INVALID_ARG, "NULL plan");
+    if (!p->d_buf) return fail(VDIT_ERR_NOT_UPLOADED, "plan not uploaded (vdit_plan_upload)");
+    if (!q || !k_cache || !v_cache || !o) return fail(VDIT_ERR_INVALID_ARG, "NULL tensor");
+    auto al = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
+    if (!al(q) || !al(k_cache) || !al(v_cache) || !al(o) || (reinterpret_cast<uintptr_t>(lse) & 3))
+        return fail(VDIT_ERR_MISALIGNED, "tensor not aligned");
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(VDIT_ERR_INVALID_ARG, "scale must be > 0");
+    int dev = 0;
+    if (int rc = vdit::cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    if (dev != p->device) return fail(VDIT_ERR_INVALID_ARG, "plan was uploaded to another device");
+    // scratch this plan's key split needs: partial O [split][q][heads][d] fp32, then partial
+    // log2-sum-exp [split][heads][q] fp32 at the next 256-byte boundary
+    const int d = p->g.head_dim;
+    const size_t o_bytes = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
+                                                p->g.heads * d : 0;
+    const size_t o_bytes_al = (o_bytes + 255) / 256 * 256;
+    const size_t l_bytes = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads *
+                                                p->q_tokens : 0;
+    if (o_bytes_al + l_bytes > kNoAllocScratchBytes)
+        return fail(VDIT_ERR_UNSUPPORTED,
+                    "this plan's key split needs " + std::to_string(o_bytes_al + l_bytes) +
+                        " bytes of scratch; the no-allocation variant's static buffer holds " +
+                        std::to_string(kNoAllocScratchBytes) + " (use vdit_attn_forward)");
+    void* scratch = nullptr;
+    if (int rc = noalloc_scratch_address(dev, &scratch)) return rc;
+    vdit::RopeTables tabs;
+    if (int rc = vdit::find_rope_tables(&p->g, &tabs)) return rc;
+    CUtensorMap mk, mv;
+    if (int rc = make_cache_map(&mk, k_cache, p->kv_tokens, p->g.heads, d)) return rc;
+    if (int rc = make_cache_map(&mv, v_cache, p->kv_tokens, p->g.heads, d)) return rc;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(attn_fwd_kernel<128>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Layout<128>::kSmemBytes);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(attn_fwd_kernel<64>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)Layout<64>::kSmemBytes);
+    });
+    if (int rc = vdit::cuda_check(attr_err, "cudaFuncSetAttribute")) return rc;
+    int* status = status_ptr();
+    if (!status) return fail(VDIT_ERR_CUDA, "cannot resolve status word");
+
+    float* ws_o = p->n_split > 1 ? static_cast<float*>(scratch) : nullptr;
+    float* ws_lse = p->n_split > 1
+                        ? reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + o_bytes_al)
+                        : nullptr;
+    AttnArgs a{};
+    a.u_row_ptr = p->d_u_row_ptr;
+    a.u_col = p->d_u_col;
+    a.u_flags = p->d_u_flags;
+    a.unit_order = p->d_unit_order;
+    a.ws_o = ws_o;
+    a.ws_lse = ws_lse;
+    a.n_qb = p->n_qb;
+    a.n_split = p->n_split;
+    a.slot_frame = p->d_slot_frame;
+    a.radius = p->d_radius;
+    a.q = static_cast<const uint4*>(q);
+    a.o = static_cast<uint4*>(o);
+    a.lse = lse;
+    a.tt = static_cast<const float2*>(tabs.t);
+    a.th = static_cast<const float2*>(tabs.h);
+    a.tw = static_cast<const float2*>(tabs.w);
+    a.status = status;
+    a.bt2 = p->g.band_t / 2;
+    a.bh2 = p->g.band_h / 2;
+    a.bw2 = p->g.band_w / 2;
+    a.q_tokens = p->q_tokens;
+    a.kv_tokens = p->kv_tokens;
+    a.heads = p->g.heads;
+    a.grid_h = p->g.grid_h;
+    a.grid_w = p->g.grid_w;
+    a.q_start = p->q_start;
+    a.causal = (p->m.kind & VDIT_MASK_BLOCK_CAUSAL) ? 1 : 0;
+    a.chunk_frames = a.causal ? p->m.chunk_frames : 1;
+    a.dt_max = p->dt_max;
+    a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    dim3 grid(p->n_qb * p->n_split, p->g.heads);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
+    else
+        attn_fwd_kernel<64><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
+    if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
+    if (p->n_split > 1) {
+        int sms = 148;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long rows = (long long)p->q_tokens * p->g.heads;
+        const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)sms * 8);
+        auto* ob = static_cast<__nv_bfloat16*>(o);
+        if (d == 128)
+            split_combine_kernel<128><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
+                                                              p->g.heads, ob, lse);
+        else
+            split_combine_kernel<64><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
+                                                             p->g.heads, ob, lse);
+        return vdit::cuda_check(cudaGetLastError(), "split merge launch");
+    }
     return VDIT_OK;
 }

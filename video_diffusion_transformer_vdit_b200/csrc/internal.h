@@ -27,6 +27,8 @@ struct RopeTables {
     const void* w;
 };
 int get_rope_tables(const vdit_geom* g, RopeTables* out);
+// Same tables, lookup only (never allocates); an error if they were never built on this device.
+int find_rope_tables(const vdit_geom* g, RopeTables* out);
 
 }  // namespace vdit
 

@@ -77,6 +77,24 @@ int get_rope_tables(const vdit_geom* g, RopeTables* out) {
     return VDIT_OK;
 }
 
+// Looks the tables up without building them: for callers that must not allocate. Fails if no
+// earlier call on this device built them for this band set.
+int find_rope_tables(const vdit_geom* g, RopeTables* out) {
+    int dev = 0;
+    if (int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    uint64_t tbits;
+    std::memcpy(&tbits, &g->theta, sizeof tbits);
+    auto key = std::make_tuple(dev, g->band_t, g->band_h, g->band_w, tbits);
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    auto it = g_tabs.find(key);
+    if (it == g_tabs.end())
+        return fail(VDIT_ERR_INVALID_ARG,
+                    "RoPE tables for these bands do not exist on this device yet; an earlier "
+                    "vdit_kv_append, vdit_rope3d_apply or vdit_attn_forward call builds them");
+    *out = it->second;
+    return VDIT_OK;
+}
+
 }  // namespace vdit
 
 namespace {
