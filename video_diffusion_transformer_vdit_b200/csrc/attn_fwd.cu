@@ -65,6 +65,15 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * 168, "regi
 constexpr uint32_t kSlabBytes = kTile * 64 * 2;  // 16 KiB: 128 rows x 128 B (one swizzle width)
 constexpr uint32_t kTmemCols = 512;              // S0/P0, S1/P1, O0, O1: 128 columns each
 constexpr float kRescaleTau = 8.0f;              // rescale O only when the max grows by > 2^8
+// Which of every 8 consecutive P pairs of a row take the FMA-pipe exp2 instead of the MUFU unit
+// (bit i set: pair i mod 8). Measured on the dense 32,760-token workload: none 1073, two of
+// eight 1028, three of eight 997 TFLOP/s, so by default every exponential uses MUFU; the
+// software path stays available for other shapes (it passed the GPU parity tests with 0x88
+// and 0xA8).
+#ifndef VDIT_POLY_PAIRS
+#define VDIT_POLY_PAIRS 0x00u
+#endif
+constexpr uint32_t kPolyPairs = VDIT_POLY_PAIRS;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // barrier indices (8 bytes each)
@@ -249,6 +258,62 @@ __device__ __forceinline__ void reg_touch32(uint32_t* r) {
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// Packed fp32 pair arithmetic (one instruction for two lanes of data).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x on the FMA pipe, for x <= 2^22 (x = -inf gives exactly 0). Cody-Waite range reduction
+// (Cody and Waite, "Software Manual for the Elementary Functions", 1980): x = n + f with
+// n = round(x) and |f| <= 1/2, so 2^x = 2^n * 2^f; 2^f comes from a cubic 1 + c1 f + c2 f^2 +
+// c3 f^3 fitted here for minimal relative error on [-1/2, 1/2] (weighted least squares with
+// Lawson reweighting in float64, coefficients rounded to float32; maximum relative error 1.0e-4
+// in float32 Horner form, far below the 2^-9 of the bf16 P it feeds). n is read from the low
+// mantissa bits of x + 1.5 * 2^23 and added to the exponent field. Inputs below -127 are clamped
+// to -127: there f = 0 and the cubic is exactly 1 (its constant term is pinned to 1 for this),
+// so the assembly gives exactly +0 for masked scores.
+constexpr float kExp2C0 = 1.0f, kExp2C1 = 0.6932829022407532f, kExp2C2 = 0.2422109693288803f,
+                kExp2C3 = 0.05500892922282219f;
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+    float x0, x1;
+    unpack2(x2, x0, x1);
+    x0 = fmaxf(x0, -127.f);
+    x1 = fmaxf(x1, -127.f);
+    const uint64_t xc = pack2(x0, x1);
+    const uint64_t t = add2(xc, pack2(12582912.f, 12582912.f));
+    const uint64_t r = add2(t, pack2(-12582912.f, -12582912.f));
+    const uint64_t f = fma2(r, pack2(-1.f, -1.f), xc);
+    uint64_t q = fma2(pack2(kExp2C3, kExp2C3), f, pack2(kExp2C2, kExp2C2));
+    q = fma2(q, f, pack2(kExp2C1, kExp2C1));
+    q = fma2(q, f, pack2(kExp2C0, kExp2C0));
+    float t0, t1, q0, q1;
+    unpack2(t, t0, t1);
+    unpack2(q, q0, q1);
+    const int n0 = __float_as_int(t0) - 0x4B400000, n1 = __float_as_int(t1) - 0x4B400000;
+    return pack2(__int_as_float(__float_as_int(q0) + (n0 << 23)),
+                 __int_as_float(__float_as_int(q1) + (n1 << 23)));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -460,14 +525,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sv[jj] = ((mw[jj >> 5] >> (jj & 31)) & 1u) ? sv[jj] : -INFINITY;
             }
             mbar_arrive(BAR(B_IEMPTY + s));
-            // row max with 8 independent chains
-            float mx[8];
+            // row max: 4 independent chains of 3-input max
+            float mx[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+            for (int i = 0; i < 4; ++i) mx[i] = sv[i];
 #pragma unroll
-            for (int jj = 8; jj < 128; ++jj) mx[jj & 7] = fmaxf(mx[jj & 7], sv[jj]);
-            const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int jj = 4; jj < 128; jj += 8) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) mx[i] = max3(mx[i], sv[jj + 2 * i], sv[jj + 2 * i + 1]);
+            }
+            const float m_tile = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
             const float m_new = fmaxf(m, m_tile);
             const bool resc = (m_new - m) * c > kRescaleTau;
             float alpha = 1.f;
@@ -489,25 +556,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st32(t_o + q4 * 32, orow);
                 }
             }
-            // P = 2^(s*c - m*c) as bf16 pairs into the S columns [0, 64) of this lane
-            float rs[8];
+            // P = 2^(s*c - m*c) as bf16 pairs into the S columns [0, 64) of this lane; the pairs
+            // selected by kPolyPairs take the FMA-pipe exp2 so the MUFU pipe is not the bound
+            uint64_t rs2[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) rs[i] = 0.f;
+            for (int i = 0; i < 4; ++i) rs2[i] = pack2(0.f, 0.f);
+            const uint64_t c2 = pack2(c, c), nmc2 = pack2(-mc, -mc);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = fast_exp2(fmaf(sv[64 * half + 2 * i], c, -mc));
-                    const float p1 = fast_exp2(fmaf(sv[64 * half + 2 * i + 1], c, -mc));
-                    rs[i & 7] += p0 + p1;
+                    const uint64_t x2 =
+                        fma2(pack2(sv[64 * half + 2 * i], sv[64 * half + 2 * i + 1]), c2, nmc2);
+                    uint64_t p2;
+                    if (kPolyPairs & (1u << (i & 7))) {
+                        p2 = exp2_fma2(x2);
+                    } else {
+                        float x0, x1;
+                        unpack2(x2, x0, x1);
+                        p2 = pack2(fast_exp2(x0), fast_exp2(x1));
+                    }
+                    rs2[i & 3] = add2(rs2[i & 3], p2);
+                    float p0, p1;
+                    unpack2(p2, p0, p1);
                     __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
                     memcpy(&pk[i], &b, 4);
                 }
                 tmem_st32(t_s + 32 * half, pk);
             }
+            float rsum;
+            {
+                const uint64_t a01 = add2(rs2[0], rs2[1]), a23 = add2(rs2[2], rs2[3]);
+                float u0, u1;
+                unpack2(add2(a01, a23), u0, u1);
+                rsum = u0 + u1;
+            }
             tmem_st_wait();
-            l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+            l = l * alpha + rsum;
             tc_fence_before();
             mbar_arrive(BAR(B_PFULL + h));
             ++cnt;
