@@ -57,10 +57,10 @@ constexpr int kSoftmaxThreads = 128 * kQTiles;
 constexpr int kWarpTMA = 8, kWarpMMA = 9;     // warps 10-11 complete the third warpgroup
 constexpr int kThreads = 384;
 // Register split (setmaxnreg, per warpgroup): launched at 168 per thread (3 warps per SM
-// sub-partition, 16384 registers each); the two softmax groups grow to 216 and the producer /
-// MMA group shrinks to 72: 2 * 128 * 216 + 128 * 72 = 64512 = 384 * 168. (No call may sit
+// sub-partition, 16384 registers each); the two softmax groups grow to 208 and the producer /
+// MMA group shrinks to 88: 2 * 128 * 208 + 128 * 88 = 64512 = 384 * 168. (No call may sit
 // inside a setmaxnreg region: the bounded wait is inlined.)
-constexpr int kRegsSoftmax = 216, kRegsOther = 72;
+constexpr int kRegsSoftmax = 208, kRegsOther = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * 168, "register split");
 constexpr uint32_t kSlabBytes = kTile * 64 * 2;  // 16 KiB: 128 rows x 128 B (one swizzle width)
 constexpr uint32_t kTmemCols = 512;              // S0/P0, S1/P1, O0, O1: 128 columns each
@@ -400,6 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int e0 = (int)((long long)n_all * sp / a.n_split);
     const int u_begin = u_first + e0;
     const int n_ent = (int)((long long)n_all * (sp + 1) / a.n_split) - e0;
+    // Every CTA walks its key tiles starting at a different position (the online softmax does
+    // not depend on the order): CTAs of one head run concurrently, and starting them all at the
+    // same tile makes them request the same 32 KiB of K / V from the same L2 slices at once.
+    const int rot = n_ent > 0 ? (int)(((unsigned)blockIdx.x * 97u + (unsigned)blockIdx.y * 31u) % (unsigned)n_ent) : 0;
+    auto entry = [&](int i) { const int e = i + rot; return e >= n_ent ? e - n_ent : e; };
     const int ft = a.grid_h * a.grid_w;
 
     if (threadIdx.x == 0) {
@@ -525,16 +530,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sv[jj] = ((mw[jj >> 5] >> (jj & 31)) & 1u) ? sv[jj] : -INFINITY;
             }
             mbar_arrive(BAR(B_IEMPTY + s));
-            // row max: 4 independent chains of 3-input max
-            float mx[4];
+            // row max: 8 independent chains of 3-input max
+            float mx[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) mx[i] = sv[i];
+            for (int i = 0; i < 8; ++i) mx[i] = sv[i];
 #pragma unroll
-            for (int jj = 4; jj < 128; jj += 8) {
+            for (int jj = 8; jj < 128; jj += 16) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) mx[i] = max3(mx[i], sv[jj + 2 * i], sv[jj + 2 * i + 1]);
+                for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], sv[jj + 2 * i], sv[jj + 2 * i + 1]);
             }
-            const float m_tile = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+            const float m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
+                                      fmaxf(mx[6], mx[7]));
             const float m_new = fmaxf(m, m_tile);
             const bool resc = (m_new - m) * c > kRescaleTau;
             float alpha = 1.f;
@@ -690,11 +696,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpTMA) {
         // ------------------------------------------------------------------ producer
         int issued = 0;
+        int kt_next = n_ent > 0 ? __ldg(a.u_col + u_begin + entry(0)) : 0;
+        int fl_next = n_ent > 0 ? __ldg(a.u_flags + u_begin + entry(0)) : 0;
         for (int it = 0; it < n_ent; ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) - 1) & 1u;
-            const int kt = __ldg(a.u_col + u_begin + it);
-            const int flags = __ldg(a.u_flags + u_begin + it);
+            const int kt = kt_next, flags = fl_next;
+            if (it + 1 < n_ent) {  // next entry's tile and flags, loaded while this one waits
+                kt_next = __ldg(a.u_col + u_begin + entry(it + 1));
+                fl_next = __ldg(a.u_flags + u_begin + entry(it + 1));
+            }
             if (it >= kStages && !warp_wait(BAR(B_KEMPTY + s), ph, abort_flag, a.status)) break;
             if (lane == 0) {
                 mbar_expect_tx(BAR(B_KFULL + s), kTileBytes);
@@ -776,39 +787,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0 && n_ent > 0) {
             constexpr uint32_t idesc_qk = instr_desc(kTile, 0), idesc_pv = instr_desc(D, 1);
+            // Descriptors are built once; each MMA only adds a compile-time offset (in 16-byte
+            // units) to a loop-invariant base, which keeps the single issuing thread at the
+            // tensor core's rate (a descriptor rebuilt from runtime indices per MMA was measured
+            // to cost more issue time than the 64-cycle M=128 N=128 K=16 MMA itself).
+            const uint64_t dq0 = smem_desc_sw128(sbase + L::OFF_Q, 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(sbase + L::OFF_K, 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(sbase + L::OFF_V, kSlabBytes, 1024);
+            constexpr uint64_t kTileDesc = kTileBytes >> 4;  // one tile further, in descriptor units
             auto issue_s = [&](int h, int s) {
-                const uint32_t q_addr = sbase + L::OFF_Q + h * kTileBytes;
-                const uint32_t k_addr = sbase + L::OFF_K + s * kTileBytes;
+                const uint64_t q0 = dq0 + (h ? kTileDesc : 0), k0 = dk0 + (s ? kTileDesc : 0);
+                const uint32_t d_t = h ? tmem + 128u : tmem;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    tc_mma(tmem + 128u * h, smem_desc_sw128(q_addr + off, 16, 1024),
-                           smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0);
+                    const uint64_t off = (uint64_t)((((kk >> 2) * kSlabBytes) + (kk & 3) * 32) >> 4);
+                    tc_mma(d_t, q0 + off, k0 + off, idesc_qk, kk > 0);
                 }
                 tc_commit(BAR(B_SFULL + h));
             };
             auto issue_pv = [&](int h, int s, bool acc) {
-                const uint32_t v_addr = sbase + L::OFF_V + s * kTileBytes;
+                const uint64_t v0 = dv0 + (s ? kTileDesc : 0);
+                const uint32_t d_t = h ? tmem + 384u : tmem + 256u;
+                const uint32_t a_t = h ? tmem + 128u : tmem;
+                const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    tc_mma_ts(tmem + 256u + 128u * h, tmem + 128u * h + 8u * kk,
-                              smem_desc_sw128(v_addr + kk * 16 * 128, kSlabBytes, 1024), idesc_pv,
-                              (acc || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(d_t, a_t + 8u * kk, v0 + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                              kk > 0 ? 1u : acc0);
             };
             const unsigned char* fl = a.u_flags + u_begin;
+            // tile flags are read three entries ahead so the global-load latency never sits
+            // between a completed barrier and the next MMA issue
+            int f_cur = __ldg(fl + entry(0));
+            int f_nxt = n_ent > 1 ? __ldg(fl + entry(1)) : 0;
+            int f_nn = n_ent > 2 ? __ldg(fl + entry(2)) : 0;
             bool ok = wait_bounded(BAR(B_KFULL + 0), 0, abort_flag, a.status);
             if (ok) {
-                const int f0 = __ldg(fl);
                 tc_fence_after();
-                if (f0 & 1) issue_s(0, 0);
-                if (f0 & 4) issue_s(1, 0);
+                if (f_cur & 1) issue_s(0, 0);
+                if (f_cur & 4) issue_s(1, 0);
                 tc_commit(BAR(B_KEMPTY + 0));
             }
             int npv[2] = {0, 0};
             for (int j = 0; ok && j < n_ent; ++j) {
                 const int s = j % kStages, s1 = (j + 1) % kStages;
-                const int f = __ldg(fl + j);
-                const int fn = j + 1 < n_ent ? __ldg(fl + j + 1) : 0;
+                const int f = f_cur, fn = f_nxt;
+                const int f3 = j + 3 < n_ent ? __ldg(fl + entry(j + 3)) : 0;
+                f_cur = f_nxt;
+                f_nxt = f_nn;
+                f_nn = f3;
                 if (!wait_bounded(BAR(B_VFULL + s), (j / kStages) & 1, abort_flag, a.status)) break;
                 bool k_ready = false;
 #pragma unroll
