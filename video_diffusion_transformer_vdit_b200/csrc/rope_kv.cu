@@ -7,12 +7,12 @@
 // past chunks. "Timeripple" (Metodologia 1) splits the channels into a temporal group and two
 // spatial groups.
 //
-// Both kernels are HBM streams: every (token, head) row is 16-byte-vector read once and written
-// once; a warp owns a run of consecutive tokens, so the token's (t, h, w) is advanced
-// incrementally instead of divided out per element, and the 32 lanes sweep the token's
-// heads x head_dim/8 16-byte chunks (fully coalesced). Each 32-bit word of a chunk is one RoPE
+// Both kernels are HBM streams: every 16-byte chunk of [tokens, heads, head_dim] is read once and
+// written once, consecutive threads on consecutive chunks, several independent loads in flight
+// per thread (the kernels are latency-bound otherwise). Each 32-bit word of a chunk is one RoPE
 // pair (channel 2j in the low half, 2j+1 in the high half), rotated in fp32 with a (cos, sin)
 // pair read from the tables (L1/L2 resident) and rounded to bf16 nearest-even.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -99,18 +99,35 @@ int find_rope_tables(const vdit_geom* g, RopeTables* out) {
 
 namespace {
 
+// Division by a run-time constant d via a 64-bit reciprocal: q = mulhi(n, ceil(2^64 / d)), exact
+// whenever n * d < 2^64 (all index math here stays far below that).
+struct FastDiv {
+    unsigned long long m;  // ceil(2^64 / d); unused when d == 1
+    unsigned long long d;
+};
+FastDiv make_fastdiv(unsigned long long d) {
+    FastDiv f;
+    f.d = d;
+    f.m = d <= 1 ? 0ull : (~0ull / d) + 1ull;
+    return f;
+}
+__device__ __forceinline__ unsigned long long fdiv(unsigned long long n, const FastDiv& f) {
+    return f.d == 1 ? n : __umul64hi(n, f.m);
+}
+
 struct StreamArgs {
     const uint4* x;     // rope: input; append: K chunk
     uint4* y;           // rope: output; append: K cache
     const uint4* v;     // append: V chunk
     uint4* vc;          // append: V cache
-    long long n_tokens;
+    unsigned long long total;  // 16-byte chunks to process = n_tokens * cpt
     int cpr_log2;       // log2(head_dim / 8): 16-byte chunks per head row
     int cpt;            // chunks per token = heads * head_dim / 8
     int grid_h, grid_w;
     int start_frame;
     int cap_frames;     // append: ring capacity in frames
     long long cap_tok;  // append: capacity_frames * grid_h * grid_w
+    FastDiv by_cpt, by_ft, by_w, by_cap;
     const float2* tt;
     const float2* th;
     const float2* tw;
@@ -142,63 +159,54 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 in, int pp0, int t, int h, i
     return make_uint4(word[0], word[1], word[2], word[3]);
 }
 
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 4;        // independent 16-byte loads per thread in flight
+constexpr int kBlocksPerSM = 4;   // 256 threads x 4 = 1024 resident threads, <= 64 registers each
 
-// APPEND = false: y[tok] = RoPE(x[tok]).  APPEND = true: K' = RoPE(k) and V go to the ring slot.
+// Flattened stream over the 16-byte chunks of [tokens, heads, head_dim]: consecutive threads take
+// consecutive chunks (fully coalesced 512-byte warp accesses), each thread first issues kUnroll
+// independent loads strided by the grid size, then decodes each chunk's (token, head, pair, t, h, w)
+// by reciprocal multiplication and rotates it.
+// APPEND = false: y[chunk] = RoPE(x[chunk]).
+// APPEND = true:  K' = RoPE(k) and V (unchanged) go to frame slot t mod capacity of the caches.
 template <bool APPEND>
-__global__ void __launch_bounds__(256) rope_stream_kernel(StreamArgs a) {
-    const long long warps = (long long)gridDim.x * (blockDim.x / 32);
-    const long long gw = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-    const int lane = threadIdx.x & 31;
-    const long long per = (a.n_tokens + warps - 1) / warps;
-    long long tok = gw * per;
-    const long long end = tok + per < a.n_tokens ? tok + per : a.n_tokens;
-    if (tok >= end) return;
-    const int ft = a.grid_h * a.grid_w;
-    int f = (int)(tok / ft);
-    int rem = (int)(tok - (long long)f * ft);
-    int h = rem / a.grid_w, w = rem - h * a.grid_w;
+__global__ void __launch_bounds__(256, kBlocksPerSM) rope_stream_kernel(StreamArgs a) {
+    const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
     const int cpr_mask = (1 << a.cpr_log2) - 1;
-    for (; tok < end; ++tok) {
-        const int t = a.start_frame + f;
-        const long long src0 = tok * a.cpt;
-        long long dst_tok = 0;
-        if (APPEND) dst_tok = (long long)(t % a.cap_frames) * ft + rem;
-        for (int k0 = 0; k0 < a.cpt; k0 += 32 * kUnroll) {
-            uint4 xin[kUnroll], vin[kUnroll];
+    const int ft = a.grid_h * a.grid_w;
+    for (unsigned long long i0 = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x;
+         i0 < a.total; i0 += stride * kUnroll) {
+        uint4 xin[kUnroll], vin[kUnroll];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int k = k0 + u * 32 + lane;
-                if (k < a.cpt) {
-                    xin[u] = __ldcs(a.x + src0 + k);
-                    if (APPEND) vin[u] = __ldcs(a.v + src0 + k);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int k = k0 + u * 32 + lane;
-                if (k < a.cpt) {
-                    const int c8 = k & cpr_mask;
-                    const uint4 r = rotate_chunk(xin[u], c8 * 4, t, h, w, a);
-                    if (APPEND) {
-                        const int head = k >> a.cpr_log2;
-                        const long long d = (((long long)head * a.cap_tok + dst_tok) << a.cpr_log2) + c8;
-                        __stcs(a.y + d, r);
-                        __stcs(a.vc + d, vin[u]);
-                    } else {
-                        __stcs(a.y + src0 + k, r);
-                    }
-                }
+        for (int u = 0; u < kUnroll; ++u) {
+            const unsigned long long idx = i0 + u * stride;
+            if (idx < a.total) {
+                xin[u] = __ldcs(a.x + idx);
+                if (APPEND) vin[u] = __ldcs(a.v + idx);
             }
         }
-        // advance (f, h, w) to the next token
-        ++rem;
-        if (++w == a.grid_w) {
-            w = 0;
-            if (++h == a.grid_h) {
-                h = 0;
-                rem = 0;
-                ++f;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const unsigned long long idx = i0 + u * stride;
+            if (idx < a.total) {
+                const unsigned long long tok = fdiv(idx, a.by_cpt);
+                const int k = (int)(idx - tok * (unsigned long long)a.cpt);
+                const int c8 = k & cpr_mask;
+                const unsigned long long f = fdiv(tok, a.by_ft);
+                const int rem = (int)(tok - f * (unsigned long long)ft);
+                const int h = (int)fdiv((unsigned long long)rem, a.by_w);
+                const int w = rem - h * a.grid_w;
+                const int t = a.start_frame + (int)f;
+                const uint4 r = rotate_chunk(xin[u], c8 * 4, t, h, w, a);
+                if (APPEND) {
+                    const int slot = t - (int)fdiv((unsigned long long)t, a.by_cap) * a.cap_frames;
+                    const int head = k >> a.cpr_log2;
+                    const long long d =
+                        (((long long)head * a.cap_tok + (long long)slot * ft + rem) << a.cpr_log2) + c8;
+                    __stcs(a.y + d, r);
+                    __stcs(a.vc + d, vin[u]);
+                } else {
+                    __stcs(a.y + idx, r);
+                }
             }
         }
     }
@@ -208,9 +216,10 @@ int launch_stream(bool append, StreamArgs& a, cudaStream_t s) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long max_warps = (long long)sms * 64;  // 8 blocks x 8 warps per SM resident
-    long long warps = a.n_tokens < max_warps ? a.n_tokens : max_warps;
-    const int blocks = (int)((warps + 7) / 8);
+    const unsigned long long per_block = 256ull * kUnroll;
+    const unsigned long long want = (a.total + per_block - 1) / per_block;
+    const int blocks = (int)std::min<unsigned long long>(want, (unsigned long long)sms * kBlocksPerSM);
+    if (blocks == 0) return VDIT_OK;
     if (append)
         rope_stream_kernel<true><<<blocks, 256, 0, s>>>(a);
     else
@@ -233,6 +242,10 @@ int fill_common(const vdit_geom* g, StreamArgs& a) {
     a.cpt = g->heads * (g->head_dim / 8);
     a.grid_h = g->grid_h;
     a.grid_w = g->grid_w;
+    a.by_cpt = make_fastdiv((unsigned long long)a.cpt);
+    a.by_ft = make_fastdiv((unsigned long long)g->grid_h * g->grid_w);
+    a.by_w = make_fastdiv((unsigned long long)g->grid_w);
+    a.by_cap = make_fastdiv(1);
     return VDIT_OK;
 }
 
@@ -259,7 +272,7 @@ extern "C" int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int
     if (int rc = fill_common(g, a)) return rc;
     a.x = static_cast<const uint4*>(x);
     a.y = static_cast<uint4*>(y);
-    a.n_tokens = n_tokens;
+    a.total = (unsigned long long)n_tokens * a.cpt;
     a.start_frame = start_frame;
     return launch_stream(false, a, static_cast<cudaStream_t>(stream));
 }
@@ -294,9 +307,10 @@ extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
     a.v = static_cast<const uint4*>(v);
     a.y = static_cast<uint4*>(k_cache);
     a.vc = static_cast<uint4*>(v_cache);
-    a.n_tokens = ft * n_frames;
+    a.total = (unsigned long long)(ft * n_frames) * a.cpt;
     a.start_frame = start_frame;
     a.cap_frames = capacity_frames;
     a.cap_tok = ft * capacity_frames;
+    a.by_cap = make_fastdiv((unsigned long long)capacity_frames);
     return launch_stream(true, a, static_cast<cudaStream_t>(stream));
 }
