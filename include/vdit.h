@@ -198,6 +198,13 @@ VDIT_API int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, const 
  * device. */
 VDIT_API int vdit_get_status(int* status);
 
+/* Test hook for failure detection (no counterpart in the pages): while on != 0, the K/V producer
+ * of every vdit_attn_forward launch issues no load, so the kernel's bounded waits expire (after
+ * about 2 s), each CTA raises VDIT_ERR_TIMEOUT in the status word, drains and frees its tensor
+ * memory and exits; the output is left unwritten and the CUDA context stays usable. Not for use
+ * outside tests. */
+VDIT_API void vdit_debug_skip_loads(int on);
+
 /* Message of the last failed call on this thread ("" if none). Valid until the next call. */
 VDIT_API const char* vdit_last_error(void);
 

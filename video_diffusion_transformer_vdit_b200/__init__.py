@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
         L.vdit_attn_forward_noalloc.argtypes = [P, P, P, P, P, P, F, P]
         L.vdit_get_status.argtypes = [ctypes.POINTER(I)]
+        L.vdit_debug_skip_loads.argtypes = [I]
+        L.vdit_debug_skip_loads.restype = None
         L.vdit_last_error.restype = ctypes.c_char_p
         _lib = L
     return _lib

@@ -35,6 +35,7 @@
 // and the device status word (VDIT_ERR_TIMEOUT), every role leaves its loop, in-flight TMA and
 // MMA work is drained (again bounded) and TMEM is freed before the CTA exits.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -124,6 +125,7 @@ struct AttnArgs {
     const float2* th;
     const float2* tw;
     int* status;
+    int skip_loads;        // test hook: the producer issues nothing, so every wait runs out
     int bt2, bh2, bw2;
     int q_tokens, kv_tokens, heads;
     int grid_h, grid_w;
@@ -698,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int issued = 0;
         int kt_next = n_ent > 0 ? __ldg(a.u_col + u_begin + entry(0)) : 0;
         int fl_next = n_ent > 0 ? __ldg(a.u_flags + u_begin + entry(0)) : 0;
-        for (int it = 0; it < n_ent; ++it) {
+        for (int it = 0; it < (a.skip_loads ? 0 : n_ent); ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) - 1) & 1u;
             const int kt = kt_next, flags = fl_next;
@@ -928,6 +930,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const float* __restr
 }
 
 __device__ int g_status = 0;
+std::atomic<int> g_skip_loads{0};
 
 // ------------------------------------------------------------------------------ host side
 
@@ -1020,6 +1023,7 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.th = static_cast<const float2*>(tabs.h);
     a.tw = static_cast<const float2*>(tabs.w);
     a.status = status;
+    a.skip_loads = g_skip_loads.load(std::memory_order_relaxed);
     a.bt2 = p->g.band_t / 2;
     a.bh2 = p->g.band_h / 2;
     a.bw2 = p->g.band_w / 2;
@@ -1056,6 +1060,8 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     }
     return vdit::cuda_check(cudaGetLastError(), "attention kernel launch");
 }
+
+extern "C" void vdit_debug_skip_loads(int on) { g_skip_loads.store(on ? 1 : 0); }
 
 extern "C" int vdit_get_status(int* status) {
     if (!status) return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL status");
