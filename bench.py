@@ -52,6 +52,25 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over the process group (the one collective of the bench: the
+    timing reduction). World size 1 needs no process group."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank does flops_per_rank per step (weak scaling), the step
+    time is the slowest rank's."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def config_of(w, extra=None):
     c = {"workload": w.name, "frames_x_grid": f"{w.q_frames}x{w.grid_h}x{w.grid_w}",
          "q_tokens": w.q_tokens, "kv_tokens": w.kv_tokens, "heads": w.heads,
@@ -64,63 +83,80 @@ def config_of(w, extra=None):
 
 # ------------------------------------------------------------------------------ oracle arm
 
-def oracle_sample(w, budget_s: float = 10.0, pilot_rows: int = 16):
-    """Times the oracle on a bounded sample of the workload: the KV appends of one step for all
-    heads, then masked attention for a sample of query rows (all heads). Returns (TFLOP/s in the
-    metric's units, seconds, sample description)."""
-    import oracle
+class OracleArm:
+    """The fp64 CPU oracle as a benchmark arm. Setup (not timed): the seeded inputs and the
+    fp64 KV cache filled by the oracle's own appends. A timed sample: RoPE of a random set of
+    query rows, their explicit mask rows, and two-pass masked attention of those rows for all
+    heads against every key slot. Throughput counts 4*d FLOP per kept pair of the sample."""
 
-    og = oracle.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, *w.bands, w.theta)
-    om = oracle.Mask(block_causal=bool(w.mask_kind & 1), radial=bool(w.mask_kind & 2),
-                     chunk_frames=w.chunk_frames, w0=w.w0, gamma_shift=w.gamma_shift, lam=w.lam)
-    ft = w.frame_tokens
-    n_kv = w.kv_stream_frames * ft
-    k = synth.bf16_bits_to_f64(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "k"))
-    v = synth.bf16_bits_to_f64(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "v"))
-    first, last = w.window()
-    kpos, kvalid = oracle.cache_positions(w.capacity_frames, first, last, w.grid_h, w.grid_w)
-    qpos_all = oracle.positions(w.q_tokens, w.grid_h, w.grid_w, w.q_start)
-    qbits = synth.qkv_bf16(w.id, w.q_tokens, w.heads, w.head_dim, "q")
-
-    def run(rows):
-        t0 = time.perf_counter()
+    def __init__(self, w):
+        import oracle
+        self.oracle, self.w = oracle, w
+        self.og = oracle.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, *w.bands, w.theta)
+        self.om = oracle.Mask(block_causal=bool(w.mask_kind & 1), radial=bool(w.mask_kind & 2),
+                              chunk_frames=w.chunk_frames, w0=w.w0, gamma_shift=w.gamma_shift,
+                              lam=w.lam)
+        ft = w.frame_tokens
+        n_kv = w.kv_stream_frames * ft
+        k = synth.bf16_bits_to_f64(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "k"))
+        v = synth.bf16_bits_to_f64(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "v"))
         kc = np.zeros((w.heads, w.kv_tokens, w.head_dim))
         vc = np.zeros_like(kc)
         for s, n in w.appends:
             off = (s - w.kv_stream_first_frame) * ft
-            oracle.kv_append(kc, vc, w.capacity_frames, og, k[off:off + n * ft], v[off:off + n * ft], s, n)
-        qp = tuple(p[rows] for p in qpos_all)
-        q = oracle.rope3d(synth.bf16_bits_to_f64(qbits[rows]), qp, og)
-        m = oracle.mask_rows(qp, kpos, kvalid, om)
-        oracle.attention(q, kc.transpose(1, 0, 2), vc.transpose(1, 0, 2), m, w.scale)
-        dt = time.perf_counter() - t0
-        return dt, int(m.sum())
+            oracle.kv_append(kc, vc, w.capacity_frames, self.og, k[off:off + n * ft],
+                             v[off:off + n * ft], s, n)
+        self.kt = np.ascontiguousarray(kc.transpose(1, 0, 2))
+        self.vt = np.ascontiguousarray(vc.transpose(1, 0, 2))
+        first, last = w.window()
+        self.kpos, self.kvalid = oracle.cache_positions(w.capacity_frames, first, last,
+                                                        w.grid_h, w.grid_w)
+        self.qpos = oracle.positions(w.q_tokens, w.grid_h, w.grid_w, w.q_start)
+        self.qbits = synth.qkv_bf16(w.id, w.q_tokens, w.heads, w.head_dim, "q")
+        self.rng = np.random.default_rng(0)
+        self.rows_per_s = None
 
-    rng = np.random.default_rng(0)
-    rows = np.sort(rng.choice(w.q_tokens, pilot_rows, replace=False))
-    dt, _ = run(rows)
-    n_rows = int(min(w.q_tokens, max(pilot_rows, pilot_rows * budget_s / max(dt, 1e-3))))
-    rows = np.sort(rng.choice(w.q_tokens, n_rows, replace=False))
-    dt, kept = run(rows)
-    flops = 4.0 * w.head_dim * w.heads * kept
-    desc = (f"oracle (fp64 C, OpenMP) KV appends of the step for all {w.heads} heads + RoPE/mask/"
-            f"two-pass attention of {n_rows} random query rows x {w.heads} heads against all "
-            f"{w.kv_tokens} keys; TFLOP/s counts 4*d per kept pair of the sample")
-    return flops / dt / 1e12, dt, desc
+    def _run(self, n_rows):
+        o, w = self.oracle, self.w
+        rows = np.sort(self.rng.choice(w.q_tokens, n_rows, replace=False))
+        t0 = time.perf_counter()
+        qp = tuple(p[rows] for p in self.qpos)
+        q = o.rope3d(synth.bf16_bits_to_f64(self.qbits[rows]), qp, self.og)
+        m = o.mask_rows(qp, self.kpos, self.kvalid, self.om)
+        o.attention(q, self.kt, self.vt, m, w.scale)
+        dt = time.perf_counter() - t0
+        return dt, 4.0 * w.head_dim * w.heads * int(m.sum()), n_rows
+
+    def sample(self, budget_s):
+        """One timed sample of about budget_s seconds: (TFLOP/s, seconds, rows)."""
+        if self.rows_per_s is None:
+            dt, _, n = self._run(8)
+            self.rows_per_s = n / max(dt, 1e-4)
+        n_rows = int(min(self.w.q_tokens, max(1, self.rows_per_s * budget_s)))
+        dt, flops, n = self._run(n_rows)
+        self.rows_per_s = n / max(dt, 1e-4)
+        return flops / dt / 1e12, dt, n
+
+    def describe(self, n_rows):
+        w = self.w
+        return (f"oracle (fp64 C, OpenMP): RoPE + explicit mask + two-pass attention of {n_rows} "
+                f"random query rows x {w.heads} heads against all {w.kv_tokens} key slots (cache "
+                f"built by the oracle's appends before timing); TFLOP/s counts 4*d per kept pair")
 
 
 def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    cores = os.cpu_count()
-    times, vals = [], []
-    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    arm = OracleArm(w)
+    budget = max(0.1, 90.0 / max(1, args.steps + args.warmup))
+    times, vals, rows = [], [], 0
     for i in range(args.warmup + args.steps):
-        val, dt, desc = oracle_sample(w, budget_s=budget)
+        val, dt, n = arm.sample(budget)
         if i >= args.warmup:
             times.append(dt)
             vals.append(val)
+            rows = n
     value = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -128,8 +164,8 @@ def run_reference(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic N(0,1), seeded SplitMix64 + Box-Muller, bf16-rounded",
             "config": config_of(w, {"parallelism": "host cores (OpenMP)"}),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": arm.describe(rows)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -282,12 +318,7 @@ def run_gpu(args, w):
     t1.record(stream)
     barrier()
     clk = clocks.stop() if clocks else None
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms / args.steps
     attn_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps))
     app_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
@@ -309,38 +340,57 @@ def run_gpu(args, w):
     rope_ms = r0.elapsed_time(r1) / n_rope
     rope_bytes = 2 * q.numel() * 2
 
-    # end to end through the public API: pinned host inputs -> device, step, output -> host
-    q_p, k_p, v_p = q_h.pin_memory(), k_h[off_last:off_last + n_last * ft].pin_memory(), \
-        v_h[off_last:off_last + n_last * ft].pin_memory()
-    o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_step), torch.empty_like(v_step)
+    # End to end through the public API: every step copies its Q, K, V from pinned host memory
+    # and its O back to pinned host memory. Inputs and outputs are double-buffered and the copies
+    # run on their own streams, so step i's copies overlap step i-1's kernels (a stream of denoise
+    # steps); the KV cache is only touched by the compute stream, in step order.
+    k_src, v_src = k_h[off_last:off_last + n_last * ft], v_h[off_last:off_last + n_last * ft]
+    q_p, k_p, v_p = q_h.pin_memory(), k_src.pin_memory(), v_src.pin_memory()
+    o_p = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
+    q_d = [torch.empty_like(q) for _ in range(2)]
+    k_d = [torch.empty_like(k_step) for _ in range(2)]
+    v_d = [torch.empty_like(v_step) for _ in range(2)]
+    o_d = [torch.empty_like(o) for _ in range(2)]
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in comp_done + d2h_done:
+        e.record(stream)
 
-    def e2e_step():
-        q_d.copy_(q_p, non_blocking=True)
-        k_d.copy_(k_p, non_blocking=True)
-        v_d.copy_(v_p, non_blocking=True)
-        vdit.kv_append(cache.k, cache.v, g, w.capacity_frames, k_d, v_d, s_last)
-        vdit.attn_forward(plan, q_d, cache, out=o, scale=w.scale)
-        o_p.copy_(o, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(s_h2d):
+            s_h2d.wait_event(comp_done[b])  # buffer b's inputs are free once step i-2 ran
+            q_d[b].copy_(q_p, non_blocking=True)
+            k_d[b].copy_(k_p, non_blocking=True)
+            v_d[b].copy_(v_p, non_blocking=True)
+            h2d_done[b].record(s_h2d)
+        stream.wait_event(h2d_done[b])
+        stream.wait_event(d2h_done[b])  # o_d[b] was read back by step i-2's copy
+        vdit.kv_append(cache.k, cache.v, g, w.capacity_frames, k_d[b], v_d[b], s_last, stream=stream)
+        vdit.attn_forward(plan, q_d[b], cache, out=o_d[b], scale=w.scale, stream=stream)
+        comp_done[b].record(stream)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(comp_done[b])
+            o_p[b].copy_(o_d[b], non_blocking=True)
+            d2h_done[b].record(s_d2h)
 
     n_e2e = max(3, min(args.steps, 20))
-    for _ in range(2):
-        e2e_step()
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_h2d)
+    for i in range(n_e2e):
+        e2e_step(i)
+    s_d2h.wait_event(comp_done[(n_e2e - 1) % 2])
+    e1.record(s_d2h)
+    torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
     h2d = (q_p.numel() + k_p.numel() + v_p.numel()) * 2
-    d2h = o_p.numel() * 2
+    d2h = o_p[0].numel() * 2
 
     if rank == 0:
         pk, src = peaks()
@@ -349,13 +399,14 @@ def run_gpu(args, w):
         traffic, tnote = traffic_per_launch(w)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            val, dt, desc = oracle_sample(w, budget_s=args.cpu_budget)
+            arm = OracleArm(w)
+            val, dt, n = arm.sample(args.cpu_budget)
             cpu = {"value": val, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-                   "sample": desc, "seconds": dt}
+                   "sample": arm.describe(n), "seconds": dt}
         info = plan.info
         line = {
             "metric": METRIC,
-            "value": world * flops / (ms_step * 1e-3) / 1e12,
+            "value": aggregate_tflops(world, flops, ms_step),
             "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
@@ -377,8 +428,10 @@ def run_gpu(args, w):
                          "traffic": traffic, "traffic_note": tnote,
                          "algorithmic": "4*head_dim FLOP per kept (query, key, head): %.4g per launch" % flops},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": aggregate_tflops(world, flops, e2e_ms), "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "how": "public API; per step H2D of Q, K, V from pinned memory and D2H of O, "
+                           "double-buffered on copy streams overlapping the previous step"},
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
             "kernels": {
