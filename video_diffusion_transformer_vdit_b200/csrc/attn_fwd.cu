@@ -348,13 +348,14 @@ __device__ __forceinline__ uint4 rope_chunk(uint4 in, int pp0, int t, int h, int
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int pp = pp0 + i;
-        float2 cs;
-        if (pp < a.bt2)
-            cs = __ldg(a.tt + (size_t)t * a.bt2 + pp);
-        else if (pp < a.bt2 + a.bh2)
-            cs = __ldg(a.th + h * a.bh2 + (pp - a.bt2));
-        else
-            cs = __ldg(a.tw + w * a.bw2 + (pp - a.bt2 - a.bh2));
+        // band of this pair, chosen without branches: the lanes of a warp hold different
+        // chunks of a head row and would otherwise split over the three table lookups
+        const bool in_h = pp >= a.bt2, in_w = pp >= a.bt2 + a.bh2;
+        const float2* tab = in_w ? a.tw : (in_h ? a.th : a.tt);
+        const int row = in_w ? w : (in_h ? h : t);
+        const int width = in_w ? a.bw2 : (in_h ? a.bh2 : a.bt2);
+        const int jj = pp - (in_w ? a.bt2 + a.bh2 : (in_h ? a.bt2 : 0));
+        const float2 cs = __ldg(tab + (size_t)row * width + jj);
         __nv_bfloat162 b;
         memcpy(&b, &word[i], 4);
         const float2 x = __bfloat1622float2(b);
