@@ -99,20 +99,31 @@ int find_rope_tables(const vdit_geom* g, RopeTables* out) {
 
 namespace {
 
-// Division by a run-time constant d via a 64-bit reciprocal: q = mulhi(n, ceil(2^64 / d)), exact
-// whenever n * d < 2^64 (all index math here stays far below that).
+// Division by a run-time invariant d (Granlund and Montgomery, "Division by invariant integers
+// using multiplication", PLDI 1994): with s = ceil(log2 d) and m = floor(2^(32+s) / d) + 1 - 2^32,
+// n / d = (mulhi(n, m) + n) >> s for every n < 2^31 (the sum cannot overflow 32 bits there).
+// All chunk, token and frame indices handled here are < 2^31 (checked on the host).
 struct FastDiv {
-    unsigned long long m;  // ceil(2^64 / d); unused when d == 1
-    unsigned long long d;
+    uint32_t m;
+    uint32_t s;
+    uint32_t d;
 };
-FastDiv make_fastdiv(unsigned long long d) {
+FastDiv make_fastdiv(uint32_t d) {
     FastDiv f;
     f.d = d;
-    f.m = d <= 1 ? 0ull : (~0ull / d) + 1ull;
+    if (d <= 1) {
+        f.m = 0;
+        f.s = 0;
+        return f;
+    }
+    uint32_t s = 0;
+    while ((1ull << s) < d) ++s;
+    f.s = s;
+    f.m = (uint32_t)(((1ull << (32 + s)) / d) + 1 - (1ull << 32));
     return f;
 }
-__device__ __forceinline__ unsigned long long fdiv(unsigned long long n, const FastDiv& f) {
-    return f.d == 1 ? n : __umul64hi(n, f.m);
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+    return f.d == 1 ? n : (__umulhi(n, f.m) + n) >> f.s;
 }
 
 struct StreamArgs {
@@ -193,17 +204,18 @@ __global__ void __launch_bounds__(256, kBlocksPerSM) rope_stream_kernel(StreamAr
         for (int u = 0; u < kUnroll; ++u) {
             const unsigned long long idx = i0 + u * stride;
             if (idx < a.total) {
-                const unsigned long long tok = fdiv(idx, a.by_cpt);
-                const int k = (int)(idx - tok * (unsigned long long)a.cpt);
+                const uint32_t i32 = (uint32_t)idx;  // total < 2^31
+                const uint32_t tok = fdiv(i32, a.by_cpt);
+                const int k = (int)(i32 - tok * (uint32_t)a.cpt);
                 const int c8 = k & cpr_mask;
-                const unsigned long long f = fdiv(tok, a.by_ft);
-                const int rem = (int)(tok - f * (unsigned long long)ft);
-                const int h = (int)fdiv((unsigned long long)rem, a.by_w);
+                const uint32_t f = fdiv(tok, a.by_ft);
+                const int rem = (int)(tok - f * (uint32_t)ft);
+                const int h = (int)fdiv((uint32_t)rem, a.by_w);
                 const int w = rem - h * a.grid_w;
                 const int t = a.start_frame + (int)f;
                 const uint4 r = rotate_chunk(xin[u], c8 * 4, t, h, w, a);
                 if (APPEND) {
-                    const int slot = t - (int)fdiv((unsigned long long)t, a.by_cap) * a.cap_frames;
+                    const int slot = t - (int)fdiv((uint32_t)t, a.by_cap) * a.cap_frames;
                     const int head = k >> a.cpr_log2;
                     const long long d =
                         (((long long)head * a.cap_tok + (long long)slot * ft + rem) << a.cpr_log2) + c8;
@@ -247,9 +259,9 @@ int fill_common(const vdit_geom* g, StreamArgs& a) {
     a.cpt = g->heads * (g->head_dim / 8);
     a.grid_h = g->grid_h;
     a.grid_w = g->grid_w;
-    a.by_cpt = make_fastdiv((unsigned long long)a.cpt);
-    a.by_ft = make_fastdiv((unsigned long long)g->grid_h * g->grid_w);
-    a.by_w = make_fastdiv((unsigned long long)g->grid_w);
+    a.by_cpt = make_fastdiv((uint32_t)a.cpt);
+    a.by_ft = make_fastdiv((uint32_t)(g->grid_h * g->grid_w));
+    a.by_w = make_fastdiv((uint32_t)g->grid_w);
     a.by_cap = make_fastdiv(1);
     return VDIT_OK;
 }
@@ -273,6 +285,8 @@ extern "C" int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int
     char* yb = static_cast<char*>(y);
     if (xb != yb && xb < yb + n_tokens * row_bytes && yb < xb + n_tokens * row_bytes)
         return fail(VDIT_ERR_INVALID_ARG, "x and y overlap without being identical");
+    if ((unsigned long long)n_tokens * g->heads * (g->head_dim / 8) >= (1ull << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "tensor larger than 2^31 16-byte chunks (32 GiB)");
     StreamArgs a{};
     if (int rc = fill_common(g, a)) return rc;
     a.x = static_cast<const uint4*>(x);
@@ -306,6 +320,8 @@ extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
         overlap(k_cache, cache_bytes, k, chunk_bytes) || overlap(k_cache, cache_bytes, v, chunk_bytes) ||
         overlap(v_cache, cache_bytes, k, chunk_bytes) || overlap(v_cache, cache_bytes, v, chunk_bytes))
         return fail(VDIT_ERR_INVALID_ARG, "caches overlap each other or the chunk");
+    if ((unsigned long long)chunk_bytes / 16 >= (1ull << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "chunk larger than 2^31 16-byte chunks (32 GiB)");
     StreamArgs a{};
     if (int rc = fill_common(g, a)) return rc;
     a.x = static_cast<const uint4*>(k);
@@ -316,6 +332,6 @@ extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
     a.start_frame = start_frame;
     a.cap_frames = capacity_frames;
     a.cap_tok = ft * capacity_frames;
-    a.by_cap = make_fastdiv((unsigned long long)capacity_frames);
+    a.by_cap = make_fastdiv((uint32_t)capacity_frames);
     return launch_stream(true, a, static_cast<cudaStream_t>(stream));
 }
