@@ -8,8 +8,8 @@
 // spatial groups.
 //
 // Both kernels are HBM streams: every 16-byte chunk of [tokens, heads, head_dim] is read once and
-// written once, consecutive threads on consecutive chunks, several independent loads in flight
-// per thread (the kernels are latency-bound otherwise). Each 32-bit word of a chunk is one RoPE
+// written once, consecutive lanes on consecutive chunks, several independent loads in flight
+// per lane (the kernels are latency-bound otherwise). Each 32-bit word of a chunk is one RoPE
 // pair (channel 2j in the low half, 2j+1 in the high half), rotated in fp32 with a (cos, sin)
 // pair read from the tables (L1/L2 resident) and rounded to bf16 nearest-even.
 #include <algorithm>
@@ -131,24 +131,23 @@ struct StreamArgs {
     uint4* y;           // rope: output; append: K cache
     const uint4* v;     // append: V chunk
     uint4* vc;          // append: V cache
-    unsigned long long total;  // 16-byte chunks to process = n_tokens * cpt
+    int n_tokens;
     int cpr_log2;       // log2(head_dim / 8): 16-byte chunks per head row
     int cpt;            // chunks per token = heads * head_dim / 8
     int grid_h, grid_w;
     int start_frame;
     int cap_frames;     // append: ring capacity in frames
     long long cap_tok;  // append: capacity_frames * grid_h * grid_w
-    FastDiv by_cpt, by_ft, by_w, by_cap;
+    FastDiv by_ft, by_w, by_cap;
     const float2* tt;
     const float2* th;
     const float2* tw;
     int bt2, bh2, bw2;  // pairs per band
 };
 
-// Rotates the four RoPE pairs of one 16-byte chunk (pairs pp0 .. pp0+3) at position (t, h, w).
-__device__ __forceinline__ uint4 rotate_chunk(uint4 in, int pp0, int t, int h, int w,
-                                              const StreamArgs& a) {
-    uint32_t word[4] = {in.x, in.y, in.z, in.w};
+// (cos, sin) of the four RoPE pairs pp0 .. pp0+3 of one 16-byte chunk at position (t, h, w).
+__device__ __forceinline__ void chunk_angles(float2 (&cs)[4], int pp0, int t, int h, int w,
+                                             const StreamArgs& a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int pp = pp0 + i;
@@ -159,70 +158,83 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 in, int pp0, int t, int h, i
         const int row = in_w ? w : (in_h ? h : t);
         const int width = in_w ? a.bw2 : (in_h ? a.bh2 : a.bt2);
         const int jj = pp - (in_w ? a.bt2 + a.bh2 : (in_h ? a.bt2 : 0));
-        const float2 cs = __ldg(tab + (size_t)row * width + jj);
+        cs[i] = __ldg(tab + (size_t)row * width + jj);
+    }
+}
+
+// Rotates the four pairs of one chunk: (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos) in fp32.
+__device__ __forceinline__ uint4 rotate_chunk(uint4 in, const float2 (&cs)[4]) {
+    uint32_t word[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
         __nv_bfloat162 b;
         memcpy(&b, &word[i], 4);
         const float2 xv = __bfloat1622float2(b);
-        const float y0 = fmaf(xv.x, cs.x, -xv.y * cs.y);
-        const float y1 = fmaf(xv.x, cs.y, xv.y * cs.x);
+        const float y0 = fmaf(xv.x, cs[i].x, -xv.y * cs[i].y);
+        const float y1 = fmaf(xv.x, cs[i].y, xv.y * cs[i].x);
         b = __floats2bfloat162_rn(y0, y1);
         memcpy(&word[i], &b, 4);
     }
     return make_uint4(word[0], word[1], word[2], word[3]);
 }
 
-// Independent 16-byte loads per thread in flight, and resident 256-thread blocks per SM. Swept
-// on B200 over (loads, blocks) = (2,8), (4,4), (4,6), (4,8), (8,4) for the 32,760-token,
-// 12-head tensors: (4,4) was best for both kernels (append 5.3-5.4 TB/s, RoPE 3.8-3.9 TB/s,
-// against 5.8 TB/s for a plain device copy of the same tensor).
-constexpr int kUnroll = 4;
-constexpr int kBlocksPerSM = 4;
+// One warp streams one token's row of heads * head_dim / 8 chunks at a time: load u of lane l
+// takes chunk 32u + l, so every warp access is 512 contiguous bytes, and since 32 is a multiple
+// of the chunks per head row, a lane meets the same RoPE pairs in every head: its four (cos, sin)
+// pairs and the token's (t, h, w) decode are done once per token, not once per chunk.
+// kBatch independent 16-byte loads per lane and tensor are in flight before any store; the
+// append holds two tensors' loads, so it runs half as many blocks per SM at twice the registers.
+constexpr int kBatch = 8;
+constexpr int kWarpsPerBlock = 8;
+template <bool APPEND>
+constexpr int blocks_per_sm() { return APPEND ? 2 : 4; }
 
-// Flattened stream over the 16-byte chunks of [tokens, heads, head_dim]: consecutive threads take
-// consecutive chunks (fully coalesced 512-byte warp accesses), each thread first issues kUnroll
-// independent loads strided by the grid size, then decodes each chunk's (token, head, pair, t, h, w)
-// by reciprocal multiplication and rotates it.
-// APPEND = false: y[chunk] = RoPE(x[chunk]).
+// APPEND = false: y = RoPE(x) at t = start_frame + local frame.
 // APPEND = true:  K' = RoPE(k) and V (unchanged) go to frame slot t mod capacity of the caches.
 template <bool APPEND>
-__global__ void __launch_bounds__(256, kBlocksPerSM) rope_stream_kernel(StreamArgs a) {
-    const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
-    const int cpr_mask = (1 << a.cpr_log2) - 1;
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, blocks_per_sm<APPEND>())
+    rope_stream_kernel(StreamArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int n_warps = gridDim.x * kWarpsPerBlock;
+    const int c8 = lane & ((1 << a.cpr_log2) - 1);
     const int ft = a.grid_h * a.grid_w;
-    for (unsigned long long i0 = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x;
-         i0 < a.total; i0 += stride * kUnroll) {
-        uint4 xin[kUnroll], vin[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const unsigned long long idx = i0 + u * stride;
-            if (idx < a.total) {
-                xin[u] = __ldcs(a.x + idx);
-                if (APPEND) vin[u] = __ldcs(a.v + idx);
-            }
+    for (int tok = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); tok < a.n_tokens; tok += n_warps) {
+        const uint32_t f = fdiv((uint32_t)tok, a.by_ft);
+        const int rem = tok - (int)f * ft;
+        const int h = (int)fdiv((uint32_t)rem, a.by_w);
+        const int w = rem - h * a.grid_w;
+        const int t = a.start_frame + (int)f;
+        float2 cs[4];
+        chunk_angles(cs, c8 * 4, t, h, w, a);
+        const size_t src0 = (size_t)tok * a.cpt;
+        size_t dst_tok = 0;  // append: chunk index of (head 0, chunk 0) of this token's cache row
+        if (APPEND) {
+            const int slot = t - (int)fdiv((uint32_t)t, a.by_cap) * a.cap_frames;
+            dst_tok = ((size_t)slot * ft + rem) << a.cpr_log2;
         }
+        for (int j0 = 0; j0 < a.cpt; j0 += 32 * kBatch) {
+            uint4 xin[kBatch], vin[kBatch];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const unsigned long long idx = i0 + u * stride;
-            if (idx < a.total) {
-                const uint32_t i32 = (uint32_t)idx;  // total < 2^31
-                const uint32_t tok = fdiv(i32, a.by_cpt);
-                const int k = (int)(i32 - tok * (uint32_t)a.cpt);
-                const int c8 = k & cpr_mask;
-                const uint32_t f = fdiv(tok, a.by_ft);
-                const int rem = (int)(tok - f * (uint32_t)ft);
-                const int h = (int)fdiv((uint32_t)rem, a.by_w);
-                const int w = rem - h * a.grid_w;
-                const int t = a.start_frame + (int)f;
-                const uint4 r = rotate_chunk(xin[u], c8 * 4, t, h, w, a);
-                if (APPEND) {
-                    const int slot = t - (int)fdiv((uint32_t)t, a.by_cap) * a.cap_frames;
-                    const int head = k >> a.cpr_log2;
-                    const long long d =
-                        (((long long)head * a.cap_tok + (long long)slot * ft + rem) << a.cpr_log2) + c8;
-                    __stcs(a.y + d, r);
-                    __stcs(a.vc + d, vin[u]);
-                } else {
-                    __stcs(a.y + idx, r);
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) {
+                    xin[u] = __ldcs(a.x + src0 + j);
+                    if (APPEND) vin[u] = __ldcs(a.v + src0 + j);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) {
+                    const uint4 r = rotate_chunk(xin[u], cs);
+                    if (APPEND) {
+                        const int head = j >> a.cpr_log2;
+                        const size_t d = dst_tok + (((size_t)head * a.cap_tok) << a.cpr_log2) + c8;
+                        __stcs(a.y + d, r);
+                        __stcs(a.vc + d, vin[u]);
+                    } else {
+                        __stcs(a.y + src0 + j, r);
+                    }
                 }
             }
         }
@@ -233,14 +245,14 @@ int launch_stream(bool append, StreamArgs& a, cudaStream_t s) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const unsigned long long per_block = 256ull * kUnroll;
-    const unsigned long long want = (a.total + per_block - 1) / per_block;
-    const int blocks = (int)std::min<unsigned long long>(want, (unsigned long long)sms * kBlocksPerSM);
+    const long long want = ((long long)a.n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int per_sm = append ? blocks_per_sm<true>() : blocks_per_sm<false>();
+    const int blocks = (int)std::min<long long>(want, (long long)sms * per_sm);
     if (blocks == 0) return VDIT_OK;
     if (append)
-        rope_stream_kernel<true><<<blocks, 256, 0, s>>>(a);
+        rope_stream_kernel<true><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
     else
-        rope_stream_kernel<false><<<blocks, 256, 0, s>>>(a);
+        rope_stream_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
     return vdit::cuda_check(cudaGetLastError(), "rope kernel launch");
 }
 
@@ -259,7 +271,6 @@ int fill_common(const vdit_geom* g, StreamArgs& a) {
     a.cpt = g->heads * (g->head_dim / 8);
     a.grid_h = g->grid_h;
     a.grid_w = g->grid_w;
-    a.by_cpt = make_fastdiv((uint32_t)a.cpt);
     a.by_ft = make_fastdiv((uint32_t)(g->grid_h * g->grid_w));
     a.by_w = make_fastdiv((uint32_t)g->grid_w);
     a.by_cap = make_fastdiv(1);
@@ -291,7 +302,7 @@ extern "C" int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int
     if (int rc = fill_common(g, a)) return rc;
     a.x = static_cast<const uint4*>(x);
     a.y = static_cast<uint4*>(y);
-    a.total = (unsigned long long)n_tokens * a.cpt;
+    a.n_tokens = (int)n_tokens;
     a.start_frame = start_frame;
     return launch_stream(false, a, static_cast<cudaStream_t>(stream));
 }
@@ -328,7 +339,7 @@ extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
     a.v = static_cast<const uint4*>(v);
     a.y = static_cast<uint4*>(k_cache);
     a.vc = static_cast<uint4*>(v_cache);
-    a.total = (unsigned long long)(ft * n_frames) * a.cpt;
+    a.n_tokens = (int)(ft * n_frames);
     a.start_frame = start_frame;
     a.cap_frames = capacity_frames;
     a.cap_tok = ft * capacity_frames;
