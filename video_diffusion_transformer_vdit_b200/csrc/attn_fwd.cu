@@ -10,26 +10,30 @@
 // One CTA = two 128-row query tiles (Q0, Q1) of one head, sharing every K/V tile it loads;
 // 12 warps (3 warpgroups):
 //   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query row r (TMEM lane r);
-//               tcgen05.ld of its S row, mask, online softmax in fp32 (log2 domain; O is rescaled
-//               in TMEM only when the running max grows by more than 2^8), P written back as
-//               bf16 into the S columns of TMEM (tcgen05.st), epilogue (O / l -> bf16, staged
-//               through shared memory for 256-byte coalesced row stores; natural-log LSE);
+//               tcgen05.ld of its S row (after which the S columns are released), mask, online
+//               softmax in fp32 (log2 domain; O is rescaled in TMEM only when the running max
+//               grows by more than 2^8), P written as bf16 into the group's own P columns of
+//               TMEM (tcgen05.st), epilogue (O / l -> bf16, staged through shared memory for
+//               256-byte coalesced row stores; natural-log LSE);
 //   warp 8      producer: TMA (cp.async.bulk.tensor, SWIZZLE_128B) of K and V tiles from the
 //               head-major cache into 2-stage rings, plus the key-position table of partial tiles;
-//   warp 9      TMEM allocator (512 columns) and single-thread MMA issuer (warps 10-11 idle), kind::f16 bf16 x bf16
-//               -> fp32, M = 128:  S_h = Q_h K^T (SS, N = 128) into columns [128h, 128h + 128);
-//               O_h += P_h V (TS: P from TMEM, V the MN-major smem operand) into [256 + 128h, ..).
-//               Issue order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1), so each softmax
-//               group works while the tensor core runs the other group's two MMAs.
+//   warp 9      TMEM allocator (512 columns) and the thread issuing the score MMAs, kind::f16
+//               bf16 x bf16 -> fp32, M = 128: S_h = Q_h K^T (SS, N = 128) into the shared S
+//               columns [0, 128). A score tile waits only until the previous one has been read
+//               out of TMEM, so the tensor core computes the next scores of a group while that
+//               group's softmax still works on the current tile;
+//   warp 10     the thread issuing O_h += P_h V (TS: P_h from TMEM columns [128 + 64h, ..), V
+//               the MN-major smem operand) into [256 + 128h, ..), as soon as P_h is stored
+//               (warp 11 idle).
 // Q is read from global memory, rotated (3-D RoPE at the plan's query positions, fp32 math on
 // fp64-built tables) and written straight into the swizzled K-major layout the MMA reads: the
 // RoPE of Q is fused into the Q load.
 //
-// Ordering facts relied on: tcgen05.commit signals when every earlier tcgen05 operation of the
-// issuing thread has completed, so when softmax h sees S_h(j+1) complete, PV_h(j) (issued before
-// it) has completed too: O_h is stable for a rescale and P_h(j)'s columns may be overwritten.
-// tcgen05.mma operations of one thread execute in issue order, so S_h(j+1) (which overwrites the
-// TMEM columns holding P_h(j)) runs after PV_h(j) has read them.
+// Ordering: a score tile is issued after an mbarrier on which the previous tile's softmax group
+// arrives once its tcgen05.ld has completed (wait::ld, fence::before_thread_sync); softmax h
+// overwrites P_h and rescales O_h only after the commit of PV_h of its previous tile has
+// arrived (tcgen05.commit signals when every earlier tcgen05 operation of the issuing thread has
+// completed).
 //
 // Every mbarrier wait is bounded (globaltimer): on expiry the thread raises the CTA abort flag
 // and the device status word (VDIT_ERR_TIMEOUT), every role leaves its loop, in-flight TMA and
@@ -55,7 +59,7 @@ constexpr int kTile = 128;
 constexpr int kStages = 2;
 constexpr int kQTiles = 2;                       // query tiles per CTA (one softmax group each)
 constexpr int kSoftmaxThreads = 128 * kQTiles;
-constexpr int kWarpTMA = 8, kWarpMMA = 9;     // warps 10-11 complete the third warpgroup
+constexpr int kWarpTMA = 8, kWarpMMA = 9, kWarpPV = 10;  // warp 11 completes the third warpgroup
 constexpr int kThreads = 384;
 // Register split (setmaxnreg, per warpgroup): launched at 168 per thread (3 warps per SM
 // sub-partition, 16384 registers each); the two softmax groups grow to 208 and the producer /
@@ -64,7 +68,10 @@ constexpr int kThreads = 384;
 constexpr int kRegsSoftmax = 208, kRegsOther = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * 168, "register split");
 constexpr uint32_t kSlabBytes = kTile * 64 * 2;  // 16 KiB: 128 rows x 128 B (one swizzle width)
-constexpr uint32_t kTmemCols = 512;              // S0/P0, S1/P1, O0, O1: 128 columns each
+// TMEM columns: S [0, 128) shared by the two query tiles, P0 [128, 192), P1 [192, 256) (bf16
+// pairs), O0 [256, 384), O1 [384, 512).
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemP = 128, kTmemO = 256;
 constexpr float kRescaleTau = 8.0f;              // rescale O only when the max grows by > 2^8
 // Which of every 8 consecutive P pairs of a row take the FMA-pipe exp2 instead of the MUFU unit
 // (bit i set: pair i mod 8). Measured on the dense 32,760-token workload: none 1073, two of
@@ -81,8 +88,8 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 enum {
     B_KFULL = 0, B_KEMPTY = B_KFULL + kStages, B_VFULL = B_KEMPTY + kStages,
     B_VEMPTY = B_VFULL + kStages, B_IFULL = B_VEMPTY + kStages, B_IEMPTY = B_IFULL + kStages,
-    B_SFULL = B_IEMPTY + kStages, B_PFULL = B_SFULL + kQTiles, B_ODONE = B_PFULL + kQTiles,
-    B_DRAIN = B_ODONE + kQTiles, B_COUNT
+    B_SFULL = B_IEMPTY + kStages, B_SFREE = B_SFULL + kQTiles, B_PFULL = B_SFREE + 1,
+    B_PVDONE = B_PFULL + kQTiles, B_DRAIN = B_PVDONE + kQTiles, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier area too small");
 // Key-position table of a partial tile, one per K stage: a 16-byte header {tile, flags, nseg}
@@ -422,9 +429,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < kQTiles; ++h) {
             mbar_init(BAR(B_SFULL + h), 1);
             mbar_init(BAR(B_PFULL + h), 128);
-            mbar_init(BAR(B_ODONE + h), 1);
+            mbar_init(BAR(B_PVDONE + h), 1);
         }
-        mbar_init(BAR(B_DRAIN), 1);
+        mbar_init(BAR(B_SFREE), 128);
+        mbar_init(BAR(B_DRAIN), 2);  // one commit from each MMA-issuing thread
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -462,8 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = warp >> 2;
         const int row = threadIdx.x & 127;  // TMEM lane == query row within the tile
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t t_s = tmem + 128u * h + lane_base;
-        const uint32_t t_o = tmem + 256u + 128u * h + lane_base;
+        const uint32_t t_s = tmem + lane_base;
+        const uint32_t t_p = tmem + kTmemP + 64u * h + lane_base;
+        const uint32_t t_o = tmem + kTmemO + 128u * h + lane_base;
         const uint32_t f_in = h ? 4u : 1u, f_full = h ? 8u : 2u;
         const int qi = (qb * kQTiles + h) * kTile + row;
         const int qf = qi / ft, qrem = qi - qf * ft;
@@ -491,6 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             reg_touch32(sr + 32);
             reg_touch32(sr + 64);
             reg_touch32(sr + 96);
+            // S is in registers: the shared S columns may take the next score tile
+            tc_fence_before();
+            mbar_arrive(BAR(B_SFREE));
             float* sv = reinterpret_cast<float*>(sr);
             if (!(flags & f_full)) {
                 const int nseg = reinterpret_cast<const int*>(info)[2];
@@ -552,7 +564,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m = m_new;
             }
             const float mc = (m == -INFINITY) ? 0.f : m * c;
-            // O_h is stable here: PV_h of the previous tile completed before S_h of this one
+            // PV_h of the previous tile must have completed: it reads P_h (overwritten below)
+            // and accumulates into O_h (rescaled below)
+            if (cnt > 0) {
+                if (!warp_wait(BAR(B_PVDONE + h), (cnt - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                tc_fence_after();
+            }
             if (cnt > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
                 for (int q4 = 0; q4 < D / 32; ++q4) {
@@ -565,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st32(t_o + q4 * 32, orow);
                 }
             }
-            // P = 2^(s*c - m*c) as bf16 pairs into the S columns [0, 64) of this lane; the pairs
+            // P = 2^(s*c - m*c) as bf16 pairs into the P_h columns of this lane; the pairs
             // selected by kPolyPairs take the FMA-pipe exp2 so the MUFU pipe is not the bound
             uint64_t rs2[4];
 #pragma unroll
@@ -592,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
                     memcpy(&pk[i], &b, 4);
                 }
-                tmem_st32(t_s + 32 * half, pk);
+                tmem_st32(t_p + 32 * half, pk);
             }
             float rsum;
             {
@@ -608,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++cnt;
         }
         if (ok && cnt > 0) {
-            if (!warp_wait(BAR(B_ODONE + h), 0, abort_flag, a.status)) ok = false;
+            if (!warp_wait(BAR(B_PVDONE + h), (cnt - 1) & 1, abort_flag, a.status)) ok = false;
         }
         // every thread of the group reaches this barrier (aborted or not); any failure skips
         // the epilogue of the whole group
@@ -786,87 +803,93 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == kWarpMMA) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == kWarpMMA || warp == kWarpPV) {
+        // ------------------------------------------------------------------ MMA issuers
+        // Two issuing threads: warp 9 issues the score MMAs, warp 10 the PV MMAs. Each waits
+        // only for its own operands, so a wait of one never leaves the tensor core without
+        // queued work from the other (an issuing thread that stops to poll an mbarrier, even
+        // a completed one, leaves a gap in the tensor pipe).
+        const bool s_role = warp == kWarpMMA;
         if (lane == 0 && n_ent > 0) {
             constexpr uint32_t idesc_qk = instr_desc(kTile, 0), idesc_pv = instr_desc(D, 1);
             // Descriptors are built once; each MMA only adds a compile-time offset (in 16-byte
-            // units) to a loop-invariant base, which keeps the single issuing thread at the
-            // tensor core's rate (a descriptor rebuilt from runtime indices per MMA was measured
-            // to cost more issue time than the 64-cycle M=128 N=128 K=16 MMA itself).
+            // units) to a loop-invariant base, which keeps the issuing thread at the tensor
+            // core's rate (a descriptor rebuilt from runtime indices per MMA was measured to
+            // cost more issue time than the 64-cycle M=128 N=128 K=16 MMA itself).
             const uint64_t dq0 = smem_desc_sw128(sbase + L::OFF_Q, 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(sbase + L::OFF_K, 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(sbase + L::OFF_V, kSlabBytes, 1024);
             constexpr uint64_t kTileDesc = kTileBytes >> 4;  // one tile further, in descriptor units
-            auto issue_s = [&](int h, int s) {
-                const uint64_t q0 = dq0 + (h ? kTileDesc : 0), k0 = dk0 + (s ? kTileDesc : 0);
-                const uint32_t d_t = h ? tmem + 128u : tmem;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = (uint64_t)((((kk >> 2) * kSlabBytes) + (kk & 3) * 32) >> 4);
-                    tc_mma(d_t, q0 + off, k0 + off, idesc_qk, kk > 0);
-                }
-                tc_commit(BAR(B_SFULL + h));
-            };
-            auto issue_pv = [&](int h, int s, bool acc) {
-                const uint64_t v0 = dv0 + (s ? kTileDesc : 0);
-                const uint32_t d_t = h ? tmem + 384u : tmem + 256u;
-                const uint32_t a_t = h ? tmem + 128u : tmem;
-                const uint32_t acc0 = acc ? 1u : 0u;
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    tc_mma_ts(d_t, a_t + 8u * kk, v0 + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
-                              kk > 0 ? 1u : acc0);
-            };
             const unsigned char* fl = a.u_flags + u_begin;
-            // tile flags are read three entries ahead so the global-load latency never sits
+            // tile flags are read two entries ahead so the global-load latency never sits
             // between a completed barrier and the next MMA issue
             int f_cur = __ldg(fl + entry(0));
             int f_nxt = n_ent > 1 ? __ldg(fl + entry(1)) : 0;
-            int f_nn = n_ent > 2 ? __ldg(fl + entry(2)) : 0;
-            bool ok = wait_bounded(BAR(B_KFULL + 0), 0, abort_flag, a.status);
-            if (ok) {
-                tc_fence_after();
-                if (f_cur & 1) issue_s(0, 0);
-                if (f_cur & 4) issue_s(1, 0);
-                tc_commit(BAR(B_KEMPTY + 0));
-            }
-            int npv[2] = {0, 0};
-            for (int j = 0; ok && j < n_ent; ++j) {
-                const int s = j % kStages, s1 = (j + 1) % kStages;
-                const int f = f_cur, fn = f_nxt;
-                const int f3 = j + 3 < n_ent ? __ldg(fl + entry(j + 3)) : 0;
-                f_cur = f_nxt;
-                f_nxt = f_nn;
-                f_nn = f3;
-                if (!wait_bounded(BAR(B_VFULL + s), (j / kStages) & 1, abort_flag, a.status)) break;
-                bool k_ready = false;
+            if (s_role) {
+                // S_h(j) = Q_h K(j)^T into the shared S columns, in list order, each after the
+                // previous score tile has been read out of TMEM by its softmax group
+                int ns = 0;
+                for (int j = 0; j < n_ent; ++j) {
+                    const int s = j % kStages;
+                    const int f = f_cur;
+                    f_cur = f_nxt;
+                    f_nxt = j + 2 < n_ent ? __ldg(fl + entry(j + 2)) : 0;
+                    if (!wait_bounded(BAR(B_KFULL + s), (j / kStages) & 1, abort_flag, a.status)) break;
+                    tc_fence_after();
+                    const uint64_t k0 = dk0 + (s ? kTileDesc : 0);
+                    bool ok = true;
 #pragma unroll
-                for (int h = 0; h < kQTiles; ++h) {
-                    if (f & (h ? 4 : 1)) {
+                    for (int h = 0; h < kQTiles; ++h) {
+                        if (!(f & (h ? 4 : 1))) continue;
+                        if (ns > 0) {
+                            if (!wait_bounded(BAR(B_SFREE), (ns - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                            tc_fence_after();
+                        }
+                        const uint64_t q0 = dq0 + (h ? kTileDesc : 0);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t off = (uint64_t)((((kk >> 2) * kSlabBytes) + (kk & 3) * 32) >> 4);
+                            tc_mma(tmem, q0 + off, k0 + off, idesc_qk, kk > 0);
+                        }
+                        tc_commit(BAR(B_SFULL + h));
+                        ++ns;
+                    }
+                    if (!ok) break;
+                    tc_commit(BAR(B_KEMPTY + s));
+                }
+            } else {
+                // O_h += P_h(j) V(j), each as soon as softmax h has stored P_h(j)
+                int npv[2] = {0, 0};
+                for (int j = 0; j < n_ent; ++j) {
+                    const int s = j % kStages;
+                    const int f = f_cur;
+                    f_cur = f_nxt;
+                    f_nxt = j + 2 < n_ent ? __ldg(fl + entry(j + 2)) : 0;
+                    if (!wait_bounded(BAR(B_VFULL + s), (j / kStages) & 1, abort_flag, a.status)) break;
+                    const uint64_t v0 = dv0 + (s ? kTileDesc : 0);
+                    bool ok = true;
+#pragma unroll
+                    for (int h = 0; h < kQTiles; ++h) {
+                        if (!(f & (h ? 4 : 1))) continue;
                         if (!wait_bounded(BAR(B_PFULL + h), npv[h] & 1, abort_flag, a.status)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv(h, s, npv[h] > 0);
+                        const uint32_t d_t = tmem + kTmemO + 128u * h;
+                        const uint32_t a_t = tmem + kTmemP + 64u * h;
+                        const uint32_t acc0 = npv[h] > 0 ? 1u : 0u;
+#pragma unroll
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            tc_mma_ts(d_t, a_t + 8u * kk, v0 + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                                      kk > 0 ? 1u : acc0);
+                        tc_commit(BAR(B_PVDONE + h));
                         ++npv[h];
                     }
-                    if (fn & (h ? 4 : 1)) {
-                        if (!k_ready) {
-                            if (!wait_bounded(BAR(B_KFULL + s1), ((j + 1) / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
-                            tc_fence_after();
-                            k_ready = true;
-                        }
-                        issue_s(h, s1);
-                    }
+                    if (!ok) break;
+                    tc_commit(BAR(B_VEMPTY + s));
                 }
-                if (!ok) break;
-                tc_commit(BAR(B_VEMPTY + s));
-                if (j + 1 < n_ent) tc_commit(BAR(B_KEMPTY + s1));
             }
-            for (int h = 0; h < kQTiles; ++h)
-                if (npv[h] > 0) tc_commit(BAR(B_ODONE + h));
         }
         if (lane == 0) {
-            // drain: all MMAs issued by this thread complete before TMEM is released
+            // drain: all MMAs issued by both threads complete before TMEM is released
             tc_commit(BAR(B_DRAIN));
             const uint64_t t0 = globaltimer();
             while (!mbar_try_wait(BAR(B_DRAIN), 0) && globaltimer() - t0 < kWaitLimitNs) {
