@@ -92,6 +92,69 @@ def test_plan_bit_exact_vs_oracle_random_geometries():
         _compare(plan, ref)
 
 
+def _check_masks(plan, grid_h, grid_w, q_start, q_frames, cap, first, last, kind, chunk, w0, g, lam,
+                 q_tiles=None):
+    """The plan's per-row keep masks of partial tiles equal the oracle's explicit mask, bit by
+    bit (for the given q-tiles, all by default)."""
+    rp, ci, fu = (t.numpy() for t in plan.export())
+    idx, words = plan.export_masks()
+    assert np.array_equal(idx >= 0, fu == 0)
+    assert len(words) == int((fu == 0).sum()) and (idx[idx >= 0] == np.arange(len(words))).all()
+    n_q = q_frames * grid_h * grid_w
+    qpos = oracle.positions(n_q, grid_h, grid_w, q_start)
+    kpos, kvalid = oracle.cache_positions(cap, first, last, grid_h, grid_w)
+    m = oracle.Mask(block_causal=bool(kind & 1), radial=bool(kind & 2), chunk_frames=chunk,
+                    w0=w0, gamma_shift=g, lam=lam)
+    n_k = len(kvalid)
+    bits = np.arange(32, dtype=np.uint32)
+    for qt in (range(len(rp) - 1) if q_tiles is None else q_tiles):
+        q0, q1 = qt * 128, min(n_q, qt * 128 + 128)
+        ref = oracle.mask_rows(tuple(p[q0:q1] for p in qpos), kpos, kvalid, m).astype(bool)
+        for i in range(rp[qt], rp[qt + 1]):
+            kt = ci[i]
+            k0, k1 = kt * 128, min(n_k, kt * 128 + 128)
+            want = np.zeros((128, 128), bool)
+            want[:q1 - q0, :k1 - k0] = ref[:, k0:k1]
+            if idx[i] < 0:
+                assert want.all()
+                continue
+            got = ((words[idx[i]][:, :, None] >> bits) & 1).reshape(128, 128).astype(bool)
+            assert np.array_equal(got, want), (qt, kt)
+
+
+@pytest.mark.parametrize("wid", sorted(WORKLOADS))
+def test_plan_masks_bit_exact_vs_oracle_workloads(wid):
+    w = WORKLOADS[wid]
+    first, last = w.window()
+    plan = vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                     kv_first_frame=first, kv_last_frame=last, upload=False)
+    n_qt = plan.info["q_tiles"]
+    # full-size workloads: the first, the last (ragged) and a spread of q-tiles in between
+    sample = None if n_qt <= 8 else sorted({0, 1, n_qt // 3, n_qt // 2, (2 * n_qt) // 3, n_qt - 2, n_qt - 1})
+    _check_masks(plan, w.grid_h, w.grid_w, w.q_start, w.q_frames, w.capacity_frames, first, last,
+                 w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, sample)
+
+
+def test_plan_masks_bit_exact_vs_oracle_random_geometries():
+    rng = np.random.default_rng(11)
+    for _ in range(40):
+        gh, gw = int(rng.integers(1, 9)), int(rng.integers(1, 40))
+        cap = int(rng.integers(1, 12))
+        last = int(rng.integers(0, 40))
+        first = max(0, last - int(rng.integers(0, cap)))
+        q_frames = int(rng.integers(1, 6))
+        q_start = int(rng.integers(max(0, last - 8), last + 3))
+        kind = int(rng.integers(0, 4))
+        chunk = int(rng.integers(1, 5))
+        w0 = int(rng.integers(0, 60))
+        gs = int(rng.integers(0, 3))
+        lam = int(rng.integers(0, 6))
+        g = vdit.Geometry(gh, gw, 1, 64, (24, 20, 20))
+        plan = vdit.Plan(g, vdit.Mask(kind, chunk, w0, gs, lam), q_start, q_frames,
+                         capacity_frames=cap, kv_first_frame=first, kv_last_frame=last, upload=False)
+        _check_masks(plan, gh, gw, q_start, q_frames, cap, first, last, kind, chunk, w0, gs, lam)
+
+
 def test_plan_rejects_bad_arguments():
     L = vdit.lib()
     g = vdit.Geometry(30, 52, 12, 128, (44, 42, 42)).c()

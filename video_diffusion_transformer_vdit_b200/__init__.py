@@ -63,7 +63,8 @@ class _PlanInfo(ctypes.Structure):
     _fields_ = [("q_tokens", ctypes.c_int), ("kv_tokens", ctypes.c_int), ("q_tiles", ctypes.c_int),
                 ("kv_tiles", ctypes.c_int), ("tiles", ctypes.c_int), ("full_tiles", ctypes.c_int),
                 ("kept_pairs", ctypes.c_longlong), ("uploaded", ctypes.c_int),
-                ("kv_splits", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong)]
+                ("kv_splits", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong),
+                ("mask_bytes", ctypes.c_longlong)]
 
 
 _lib = None
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_upload.argtypes = [P, P]
         L.vdit_plan_info.argtypes = [P, ctypes.POINTER(_PlanInfo)]
         L.vdit_plan_export.argtypes = [P, P, P, P]
+        L.vdit_plan_export_masks.argtypes = [P, P, P]
         L.vdit_plan_destroy.argtypes = [P]
         L.vdit_plan_destroy.restype = None
         L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
@@ -264,6 +266,17 @@ class Plan:
                                       ctypes.c_void_p(ci.data_ptr()), ctypes.c_void_p(fu.data_ptr())))
         n = inf["tiles"]
         return rp, ci[:n], fu[:n]
+
+    def export_masks(self):
+        """(mask_index [tiles] int32, words [blocks, 128, 4] uint32 as int64 numpy): the per-row
+        keep masks of the partial tiles (mask_index -1 for a full tile)."""
+        import numpy as np
+        inf = self.info
+        idx = np.zeros(max(1, inf["tiles"]), np.int32)
+        words = np.zeros(max(4, inf["mask_bytes"] // 4), np.uint32)
+        _check(lib().vdit_plan_export_masks(self._h, ctypes.c_void_p(idx.ctypes.data),
+                                            ctypes.c_void_p(words.ctypes.data)))
+        return idx[:inf["tiles"]], words[:inf["mask_bytes"] // 4].reshape(-1, 128, 4)
 
     def flops(self) -> float:
         """Unmasked-entry FLOPs of one forward: 4 * head_dim per kept (query, key, head)."""

@@ -5,7 +5,7 @@
 // Video Generation Inference with Sequential-Parallel 3D Positional Encoding Using a Global Time
 // Index", section 1) over the block-causal / radial tile schedule ("DynamicRad", section 2;
 // Wave Forcing / WaveRT block-causal chunks). Only the tiles the plan lists are visited; a tile
-// flagged full skips the per-pair predicate.
+// flagged full needs no mask; a partial one applies the per-row keep bits the plan computed.
 //
 // One CTA = two 128-row query tiles (Q0, Q1) of one head, sharing every K/V tile it loads;
 // 12 warps (3 warpgroups):
@@ -16,7 +16,8 @@
 //               TMEM (tcgen05.st), epilogue (O / l -> bf16, staged through shared memory for
 //               256-byte coalesced row stores; natural-log LSE);
 //   warp 8      producer: TMA (cp.async.bulk.tensor, SWIZZLE_128B) of K and V tiles from the
-//               head-major cache into 2-stage rings, plus the key-position table of partial tiles;
+//               head-major cache into 2-stage rings, plus (bulk copy) the plan's per-row keep
+//               masks of the partial tiles;
 //   warp 9      TMEM allocator (512 columns) and the thread issuing the score MMAs, kind::f16
 //               bf16 x bf16 -> fp32, M = 128: S_h = Q_h K^T (SS, N = 128) into the shared S
 //               columns [0, 128). A score tile waits only until the previous one has been read
@@ -92,12 +93,11 @@ enum {
     B_PVDONE = B_PFULL + kQTiles, B_DRAIN = B_PVDONE + kQTiles, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier area too small");
-// Key-position table of a partial tile, one per K stage: a 16-byte header {tile, flags, nseg}
-// and either nseg row segments (nseg >= 0; consecutive keys of one frame slot and patch row,
-// int4 {k0 | len << 8 | h << 16, frame, causal chunk, first w}) or, when the tile holds more
-// than kMaxSeg segments (very narrow grids), one int4 {frame, h, w, chunk} per key (nseg = -1).
-constexpr int kMaxSeg = 32;
-constexpr uint32_t kKinfoBytes = 16 + kTile * 16;
+// Stage of the keep masks, one per K stage: a 16-byte header {tile, flags} and, for each query
+// tile whose entry is partial, its 2 KiB block of per-row keep masks (128 rows x 4 words, bit k of
+// row r: key k kept for query r), copied from the plan by the producer.
+constexpr uint32_t kMaskBlockBytes = kTile * 16;
+constexpr uint32_t kKinfoBytes = 16 + kQTiles * kMaskBlockBytes;
 
 // Shared-memory map for head_dim D (offsets from a 1024-byte aligned base).
 template <int D>
@@ -110,8 +110,8 @@ struct Layout {
     static constexpr uint32_t OFF_BAR = OFF_V + kStages * kTileBytes;
     static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 32;  // [0] tmem base, [1] abort flag
     static constexpr uint32_t OFF_KINFO = OFF_MISC + 64;
-    static constexpr uint32_t OFF_RAD = OFF_KINFO + kStages * kKinfoBytes;
-    static constexpr uint32_t kSmemBytes = OFF_RAD + (VDIT_MAX_DT + 1) * 4 + 1024;  // + align slack
+    static constexpr uint32_t kSmemBytes = OFF_KINFO + kStages * kKinfoBytes + 1024;  // + align slack
+    static_assert(OFF_KINFO % 16 == 0 && kKinfoBytes % 16 == 0, "bulk-copy destinations 16-byte aligned");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -123,8 +123,8 @@ struct AttnArgs {
     float* ws_o;           // split > 1: normalised partial O [split][q_tokens][heads][D]
     float* ws_lse;         // split > 1: partial log2-sum-exp [split][heads][q_tokens]
     int n_qb, n_split;
-    const int* slot_frame;
-    const int* radius;
+    const uint32_t* masks; // keep-mask blocks of the partial tiles (2 KiB each)
+    const int* u_mask;     // per union entry and query tile: mask block, or -1
     const uint4* q;
     uint4* o;
     float* lse;
@@ -137,8 +137,6 @@ struct AttnArgs {
     int q_tokens, kv_tokens, heads;
     int grid_h, grid_w;
     int q_start;
-    int causal, chunk_frames;
-    int dt_max;
     float scale_log2;
 };
 
@@ -204,6 +202,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+// Plain (untiled) bulk copy global -> this CTA's shared memory, completing on an mbarrier;
+// dst, src and bytes are multiples of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -399,7 +405,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto BAR = [&](int i) { return sbase + L::OFF_BAR + 8u * (uint32_t)i; };
     volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-    int* rad_s = reinterpret_cast<int*>(smem + L::OFF_RAD);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // work unit: q-block (longest lists first), head, and the piece `sp` of its key tiles
@@ -444,7 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     // radius table and the two rotated Q tiles (all threads)
-    for (int i = threadIdx.x; i <= a.dt_max; i += kThreads) rad_s[i] = __ldg(a.radius + i);
     for (int idx = threadIdx.x; idx < kQTiles * kTile * kC16; idx += kThreads) {
         const int h = idx / (kTile * kC16), rem = idx - h * (kTile * kC16);
         const int r = rem / kC16, c16 = rem - r * kC16;
@@ -475,9 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_o = tmem + kTmemO + 128u * h + lane_base;
         const uint32_t f_in = h ? 4u : 1u, f_full = h ? 8u : 2u;
         const int qi = (qb * kQTiles + h) * kTile + row;
-        const int qf = qi / ft, qrem = qi - qf * ft;
-        const int tq = a.q_start + qf, hq = qrem / a.grid_w, wq = qrem - hq * a.grid_w;
-        const int cq = a.causal ? tq / a.chunk_frames : 0x7fffffff;
         const float c = a.scale_log2;
         float m = -INFINITY, l = 0.f;  // running max (raw score units) and sum
         int cnt = 0;
@@ -505,41 +506,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(BAR(B_SFREE));
             float* sv = reinterpret_cast<float*>(sr);
             if (!(flags & f_full)) {
-                const int nseg = reinterpret_cast<const int*>(info)[2];
-                const int4* ki = reinterpret_cast<const int4*>(info + 16);
-                uint32_t mw[4] = {0u, 0u, 0u, 0u};  // keep bit per key of the tile
-                if (nseg >= 0) {
-                    // kept keys of this row: one contiguous run per segment
-                    for (int sg = 0; sg < nseg; ++sg) {
-                        const int4 e = ki[sg];
-                        const int k0 = e.x & 0xff, len = (e.x >> 8) & 0xff, hk = e.x >> 16;
-                        if (e.y < 0 || e.z > cq) continue;
-                        const int dt = min(abs(tq - e.y), a.dt_max);
-                        const int r = min(rad_s[dt], 1 << 20);
-                        if (abs(hq - hk) > r) continue;
-                        const int lo = max(e.w, wq - r) - e.w + k0;
-                        const int hi = min(e.w + len - 1, wq + r) - e.w + k0;
-#pragma unroll
-                        for (int wd = 0; wd < 4; ++wd) {
-                            const int a0 = max(lo - 32 * wd, 0), b0 = min(hi - 32 * wd, 31);
-                            if (a0 <= b0) mw[wd] |= (0xffffffffu >> (31 - b0)) & (0xffffffffu << a0);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int wd = 0; wd < 4; ++wd) {
-                        uint32_t m = 0u;
-#pragma unroll 1
-                        for (int b = 0; b < 32; ++b) {
-                            const int4 e = ki[32 * wd + b];
-                            const int dt = min(abs(tq - e.x), a.dt_max);
-                            const int cheb = max(abs(hq - e.y), abs(wq - e.z));
-                            const bool keep = (e.x >= 0) & (e.w <= cq) & (cheb <= rad_s[dt]);
-                            m |= (uint32_t)keep << b;
-                        }
-                        mw[wd] = m;
-                    }
-                }
+                // this row's keep bits for the 128 keys of the tile, from the plan's mask block
+                const uint4 km = *reinterpret_cast<const uint4*>(info + 16 + h * kMaskBlockBytes + row * 16);
+                const uint32_t mw[4] = {km.x, km.y, km.z, km.w};
 #pragma unroll
                 for (int jj = 0; jj < 128; ++jj)
                     sv[jj] = ((mw[jj >> 5] >> (jj & 31)) & 1u) ? sv[jj] : -INFINITY;
@@ -716,15 +685,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpTMA) {
         // ------------------------------------------------------------------ producer
         int issued = 0;
+        int mask_it[kStages];  // per stage: last entry whose mask copies were issued (drain)
+#pragma unroll
+        for (int i = 0; i < kStages; ++i) mask_it[i] = -1;
         int kt_next = n_ent > 0 ? __ldg(a.u_col + u_begin + entry(0)) : 0;
         int fl_next = n_ent > 0 ? __ldg(a.u_flags + u_begin + entry(0)) : 0;
+        int mk0_next = n_ent > 0 ? __ldg(a.u_mask + 2 * (u_begin + entry(0))) : -1;
+        int mk1_next = n_ent > 0 ? __ldg(a.u_mask + 2 * (u_begin + entry(0)) + 1) : -1;
         for (int it = 0; it < (a.skip_loads ? 0 : n_ent); ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) - 1) & 1u;
-            const int kt = kt_next, flags = fl_next;
-            if (it + 1 < n_ent) {  // next entry's tile and flags, loaded while this one waits
-                kt_next = __ldg(a.u_col + u_begin + entry(it + 1));
-                fl_next = __ldg(a.u_flags + u_begin + entry(it + 1));
+            const int kt = kt_next, flags = fl_next, mk0 = mk0_next, mk1 = mk1_next;
+            if (it + 1 < n_ent) {  // next entry's tile, flags and masks, loaded while this one waits
+                const int e1 = u_begin + entry(it + 1);
+                kt_next = __ldg(a.u_col + e1);
+                fl_next = __ldg(a.u_flags + e1);
+                mk0_next = __ldg(a.u_mask + 2 * e1);
+                mk1_next = __ldg(a.u_mask + 2 * e1 + 1);
             }
             if (it >= kStages && !warp_wait(BAR(B_KEMPTY + s), ph, abort_flag, a.status)) break;
             if (lane == 0) {
@@ -741,46 +718,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 reinterpret_cast<int*>(info)[0] = kt;
                 reinterpret_cast<int*>(info)[1] = flags;
             }
-            const bool partial = ((flags & 1) && !(flags & 2)) || ((flags & 4) && !(flags & 8));
-            if (partial) {
-                int4* ki = reinterpret_cast<int4*>(info + 16);
-                // row segments of the tile (lane 0 walks them; a 30 x 52 grid gives at most 4)
-                int nseg = 0;
-                if (lane == 0) {
-                    int k = 0;
-                    const int key0 = kt * kTile;
-                    while (k < kTile && key0 + k < a.kv_tokens) {
-                        if (nseg == kMaxSeg) { nseg = -1; break; }
-                        const int key = key0 + k;
-                        const int slot = key / ft, rem = key - slot * ft;
-                        const int hh = rem / a.grid_w, ww = rem - hh * a.grid_w;
-                        const int len = min(min(a.grid_w - ww, kTile - k), a.kv_tokens - key);
-                        const int tk = __ldg(a.slot_frame + slot);
-                        const int ch = tk < 0 ? 0x7fffffff : (a.causal ? tk / a.chunk_frames : 0);
-                        ki[nseg++] = make_int4(k | (len << 8) | (hh << 16), tk, ch, ww);
-                        k += len;
-                    }
-                    reinterpret_cast<int*>(info)[2] = nseg;
-                }
-                nseg = __shfl_sync(0xffffffffu, nseg, 0);
-                if (nseg < 0) {
-                    for (int jj = lane; jj < kTile; jj += 32) {
-                        const int key = kt * kTile + jj;
-                        int4 e = make_int4(-1, 0, 0, 0x7fffffff);
-                        if (key < a.kv_tokens) {
-                            const int slot = key / ft, rem = key - slot * ft;
-                            const int hh = rem / a.grid_w;
-                            const int tk = __ldg(a.slot_frame + slot);
-                            e = make_int4(tk, hh, rem - hh * a.grid_w,
-                                          (tk >= 0 && a.causal) ? tk / a.chunk_frames : 0);
-                            if (tk < 0) e.w = 0x7fffffff;
-                        }
-                        ki[jj] = e;
-                    }
+            if (lane == 0) {
+                // keep masks of the partial query tiles of this entry (2 KiB each), else a plain
+                // arrival: the header above is published by the arrive's release either way
+                const uint32_t nbytes = (mk0 >= 0 ? kMaskBlockBytes : 0u) + (mk1 >= 0 ? kMaskBlockBytes : 0u);
+                if (nbytes) {
+                    mbar_expect_tx(BAR(B_IFULL + s), nbytes);
+                    const uint32_t dst = sbase + L::OFF_KINFO + s * kKinfoBytes + 16;
+                    if (mk0 >= 0)
+                        bulk_load(dst, a.masks + (size_t)mk0 * (kMaskBlockBytes / 4), kMaskBlockBytes, BAR(B_IFULL + s));
+                    if (mk1 >= 0)
+                        bulk_load(dst + kMaskBlockBytes, a.masks + (size_t)mk1 * (kMaskBlockBytes / 4),
+                                  kMaskBlockBytes, BAR(B_IFULL + s));
+                    mask_it[s] = it;
+                } else {
+                    mbar_arrive(BAR(B_IFULL + s));
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(B_IFULL + s));
             if (it >= kStages && !warp_wait(BAR(B_VEMPTY + s), ph, abort_flag, a.status)) break;
             if (lane == 0) {
                 mbar_expect_tx(BAR(B_VFULL + s), kTileBytes);
@@ -794,6 +749,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // drain: every TMA this warp issued must have landed before the CTA may exit
         if (*abort_flag) {
+#pragma unroll
+            for (int st = 0; st < kStages; ++st) {
+                if (mask_it[st] < 0) continue;
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(BAR(B_IFULL + st), (uint32_t)(mask_it[st] / kStages) & 1u) &&
+                       globaltimer() - t0 < kWaitLimitNs) {
+                }
+            }
             for (int jn = (issued - 2 * kStages > 0 ? issued - 2 * kStages : 0); jn < issued; ++jn) {
                 const int it = jn >> 1, s = it % kStages;
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -1038,8 +1001,8 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.ws_lse = p->d_ws_lse;
     a.n_qb = p->n_qb;
     a.n_split = p->n_split;
-    a.slot_frame = p->d_slot_frame;
-    a.radius = p->d_radius;
+    a.masks = p->d_masks;
+    a.u_mask = p->d_u_mask;
     a.q = static_cast<const uint4*>(q);
     a.o = static_cast<uint4*>(o);
     a.lse = lse;
@@ -1057,9 +1020,6 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.grid_h = p->g.grid_h;
     a.grid_w = p->g.grid_w;
     a.q_start = p->q_start;
-    a.causal = (p->m.kind & VDIT_MASK_BLOCK_CAUSAL) ? 1 : 0;
-    a.chunk_frames = a.causal ? p->m.chunk_frames : 1;
-    a.dt_max = p->dt_max;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
     dim3 grid(p->n_qb * p->n_split, p->g.heads);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1202,8 +1162,8 @@ extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, cons
     a.ws_lse = ws_lse;
     a.n_qb = p->n_qb;
     a.n_split = p->n_split;
-    a.slot_frame = p->d_slot_frame;
-    a.radius = p->d_radius;
+    a.masks = p->d_masks;
+    a.u_mask = p->d_u_mask;
     a.q = static_cast<const uint4*>(q);
     a.o = static_cast<uint4*>(o);
     a.lse = lse;
@@ -1220,9 +1180,6 @@ extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, cons
     a.grid_h = p->g.grid_h;
     a.grid_w = p->g.grid_w;
     a.q_start = p->q_start;
-    a.causal = (p->m.kind & VDIT_MASK_BLOCK_CAUSAL) ? 1 : 0;
-    a.chunk_frames = a.causal ? p->m.chunk_frames : 1;
-    a.dt_max = p->dt_max;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
     dim3 grid(p->n_qb * p->n_split, p->g.heads);
     cudaStream_t st = static_cast<cudaStream_t>(stream);

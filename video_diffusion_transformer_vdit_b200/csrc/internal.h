@@ -53,6 +53,12 @@ struct vdit_plan {
     std::vector<int> u_row_ptr, u_col;
     std::vector<unsigned char> u_flags;
     std::vector<int> unit_order;  // q-blocks by descending union-list length (longest first)
+    // keep masks of the partial tiles: mask_of[i] = block of CSR entry i (-1: full tile); block b
+    // = masks[512 b ..): 128 rows x 4 words, bit k of row r = key k of the tile kept for query r.
+    // u_mask[2 e + x] = block of union entry e for q-tile 2b + x (-1: not listed or full)
+    std::vector<int> mask_of;
+    std::vector<uint32_t> masks;
+    std::vector<int> u_mask;
     // key-range split of every (q-block, head) unit, chosen at upload from the SM count so the
     // number of CTAs fills whole waves; > 1 uses the fp32 partial workspace below
     int n_split = 1;
@@ -69,6 +75,8 @@ struct vdit_plan {
     const int* d_u_col = nullptr;
     const unsigned char* d_u_flags = nullptr;
     const int* d_unit_order = nullptr;
+    const uint32_t* d_masks = nullptr;
+    const int* d_u_mask = nullptr;
     float* d_ws_o = nullptr;    // [n_split][q_tokens][heads][head_dim] normalised partial O
     float* d_ws_lse = nullptr;  // [n_split][heads][q_tokens] partial log2-sum-exp
     size_t ws_bytes = 0;

@@ -63,6 +63,7 @@ struct Seg {
     int t;      // global frame (queries) or held frame (keys); -1 = empty slot
     int h;      // patch row
     int wlo, whi;  // inclusive column range
+    int off;    // offset of the segment's first token from the start of the split range
 };
 
 // Splits tokens [lo, hi) of a frame-major (frame, h, w) sequence into row segments. frame_of maps
@@ -75,7 +76,7 @@ void segments(int lo, int hi, int grid_h, int grid_w, F frame_of, std::vector<Se
     while (tok < hi) {
         const int f = tok / ft, rem = tok % ft, h = rem / grid_w, w = rem % grid_w;
         const int run = std::min(hi - tok, grid_w - w);
-        out.push_back(Seg{frame_of(f), h, w, w + run - 1});
+        out.push_back(Seg{frame_of(f), h, w, w + run - 1, tok - lo});
         tok += run;
     }
 }
@@ -101,6 +102,38 @@ long long pairs_within(int a0, int a1, int b0, int b1, int r) {
         if (hi >= lo) n += hi - lo + 1;
     }
     return n;
+}
+
+// Appends the keep mask of one partial tile: rows q0 .. q1-1 (query tokens) against the key tile
+// whose row segments are `keys`; 128 rows x 4 words, bit k of row r set iff key k is kept for
+// query q0 + r. Per (query, key segment) the kept keys form one run of columns (the predicate's
+// frame and row terms are constant on a segment and the Chebyshev window is an interval of w).
+void tile_mask(const vdit_plan& p, int q0, int q1, const std::vector<Seg>& keys,
+               std::vector<uint32_t>& out) {
+    const size_t base = out.size();
+    out.resize(base + 512, 0u);
+    uint32_t* blk = out.data() + base;
+    const int ft = p.g.grid_h * p.g.grid_w;
+    const bool causal = p.m.kind & VDIT_MASK_BLOCK_CAUSAL;
+    for (int r = 0; r < q1 - q0; ++r) {
+        const int qi = q0 + r, f = qi / ft, rem = qi % ft;
+        const int tq = p.q_start + f, hq = rem / p.g.grid_w, wq = rem % p.g.grid_w;
+        uint32_t* row = blk + 4 * r;
+        for (const Seg& b : keys) {
+            if (b.t < 0) continue;
+            if (causal && b.t / p.m.chunk_frames > tq / p.m.chunk_frames) continue;
+            const long long rad = p.radius[std::abs(tq - b.t)];
+            if (std::abs(hq - b.h) > rad) continue;
+            const long long lo = std::max<long long>(b.wlo, wq - rad);
+            const long long hi = std::min<long long>(b.whi, wq + rad);
+            if (lo > hi) continue;
+            const int k0 = b.off + (int)(lo - b.wlo), k1 = b.off + (int)(hi - b.wlo);
+            for (int wd = k0 >> 5; wd <= k1 >> 5; ++wd) {
+                const int a0 = std::max(k0 - 32 * wd, 0), a1 = std::min(k1 - 32 * wd, 31);
+                row[wd] |= (0xffffffffu >> (31 - a1)) & (0xffffffffu << a0);
+            }
+        }
+    }
 }
 
 }  // namespace
@@ -198,6 +231,8 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
                 p->col_idx.push_back(kt);
                 p->full.push_back(all ? 1 : 0);
                 p->n_full += all;
+                p->mask_of.push_back(all ? -1 : (int)(p->masks.size() / 512));
+                if (!all) tile_mask(*p, q0, q1, kseg[kt], p->masks);
             }
         }
         p->row_ptr[qt + 1] = (int)p->col_idx.size();
@@ -213,10 +248,13 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
             const int ci = i < ie ? p->col_idx[i] : INT_MAX, ck = k < ke ? p->col_idx[k] : INT_MAX;
             const int c = std::min(ci, ck);
             unsigned char f = 0;
-            if (ci == c) { f |= 1 | (p->full[i] ? 2 : 0); ++i; }
-            if (ck == c) { f |= 4 | (p->full[k] ? 8 : 0); ++k; }
+            int m0 = -1, m1 = -1;
+            if (ci == c) { f |= 1 | (p->full[i] ? 2 : 0); m0 = p->mask_of[i]; ++i; }
+            if (ck == c) { f |= 4 | (p->full[k] ? 8 : 0); m1 = p->mask_of[k]; ++k; }
             p->u_col.push_back(c);
             p->u_flags.push_back(f);
+            p->u_mask.push_back(m0);
+            p->u_mask.push_back(m1);
         }
         p->u_row_ptr[b + 1] = (int)p->u_col.size();
     }
@@ -248,6 +286,15 @@ extern "C" int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info) {
     info->uploaded = p->d_buf != nullptr;
     info->kv_splits = p->n_split;
     info->workspace_bytes = (long long)p->ws_bytes;
+    info->mask_bytes = (long long)(sizeof(uint32_t) * p->masks.size());
+    return VDIT_OK;
+}
+
+extern "C" int vdit_plan_export_masks(const vdit_plan* p, int* mask_index, unsigned int* words) {
+    if (!p || (!p->mask_of.empty() && !mask_index) || (!p->masks.empty() && !words))
+        return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or output");
+    if (!p->mask_of.empty()) std::memcpy(mask_index, p->mask_of.data(), sizeof(int) * p->mask_of.size());
+    if (!p->masks.empty()) std::memcpy(words, p->masks.data(), sizeof(uint32_t) * p->masks.size());
     return VDIT_OK;
 }
 
@@ -290,7 +337,7 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     }
     p->n_split = best;
     // one allocation: row_ptr | qtile_order | slot_frame | radius | u_row_ptr | col_idx | full |
-    // u_col | u_flags | unit_order | (split workspace: partial O | partial lse)
+    // u_col | u_flags | unit_order | u_mask | masks | (split workspace: partial O | partial lse)
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     const size_t n_rp = sizeof(int) * p->row_ptr.size(), n_qo = sizeof(int) * p->qtile_order.size();
     const size_t n_sf = sizeof(int) * p->slot_frame.size(), n_ra = sizeof(int) * p->radius.size();
@@ -300,11 +347,13 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t n_uc = sizeof(int) * std::max<size_t>(1, p->u_col.size());
     const size_t n_uf = std::max<size_t>(1, p->u_flags.size());
     const size_t n_uo = sizeof(int) * std::max<size_t>(1, p->unit_order.size());
+    const size_t n_um = sizeof(int) * std::max<size_t>(1, p->u_mask.size());
+    const size_t n_mk = sizeof(uint32_t) * std::max<size_t>(4, p->masks.size());
     const size_t n_wo = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
                                              p->g.heads * p->g.head_dim : 0;
     const size_t n_wl = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads * p->q_tokens : 0;
     const size_t meta = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_urp) + up(n_ci) +
-                        up(n_fu) + up(n_uc) + up(n_uf) + up(n_uo);
+                        up(n_fu) + up(n_uc) + up(n_uf) + up(n_uo) + up(n_um) + up(n_mk);
     const size_t total = meta + up(n_wo) + up(n_wl);
     std::vector<unsigned char> host(total, 0);
     size_t off = 0;
@@ -329,6 +378,10 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     off = o_uf + up(n_uf);
     const size_t o_uo = put(p->unit_order.data(), sizeof(int) * p->unit_order.size());
     off = o_uo + up(n_uo);
+    const size_t o_um = put(p->u_mask.data(), sizeof(int) * p->u_mask.size());
+    off = o_um + up(n_um);
+    const size_t o_mk = put(p->masks.data(), sizeof(uint32_t) * p->masks.size());
+    off = o_mk + up(n_mk);
     if (off != meta) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
     host.resize(meta);  // the workspace is not initialised: every entry is written before use
     void* d = nullptr;
@@ -353,6 +406,8 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     p->d_u_col = reinterpret_cast<const int*>(b + o_uc);
     p->d_u_flags = b + o_uf;
     p->d_unit_order = reinterpret_cast<const int*>(b + o_uo);
+    p->d_u_mask = reinterpret_cast<const int*>(b + o_um);
+    p->d_masks = reinterpret_cast<const uint32_t*>(b + o_mk);
     p->ws_bytes = n_wo + n_wl;
     if (p->n_split > 1) {
         p->d_ws_o = reinterpret_cast<float*>(b + meta);
