@@ -344,6 +344,31 @@ def run_gpu(args, w):
     del xs, ys
     rope_bytes = 2 * q.numel() * 2
 
+    # fused QKV projection + RoPE + cache append (vdit_qkv_rope) of the step's newest frames,
+    # d_model = heads * head_dim (as in Wan2.1), random bf16 weights, its own cache
+    qkv = None
+    dm = g.heads * g.head_dim
+    if dm % 256 == 0:
+        n_tok = w.appends[-1][1] * ft
+        gen = torch.Generator(device="cuda").manual_seed(7)
+        xq = torch.randn(n_tok, dm, device="cuda", generator=gen).to(torch.bfloat16)
+        wq = (torch.randn(3 * dm, dm, device="cuda", generator=gen) * dm ** -0.5).to(torch.bfloat16)
+        qc = vdit.KVCache(g, w.capacity_frames)
+        qo = torch.empty(n_tok, g.heads, g.head_dim, dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            vdit.qkv_rope(xq, wq, g, s_last, qc.k, qc.v, w.capacity_frames, q_out=qo)
+        torch.cuda.synchronize()
+        n_qkv = 10
+        r0.record(stream)
+        for _ in range(n_qkv):
+            vdit.qkv_rope(xq, wq, g, s_last, qc.k, qc.v, w.capacity_frames, q_out=qo)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        qkv_ms = r0.elapsed_time(r1) / n_qkv
+        qkv = {"ms": qkv_ms, "tflops": 2.0 * n_tok * dm * 3 * dm / (qkv_ms * 1e-3) / 1e12,
+               "shape": f"[{n_tok}, {dm}] x [{3 * dm}, {dm}]^T"}
+        del xq, wq, qc, qo
+
     # End to end through the public API: every step copies its Q, K, V from pinned host memory
     # and its O back to pinned host memory. Inputs and outputs are double-buffered and the copies
     # run on their own streams, so step i's copies overlap step i-1's kernels (a stream of denoise
@@ -442,7 +467,8 @@ def run_gpu(args, w):
                 "how": "pairs_per_s: kept (query, key, head) triples per second of attn_fwd; "
                        "query_tokens_per_s: query tokens through the whole step (append + "
                        "attention, all heads) per second; both summed over the replicas"},
-            "gpu_launches": 2 * args.steps,
+            # per step: the append, the attention kernel and, with a key split, the merge
+            "gpu_launches": args.steps * (2 + (1 if info["kv_splits"] > 1 else 0)),
             "clocks": clk,
             "kernels": {
                 "attn_fwd_ms": attn_ms, "attn_fwd_tflops": achieved,
@@ -450,7 +476,12 @@ def run_gpu(args, w):
                 "kv_append_frac_hbm": append_bytes / (app_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "rope3d_apply_ms": rope_ms, "rope3d_apply_gbs": rope_bytes / (rope_ms * 1e-3) / 1e9,
                 "rope3d_apply_frac_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                "hbm_peak_gbs": pk["hbm_gbs"]},
+                "hbm_peak_gbs": pk["hbm_gbs"],
+                "qkv_rope": None if qkv is None else dict(
+                    qkv, frac_of_sustained_peak=qkv["tflops"] / peak,
+                    frac_of_burst_peak=qkv["tflops"] / pk["bf16_tflops"],
+                    how="vdit_qkv_rope: X W^T on tcgen05, RoPE of Q and K, K' and V into the "
+                        "ring cache; 10 launches back to back, not part of the step")},
             "status": status,
         }
         print(json.dumps(line), flush=True)

@@ -203,6 +203,23 @@ VDIT_API int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, const 
                                        const void* v_cache, void* o, float* lse, float scale,
                                        void* stream);
 
+/* Fused QKV projection + 3-D RoPE + KV-cache append ([CRoPE] 2.C: the QKV projections and the
+ * causal RoPE in one kernel; 2.B global time index; 2.A cache of past chunks). For the tokens of
+ * frames start_frame .. start_frame + n_frames - 1 of one chunk (local patch (0, 0) first):
+ *   [Q | K | V] = X W^T in fp32 (tcgen05 tensor cores),
+ *   q_out[n, head, :] = R(pos(n)) Q[n, head, :] (as vdit_rope3d_apply), bf16;
+ *   K' = R(pos(n)) K and V go, bf16, to frame slot (frame mod capacity_frames) of k_cache /
+ *   v_cache in the ring layout of vdit_kv_append.
+ * x: device bf16 [n_frames * grid_h * grid_w, d_model] (row-major); w: device bf16
+ * [3 * heads * head_dim, d_model] (the rows of W_q, then W_k, then W_v: the weight layout of a
+ * linear layer); q_out: device bf16 [tokens, heads, head_dim]. No bias, no normalisation.
+ * Requires heads * head_dim a multiple of 256, d_model a positive multiple of 8, 16-byte aligned
+ * pointers and 1 <= n_frames <= capacity_frames. Builds the RoPE tables on first use per device
+ * and band set (as vdit_rope3d_apply). */
+VDIT_API int vdit_qkv_rope(const vdit_geom* g, const void* x, const void* w, int d_model,
+                           int start_frame, int n_frames, void* q_out, void* k_cache, void* v_cache,
+                           int capacity_frames, void* stream);
+
 /* Reads and clears the current device's kernel status word: *status = VDIT_OK, or
  * VDIT_ERR_TIMEOUT when a bounded wait in a kernel gave up since the last read. Synchronises the
  * device. */

@@ -5,7 +5,8 @@ reference leg of ``bench.py`` import this package. It shares no code with the pr
 (``video_diffusion_transformer_vdit_b200``) and never imports it.
 
 Every function converts numpy arrays to contiguous C buffers and calls the C oracle; the
-arithmetic lives in ``vdit_oracle.c`` (see its header for the pages each step follows).
+arithmetic lives in ``vdit_oracle.c`` (see its header for the pages each step follows), except
+``qkv_project``, whose one step is numpy's float64 matrix product.
 """
 from __future__ import annotations
 
@@ -114,6 +115,22 @@ def rope3d(x: np.ndarray, pos, g: Geometry) -> np.ndarray:
     t, h, w = (_c(p, np.int32) for p in pos)
     lib().vo_rope3d(x, y, n, heads, d, t, h, w, g.band_t, g.band_h, g.band_w, g.theta)
     return y
+
+
+def qkv_project(x: np.ndarray, w: np.ndarray, heads: int, head_dim: int):
+    """The QKV projections ("Accelerating Video Generation Inference with Sequential-Parallel 3D
+    Positional Encoding Using a Global Time Index", section 2.C, names them as the producer of the
+    rotated Q and K): [Q | K | V] = x w^T in float64, x [n, d_model], w [3 * heads * head_dim,
+    d_model] (rows of W_q, W_k, W_v), split into three [n, heads, head_dim] arrays. Its one step
+    is numpy's matrix product (a library primitive); RoPE and the cache write are the separate
+    oracle functions rope3d and kv_append."""
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w, np.float64)
+    hd = heads * head_dim
+    if w.shape != (3 * hd, x.shape[1]):
+        raise ValueError("w must be [3 * heads * head_dim, d_model]")
+    y = x @ w.T
+    return tuple(y[:, i * hd:(i + 1) * hd].reshape(-1, heads, head_dim) for i in range(3))
 
 
 def mask_rows(qpos, kpos, kvalid, m: Mask) -> np.ndarray:

@@ -380,3 +380,37 @@ def test_kv_append_ring_placement():
         slot = f % cap
         assert np.array_equal(vc[:, slot * ft:(slot + 1) * ft], v_all[f * ft:(f + 1) * ft].transpose(1, 0, 2))
         assert np.array_equal(kc[:, slot * ft:(slot + 1) * ft], krot[f * ft:(f + 1) * ft].transpose(1, 0, 2))
+
+
+# ----------------------------------------------------------------------------- QKV projection
+
+def test_qkv_project_hand_worked_example():
+    # 2 tokens, d_model 2, one head of dimension 2; products worked out by hand
+    x = np.array([[1.0, 2.0], [3.0, -1.0]])
+    w = np.array([[1, 0], [0, 1], [2, 1], [1, -1], [0, 3], [1, 1]], dtype=np.float64)
+    q, k, v = oracle.qkv_project(x, w, 1, 2)
+    assert np.array_equal(q[:, 0], [[1, 2], [3, -1]])
+    assert np.array_equal(k[:, 0], [[4, -1], [5, 4]])
+    assert np.array_equal(v[:, 0], [[6, 3], [-3, 2]])
+
+
+def test_qkv_project_identity_weights_split_heads():
+    # W = [I; 2 I; -I] gives Q = x, K = 2 x, V = -x, cut into heads of head_dim channels
+    rng = np.random.default_rng(3)
+    heads, d = 3, 4
+    x = rng.standard_normal((5, heads * d))
+    eye = np.eye(heads * d)
+    q, k, v = oracle.qkv_project(x, np.vstack([eye, 2 * eye, -eye]), heads, d)
+    assert np.array_equal(q, x.reshape(5, heads, d))
+    assert np.array_equal(k, 2 * x.reshape(5, heads, d))
+    assert np.array_equal(v, -x.reshape(5, heads, d))
+
+
+def test_qkv_project_is_linear_in_x():
+    rng = np.random.default_rng(4)
+    x1, x2 = rng.standard_normal((2, 7, 16))
+    w = rng.standard_normal((3 * 8, 16))
+    a = oracle.qkv_project(x1 + 3 * x2, w, 2, 4)
+    b1, b2 = oracle.qkv_project(x1, w, 2, 4), oracle.qkv_project(x2, w, 2, 4)
+    for i in range(3):
+        assert np.allclose(a[i], b1[i] + 3 * b2[i], rtol=1e-12, atol=1e-12)

@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_info.argtypes = [P, ctypes.POINTER(_PlanInfo)]
         L.vdit_plan_export.argtypes = [P, P, P, P]
         L.vdit_plan_export_masks.argtypes = [P, P, P]
+        L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
         L.vdit_plan_destroy.argtypes = [P]
         L.vdit_plan_destroy.restype = None
         L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
@@ -198,6 +199,28 @@ def kv_append(k_cache: torch.Tensor, v_cache: torch.Tensor, g: Geometry, capacit
                                 k.shape[0] // ft, _stream(stream)))
 
 
+def qkv_rope(x: torch.Tensor, w: torch.Tensor, g: Geometry, start_frame: int,
+             k_cache: torch.Tensor, v_cache: torch.Tensor, capacity_frames: int,
+             q_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Fused [Q | K | V] = x w^T, RoPE of Q and K at global frames from start_frame, K' and V into
+    ring slots f mod capacity_frames. x: bf16 [n_frames * frame_tokens, d_model]; w: bf16
+    [3 * heads * head_dim, d_model]. Returns the rotated Q [tokens, heads, head_dim]."""
+    ft = g.frame_tokens
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] % ft:
+        raise ValueError("x must be bf16 [n_frames * frame_tokens, d_model]")
+    hd = g.heads * g.head_dim
+    if w.dtype != torch.bfloat16 or tuple(w.shape) != (3 * hd, x.shape[1]):
+        raise ValueError("w must be bf16 [3 * heads * head_dim, d_model]")
+    q = torch.empty(x.shape[0], g.heads, g.head_dim, dtype=torch.bfloat16, device=x.device) \
+        if q_out is None else q_out
+    gc = g.c()
+    _check(lib().vdit_qkv_rope(ctypes.byref(gc), _dev_ptr(x, "x"), _dev_ptr(w, "w"), x.shape[1],
+                               int(start_frame), x.shape[0] // ft, _dev_ptr(q, "q_out"),
+                               _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+                               int(capacity_frames), _stream(stream)))
+    return q
+
+
 class KVCache:
     """Ring KV cache [heads, capacity_frames * frame_tokens, head_dim] (bf16, zero-filled) plus
     the bookkeeping of which global frames it holds."""
@@ -211,18 +234,33 @@ class KVCache:
         self.first_frame: Optional[int] = None
         self.last_frame: Optional[int] = None
 
-    def append(self, k: torch.Tensor, v: torch.Tensor, start_frame: int, stream=None) -> None:
-        n = k.shape[0] // self.g.frame_tokens
+    def _check_next(self, start_frame: int) -> None:
         if self.last_frame is not None:
             if start_frame > self.last_frame + 1:
                 raise ValueError("append would leave a gap of frames")
             if start_frame < self.first_frame:
                 raise ValueError("frame older than the cache window")
-        kv_append(self.k, self.v, self.g, self.capacity_frames, k, v, start_frame, stream)
+
+    def _note(self, start_frame: int, n: int) -> None:
         last = start_frame + n - 1
         self.last_frame = last if self.last_frame is None else max(self.last_frame, last)
         first = start_frame if self.first_frame is None else self.first_frame
         self.first_frame = max(first, self.last_frame - self.capacity_frames + 1)
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, start_frame: int, stream=None) -> None:
+        """Rotate K at its global frames and write K', V into the ring (vdit_kv_append)."""
+        self._check_next(start_frame)
+        kv_append(self.k, self.v, self.g, self.capacity_frames, k, v, start_frame, stream)
+        self._note(start_frame, k.shape[0] // self.g.frame_tokens)
+
+    def project_append(self, x: torch.Tensor, w: torch.Tensor, start_frame: int,
+                       q_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Fused QKV projection of the chunk x (vdit_qkv_rope): K', V into the ring; returns the
+        rotated Q."""
+        self._check_next(start_frame)
+        q = qkv_rope(x, w, self.g, start_frame, self.k, self.v, self.capacity_frames, q_out, stream)
+        self._note(start_frame, x.shape[0] // self.g.frame_tokens)
+        return q
 
 
 class Plan:

@@ -19,8 +19,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libvdit.so")
-SOURCES = ["plan.cpp", "rope_kv.cu", "attn_fwd.cu"]
-HEADERS = [os.path.join(CSRC, "internal.h"), os.path.join(INCLUDE, "vdit.h")]
+SOURCES = ["plan.cpp", "rope_kv.cu", "attn_fwd.cu", "qkv_rope.cu"]
+HEADERS = [os.path.join(CSRC, "internal.h"), os.path.join(CSRC, "sm100.h"), os.path.join(INCLUDE, "vdit.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-I", INCLUDE, "-I", CSRC]

@@ -30,6 +30,9 @@ int get_rope_tables(const vdit_geom* g, RopeTables* out);
 // Same tables, lookup only (never allocates); an error if they were never built on this device.
 int find_rope_tables(const vdit_geom* g, RopeTables* out);
 
+// Reads and clears the device status word of the fused QKV projection kernel.
+int qkv_status_take(int* out);
+
 }  // namespace vdit
 
 // Plan object (host schedule + optional device copy).
