@@ -33,7 +33,9 @@ from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS  # noqa: E
 
 METRIC = "attention TFLOP/s (unmasked) & % of B200 BF16 peak; RoPE/KV-append GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-MASK_NAMES = {0: "dense", 1: "block-causal", 2: "radial", 3: "block-causal+radial"}
+MASK_NAMES = {0: "dense", 1: "block-causal", 2: "radial", 3: "block-causal+radial",
+              4: "dense candidates + dynamic threshold", 5: "block-causal + dynamic threshold",
+              6: "radial + dynamic threshold", 7: "block-causal+radial + dynamic threshold"}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
 ATTN_SRC = os.path.join(ROOT, "video_diffusion_transformer_vdit_b200", "csrc", "attn_fwd.cu")
 
@@ -76,6 +78,10 @@ def config_of(w, extra=None):
          "q_tokens": w.q_tokens, "kv_tokens": w.kv_tokens, "heads": w.heads,
          "head_dim": w.head_dim, "mask": MASK_NAMES[w.mask_kind], "q_start_frame": w.q_start,
          "batch": 1}
+    if w.mask_kind & 4:
+        c["tau"] = w.tau
+        c["dynamic"] = ("two passes over the candidate tiles (row logit maxima, then attention "
+                        "over candidates within tau of them); FLOPs count 4*d per candidate pair")
     if extra:
         c.update(extra)
     return c
@@ -123,7 +129,10 @@ class OracleArm:
         qp = tuple(p[rows] for p in self.qpos)
         q = o.rope3d(synth.bf16_bits_to_f64(self.qbits[rows]), qp, self.og)
         m = o.mask_rows(qp, self.kpos, self.kvalid, self.om)
-        o.attention(q, self.kt, self.vt, m, w.scale)
+        if w.mask_kind & 4:
+            o.attention_dynamic(q, self.kt, self.vt, m, w.scale, w.tau)
+        else:
+            o.attention(q, self.kt, self.vt, m, w.scale)
         dt = time.perf_counter() - t0
         return dt, 4.0 * w.head_dim * w.heads * int(m.sum()), n_rows
 
@@ -258,7 +267,7 @@ def run_gpu(args, w):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     g = vdit.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, w.bands, w.theta)
-    m = vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+    m = vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, w.tau)
     ft = w.frame_tokens
 
     def bf16(bits):

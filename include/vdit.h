@@ -67,6 +67,7 @@ enum {
 #define VDIT_MASK_DENSE 0
 #define VDIT_MASK_BLOCK_CAUSAL 1
 #define VDIT_MASK_RADIAL 2
+#define VDIT_MASK_DYNAMIC 4
 
 #define VDIT_TILE 128         /* query and key tile edge of the schedule and of the kernel   */
 #define VDIT_MAX_FRAME 16383  /* largest global frame index the RoPE tables cover           */
@@ -89,13 +90,19 @@ typedef struct vdit_geom {
  *   RADIAL ([DR] sec. 2, static-ratio mode): with dt = |t_q - t_k| and
  *     d = max(|h_q - h_k|, |w_q - w_k|) (Chebyshev patch distance), kept iff
  *     (lambda > 0 and dt mod lambda == 0) or d <= w0 * 2^(-gamma_shift * dt).
- *   Both bits: AND of the two. 0: dense. Keys in never-written cache slots are never kept. */
+ *   Both bits: AND of the two. 0: dense. Keys in never-written cache slots are never kept.
+ *   DYNAMIC ([DR] sec. 2, dynamic-threshold mode; combined with any of the above, which then
+ *     form the candidate set): the pre-softmax logits are the importance proxies. With
+ *     z = scale * q . k over a query row's candidates and z_max their maximum, a candidate is
+ *     kept iff z >= z_max - tau (tau > 0): the threshold adapts to each row. The attention
+ *     kernel then makes two passes over the candidate tiles (logit maxima, then the softmax). */
 typedef struct vdit_mask {
     int kind;          /* VDIT_MASK_* bits */
     int chunk_frames;  /* >= 1 when BLOCK_CAUSAL (Wan2.1 causal decode: 3) */
     long long w0;      /* >= 0 when RADIAL (52 on a 30 x 52 grid) */
     int gamma_shift;   /* >= 0; gamma = 2^-gamma_shift (1 -> gamma = 1/2) */
     int lambda;        /* >= 0; 0 disables the long-range frames (8) */
+    double tau;        /* > 0 when DYNAMIC: logit margin below the row maximum (natural log) */
 } vdit_mask;
 
 /* Opaque attention schedule: the non-empty 128 x 128 (query x key) tiles of the mask. */

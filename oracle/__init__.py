@@ -155,6 +155,33 @@ def attention(q, k, v, mask, scale: float):
     return o, lse
 
 
+def attention_dynamic(q, k, v, cand, scale: float, tau: float):
+    """Attention in the dynamic-threshold mode of "DynamicRad: Content-Adaptive Sparse Attention
+    for Long Video Diffusion", section 2: the pre-softmax logits serve as importance proxies and
+    an adaptive threshold filters the structured candidate set. Reading taken: per head and query
+    row, with z = scale * q . k over the row's candidates (cand [nq, nk], from mask_rows) and
+    z_max their maximum, a candidate is kept iff z >= z_max - tau; then masked softmax attention
+    over the kept keys. The logits are numpy float64 matrix products (a library primitive), the
+    attention is the C oracle's. Returns (o [nq, heads, D], lse [heads, nq], keep [heads, nq, nk])."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    cand = np.asarray(cand).astype(bool)
+    nq, heads, d = q.shape
+    o = np.empty((nq, heads, d))
+    lse = np.empty((heads, nq))
+    keep = np.zeros((heads,) + cand.shape, bool)
+    for h in range(heads):
+        z = scale * (q[:, h] @ k[:, h].T)
+        zc = np.where(cand, z, -np.inf)
+        zmax = zc.max(axis=1, keepdims=True) if cand.shape[1] else np.full((nq, 1), -np.inf)
+        keep[h] = cand & (z >= zmax - tau)
+        oh, lh = attention(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], keep[h].astype(np.uint8), scale)
+        o[:, h] = oh[:, 0]
+        lse[h] = lh[0]
+    return o, lse, keep
+
+
 def tiles(qpos, kpos, kvalid, m: Mask, tile: int = 128):
     """(row_ptr, col_idx, full, kept_pairs) of the explicit mask's tile list."""
     tq, hq, wq = (_c(p, np.int32) for p in qpos)

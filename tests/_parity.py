@@ -33,7 +33,7 @@ def ogeom(w, heads=None):
 
 
 def mask(w):
-    return vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+    return vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, w.tau)
 
 
 def omask(w):
@@ -85,6 +85,10 @@ def run_oracle(w, q, k, v, rows, heads):
     qpos = tuple(p[rows] for p in qpos_all)
     qrot = oracle.rope3d(synth.bf16_bits_to_f64(q[rows][:, hs]), qpos, og)
     m = oracle.mask_rows(qpos, kpos, kvalid, omask(w))
+    if w.mask_kind & 4:  # dynamic threshold over the candidates of the static bits
+        o, lse, _ = oracle.attention_dynamic(qrot, kc.transpose(1, 0, 2), vc.transpose(1, 0, 2), m,
+                                             w.scale, w.tau)
+        return o, lse
     return oracle.attention(qrot, kc.transpose(1, 0, 2), vc.transpose(1, 0, 2), m, w.scale)
 
 

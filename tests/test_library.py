@@ -27,7 +27,7 @@ def _geom(w):
 
 
 def _mask(w):
-    return vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+    return vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, w.tau)
 
 
 def _oracle_tiles(grid_h, grid_w, q_start, q_frames, cap, first, last, mask_kind, chunk, w0, g, lam):

@@ -414,3 +414,60 @@ def test_qkv_project_is_linear_in_x():
     b1, b2 = oracle.qkv_project(x1, w, 2, 4), oracle.qkv_project(x2, w, 2, 4)
     for i in range(3):
         assert np.allclose(a[i], b1[i] + 3 * b2[i], rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- dynamic threshold
+
+def test_dynamic_threshold_hand_worked_example():
+    # one query, four candidate keys with logits 2.0, 1.0, -0.5, 1.9 (scale 1, d = 1): tau 0.5
+    # keeps {0, 3}, tau 1.2 keeps {0, 1, 3}, and a masked-out key is never kept
+    q = np.ones((1, 1, 1))
+    k = np.array([2.0, 1.0, -0.5, 1.9, 5.0]).reshape(5, 1, 1)
+    v = np.arange(5, dtype=np.float64).reshape(5, 1, 1)
+    cand = np.array([[1, 1, 1, 1, 0]], np.uint8)
+    _, _, keep = oracle.attention_dynamic(q, k, v, cand, 1.0, 0.5)
+    assert keep[0, 0].tolist() == [True, False, False, True, False]
+    o, lse, keep = oracle.attention_dynamic(q, k, v, cand, 1.0, 1.2)
+    assert keep[0, 0].tolist() == [True, True, False, True, False]
+    w = np.exp(np.array([2.0, 1.0, 1.9]))
+    assert np.isclose(o[0, 0, 0], (w * np.array([0.0, 1.0, 3.0])).sum() / w.sum(), rtol=1e-14)
+    assert np.isclose(lse[0, 0], np.log(w.sum()), rtol=1e-14)
+
+
+def _rand_case(seed, nq=6, nk=40, heads=2, d=8):
+    rng = np.random.default_rng(seed)
+    q, k, v = rng.standard_normal((nq, heads, d)), rng.standard_normal((nk, heads, d)), rng.standard_normal((nk, heads, d))
+    cand = (rng.random((nq, nk)) < 0.6).astype(np.uint8)
+    cand[0] = 0  # a row without candidates
+    return q, k, v, cand
+
+
+def test_dynamic_threshold_large_tau_equals_the_candidate_mask():
+    q, k, v, cand = _rand_case(1)
+    o, lse, keep = oracle.attention_dynamic(q, k, v, cand, 0.35, 1e9)
+    o2, lse2 = oracle.attention(q, k, v, cand, 0.35)
+    assert (keep == cand.astype(bool)[None]).all()
+    assert np.allclose(o, o2, atol=1e-13) and np.allclose(lse[:, 1:], lse2[:, 1:], atol=1e-13)
+    assert (o[0] == 0).all() and np.isneginf(lse[:, 0]).all()
+
+
+def test_dynamic_threshold_tiny_tau_keeps_only_the_argmax():
+    q, k, v, cand = _rand_case(2)
+    o, _, keep = oracle.attention_dynamic(q, k, v, cand, 0.35, 1e-12)
+    for h in range(2):
+        z = np.where(cand.astype(bool), 0.35 * q[:, h] @ k[:, h].T, -np.inf)
+        for r in range(1, z.shape[0]):
+            j = int(np.argmax(z[r]))
+            assert keep[h, r].sum() == 1 and keep[h, r, j]
+            assert np.allclose(o[r, h], v[j, h], atol=1e-13)
+
+
+def test_dynamic_threshold_kept_sets_grow_with_tau():
+    q, k, v, cand = _rand_case(3)
+    prev = None
+    for tau in (0.1, 0.5, 1.0, 2.0, 8.0):
+        _, _, keep = oracle.attention_dynamic(q, k, v, cand, 0.35, tau)
+        assert (keep <= cand.astype(bool)[None]).all()
+        if prev is not None:
+            assert (prev <= keep).all()
+        prev = keep

@@ -39,6 +39,7 @@ ERR_NOT_UPLOADED = -6
 MASK_DENSE = 0
 MASK_BLOCK_CAUSAL = 1
 MASK_RADIAL = 2
+MASK_DYNAMIC = 4
 TILE = 128
 
 
@@ -56,7 +57,7 @@ class _Geom(ctypes.Structure):
 
 class _Mask(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("chunk_frames", ctypes.c_int), ("w0", ctypes.c_longlong),
-                ("gamma_shift", ctypes.c_int), ("lambda_", ctypes.c_int)]
+                ("gamma_shift", ctypes.c_int), ("lambda_", ctypes.c_int), ("tau", ctypes.c_double)]
 
 
 class _PlanInfo(ctypes.Structure):
@@ -146,12 +147,13 @@ class Geometry:
 
 @dataclass(frozen=True)
 class Mask:
-    """Mask kind bits (MASK_BLOCK_CAUSAL | MASK_RADIAL) and parameters."""
+    """Mask kind bits (MASK_BLOCK_CAUSAL | MASK_RADIAL | MASK_DYNAMIC) and parameters."""
     kind: int = MASK_DENSE
     chunk_frames: int = 3
     w0: int = 52
     gamma_shift: int = 1
     lam: int = 8
+    tau: float = 0.0
 
     @staticmethod
     def dense() -> "Mask":
@@ -167,7 +169,7 @@ class Mask:
         return Mask(kind, chunk_frames=chunk_frames or 3, w0=w0, gamma_shift=gamma_shift, lam=lam)
 
     def c(self) -> _Mask:
-        return _Mask(self.kind, self.chunk_frames, self.w0, self.gamma_shift, self.lam)
+        return _Mask(self.kind, self.chunk_frames, self.w0, self.gamma_shift, self.lam, float(self.tau))
 
 
 def rope3d_apply(x: torch.Tensor, g: Geometry, start_frame: int,

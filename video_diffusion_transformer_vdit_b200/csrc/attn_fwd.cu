@@ -138,6 +138,7 @@ struct AttnArgs {
     int grid_h, grid_w;
     int q_start;
     float scale_log2;
+    float tau_log2;        // dynamic-threshold mode: tau * log2(e)
 };
 
 // ------------------------------------------------------------------------------ PTX wrappers
@@ -207,7 +208,7 @@ __device__ __forceinline__ uint4 rope_chunk(uint4 in, int pp0, int t, int h, int
 
 // ------------------------------------------------------------------------------ the kernel
 
-template <int D>
+template <int D, bool DYN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
@@ -236,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // same tile makes them request the same 32 KiB of K / V from the same L2 slices at once.
     const int rot = n_ent > 0 ? (int)(((unsigned)blockIdx.x * 97u + (unsigned)blockIdx.y * 31u) % (unsigned)n_ent) : 0;
     auto entry = [&](int i) { const int e = i + rot; return e >= n_ent ? e - n_ent : e; };
+    // visits of the entries: the dynamic-threshold mode walks the list twice
+    const int n_v = DYN ? 2 * n_ent : n_ent;
     const int ft = a.grid_h * a.grid_w;
 
     if (threadIdx.x == 0) {
@@ -297,9 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qi = (qb * kQTiles + h) * kTile + row;
         const float c = a.scale_log2;
         float m = -INFINITY, l = 0.f;  // running max (raw score units) and sum
-        int cnt = 0;
+        int cnt = 0;                   // score tiles read
+        int npv_dyn = 0;               // dynamic-threshold mode: P tiles stored (else == cnt)
         bool ok = true;
-        for (int j = 0; j < n_ent; ++j) {
+        for (int j = 0; j < n_v; ++j) {
+            // dynamic-threshold mode: pass 0 (j < n_ent) only takes the row maxima of the
+            // candidates' logits; pass 1 keeps a candidate iff its logit is within tau of it
+            const bool pass0 = DYN && j < n_ent, pass1 = DYN && j >= n_ent;
+            const int npv = DYN ? npv_dyn : cnt;
             const int s = j % kStages;
             if (!warp_wait(BAR(B_IFULL + s), (j / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
             const uint8_t* info = smem + L::OFF_KINFO + s * kKinfoBytes;
@@ -330,17 +338,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sv[jj] = ((mw[jj >> 5] >> (jj & 31)) & 1u) ? sv[jj] : -INFINITY;
             }
             mbar_arrive(BAR(B_IEMPTY + s));
-            // row max: 8 independent chains of 3-input max
-            float mx[8];
+            float m_tile = -INFINITY;
+            if (pass1) {
+                // the row maximum m is final: drop candidates more than tau below it
+                const float thr = m * c - a.tau_log2;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+                for (int jj = 0; jj < 128; ++jj) sv[jj] = sv[jj] * c >= thr ? sv[jj] : -INFINITY;
+            } else {
+                // row max: 8 independent chains of 3-input max
+                float mx[8];
 #pragma unroll
-            for (int jj = 8; jj < 128; jj += 16) {
+                for (int i = 0; i < 8; ++i) mx[i] = sv[i];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], sv[jj + 2 * i], sv[jj + 2 * i + 1]);
+                for (int jj = 8; jj < 128; jj += 16) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], sv[jj + 2 * i], sv[jj + 2 * i + 1]);
+                }
+                m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             }
-            const float m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
-                                      fmaxf(mx[6], mx[7]));
+            if (pass0) {
+                m = fmaxf(m, m_tile);
+                ++cnt;
+                continue;
+            }
             const float m_new = fmaxf(m, m_tile);
             const bool resc = (m_new - m) * c > kRescaleTau;
             float alpha = 1.f;
@@ -351,11 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mc = (m == -INFINITY) ? 0.f : m * c;
             // PV_h of the previous tile must have completed: it reads P_h (overwritten below)
             // and accumulates into O_h (rescaled below)
-            if (cnt > 0) {
-                if (!warp_wait(BAR(B_PVDONE + h), (cnt - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+            if (npv > 0) {
+                if (!warp_wait(BAR(B_PVDONE + h), (npv - 1) & 1, abort_flag, a.status)) { ok = false; break; }
                 tc_fence_after();
             }
-            if (cnt > 0 && __any_sync(0xffffffffu, resc)) {
+            if (npv > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
                 for (int q4 = 0; q4 < D / 32; ++q4) {
                     uint32_t orow[32];
@@ -408,9 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(BAR(B_PFULL + h));
             ++cnt;
+            if (DYN) ++npv_dyn;
         }
-        if (ok && cnt > 0) {
-            if (!warp_wait(BAR(B_PVDONE + h), (cnt - 1) & 1, abort_flag, a.status)) ok = false;
+        const int n_pv = DYN ? npv_dyn : cnt;
+        if (ok && n_pv > 0) {
+            if (!warp_wait(BAR(B_PVDONE + h), (n_pv - 1) & 1, abort_flag, a.status)) ok = false;
         }
         // every thread of the group reaches this barrier (aborted or not); any failure skips
         // the epilogue of the whole group
@@ -432,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
             for (int q4 = 0; q4 < D / 32; ++q4) {
                 uint32_t orow[32];
-                if (cnt > 0) {
+                if (n_pv > 0) {
                     tmem_ld32(t_o + q4 * 32, orow);
                     tmem_ld_wait(orow);
                 } else {
@@ -458,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
             for (int q4 = 0; q4 < D / 32; ++q4) {
                 uint32_t orow[32];
-                if (cnt > 0) {
+                if (n_pv > 0) {
                     tmem_ld32(t_o + q4 * 32, orow);
                     tmem_ld_wait(orow);
                 } else {
@@ -500,25 +522,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == kWarpTMA) {
         // ------------------------------------------------------------------ producer
-        int issued = 0;
-        int mask_it[kStages];  // per stage: last entry whose mask copies were issued (drain)
-#pragma unroll
-        for (int i = 0; i < kStages; ++i) mask_it[i] = -1;
-        int kt_next = n_ent > 0 ? __ldg(a.u_col + u_begin + entry(0)) : 0;
-        int fl_next = n_ent > 0 ? __ldg(a.u_flags + u_begin + entry(0)) : 0;
-        int mk0_next = n_ent > 0 ? __ldg(a.u_mask + 2 * (u_begin + entry(0))) : -1;
-        int mk1_next = n_ent > 0 ? __ldg(a.u_mask + 2 * (u_begin + entry(0)) + 1) : -1;
-        for (int it = 0; it < (a.skip_loads ? 0 : n_ent); ++it) {
+        // Pass 0 of the dynamic-threshold mode visits the entries for the logit maxima only (K
+        // and masks); the attention pass loads K, masks and V. it: K / mask sequence number,
+        // jv: V sequence number.
+        // for the drain: last K and V sequence numbers issued, and per stage the last sequence
+        // number whose masks were copied (scalars: the stage index is not a compile-time value)
+        static_assert(kStages == 2, "drain bookkeeping assumes two stages");
+        int k_last = -1, v_last = -1, mask_it0 = -1, mask_it1 = -1;
+        auto load_entry = [&](int v, int& kt, int& fl, int& m0, int& m1) {
+            const int e = u_begin + entry(DYN && v >= n_ent ? v - n_ent : v);
+            kt = __ldg(a.u_col + e);
+            fl = __ldg(a.u_flags + e);
+            m0 = __ldg(a.u_mask + 2 * e);
+            m1 = __ldg(a.u_mask + 2 * e + 1);
+        };
+        int kt_next = 0, fl_next = 0, mk0_next = -1, mk1_next = -1;
+        if (n_ent > 0) load_entry(0, kt_next, fl_next, mk0_next, mk1_next);
+        for (int it = 0; it < (a.skip_loads ? 0 : n_v); ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) - 1) & 1u;
             const int kt = kt_next, flags = fl_next, mk0 = mk0_next, mk1 = mk1_next;
-            if (it + 1 < n_ent) {  // next entry's tile, flags and masks, loaded while this one waits
-                const int e1 = u_begin + entry(it + 1);
-                kt_next = __ldg(a.u_col + e1);
-                fl_next = __ldg(a.u_flags + e1);
-                mk0_next = __ldg(a.u_mask + 2 * e1);
-                mk1_next = __ldg(a.u_mask + 2 * e1 + 1);
-            }
+            // next entry's tile, flags and masks, loaded while this one waits
+            if (it + 1 < n_v) load_entry(it + 1, kt_next, fl_next, mk0_next, mk1_next);
             if (it >= kStages && !warp_wait(BAR(B_KEMPTY + s), ph, abort_flag, a.status)) break;
             if (lane == 0) {
                 mbar_expect_tx(BAR(B_KFULL + s), kTileBytes);
@@ -526,15 +551,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int sl = 0; sl < L::kSlabs; ++sl)
                     tma_load_3d(dst + sl * kSlabBytes, &tmap_k, BAR(B_KFULL + s), 64 * sl, kt * kTile, head);
+                k_last = it;
             }
-            issued = it * 2 + 1;
             if (it >= kStages && !warp_wait(BAR(B_IEMPTY + s), ph, abort_flag, a.status)) break;
             uint8_t* info = smem + L::OFF_KINFO + s * kKinfoBytes;
             if (lane == 0) {
                 reinterpret_cast<int*>(info)[0] = kt;
                 reinterpret_cast<int*>(info)[1] = flags;
-            }
-            if (lane == 0) {
                 // keep masks of the partial query tiles of this entry (2 KiB each), else a plain
                 // arrival: the header above is published by the arrive's release either way
                 const uint32_t nbytes = (mk0 >= 0 ? kMaskBlockBytes : 0u) + (mk1 >= 0 ? kMaskBlockBytes : 0u);
@@ -546,41 +569,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mk1 >= 0)
                         bulk_load(dst + kMaskBlockBytes, a.masks + (size_t)mk1 * (kMaskBlockBytes / 4),
                                   kMaskBlockBytes, BAR(B_IFULL + s));
-                    mask_it[s] = it;
+                    if (s == 0) mask_it0 = it; else mask_it1 = it;
                 } else {
                     mbar_arrive(BAR(B_IFULL + s));
                 }
             }
             __syncwarp();
-            if (it >= kStages && !warp_wait(BAR(B_VEMPTY + s), ph, abort_flag, a.status)) break;
+            if (DYN && it < n_ent) continue;  // logit pass: no V
+            const int jv = DYN ? it - n_ent : it;
+            const int sv = jv % kStages;
+            if (jv >= kStages &&
+                !warp_wait(BAR(B_VEMPTY + sv), (uint32_t)((jv / kStages) - 1) & 1u, abort_flag, a.status))
+                break;
             if (lane == 0) {
-                mbar_expect_tx(BAR(B_VFULL + s), kTileBytes);
-                const uint32_t dst = sbase + L::OFF_V + s * kTileBytes;
+                mbar_expect_tx(BAR(B_VFULL + sv), kTileBytes);
+                const uint32_t dst = sbase + L::OFF_V + sv * kTileBytes;
 #pragma unroll
                 for (int sl = 0; sl < L::kSlabs; ++sl)
-                    tma_load_3d(dst + sl * kSlabBytes, &tmap_v, BAR(B_VFULL + s), 64 * sl, kt * kTile, head);
+                    tma_load_3d(dst + sl * kSlabBytes, &tmap_v, BAR(B_VFULL + sv), 64 * sl, kt * kTile, head);
+                v_last = jv;
             }
-            issued = it * 2 + 2;
             __syncwarp();
         }
-        // drain: every TMA this warp issued must have landed before the CTA may exit
-        if (*abort_flag) {
-#pragma unroll
-            for (int st = 0; st < kStages; ++st) {
-                if (mask_it[st] < 0) continue;
+        // drain: every copy this warp issued must have landed before the CTA may exit
+        if (*abort_flag && lane == 0) {
+            auto drain = [&](int bar, int seq) {
+                if (seq < 0) return;
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(BAR(B_IFULL + st), (uint32_t)(mask_it[st] / kStages) & 1u) &&
+                while (!mbar_try_wait(BAR(bar + seq % kStages), (uint32_t)(seq / kStages) & 1u) &&
                        globaltimer() - t0 < kWaitLimitNs) {
                 }
-            }
-            for (int jn = (issued - 2 * kStages > 0 ? issued - 2 * kStages : 0); jn < issued; ++jn) {
-                const int it = jn >> 1, s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                const int b = (jn & 1) ? B_VFULL + s : B_KFULL + s;
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(BAR(b), ph) && globaltimer() - t0 < kWaitLimitNs) {
-                }
-            }
+            };
+            drain(B_IFULL, mask_it0);
+            drain(B_IFULL, mask_it1);
+            for (int x = k_last - kStages + 1; x <= k_last; ++x) drain(B_KFULL, x);
+            for (int x = v_last - kStages + 1; x <= v_last; ++x) drain(B_VFULL, x);
         }
     } else if (warp == kWarpMMA || warp == kWarpPV) {
         // ------------------------------------------------------------------ MMA issuers
@@ -602,17 +625,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const unsigned char* fl = a.u_flags + u_begin;
             // tile flags are read two entries ahead so the global-load latency never sits
             // between a completed barrier and the next MMA issue
-            int f_cur = __ldg(fl + entry(0));
-            int f_nxt = n_ent > 1 ? __ldg(fl + entry(1)) : 0;
+            auto flag_of = [&](int v) { return (int)__ldg(fl + entry(DYN && v >= n_ent ? v - n_ent : v)); };
+            int f_cur = flag_of(0);
+            int f_nxt = n_ent > 1 || DYN ? flag_of(1 % n_v) : 0;
             if (s_role) {
                 // S_h(j) = Q_h K(j)^T into the shared S columns, in list order, each after the
                 // previous score tile has been read out of TMEM by its softmax group
                 int ns = 0;
-                for (int j = 0; j < n_ent; ++j) {
+                for (int j = 0; j < n_v; ++j) {  // both passes in the dynamic-threshold mode
                     const int s = j % kStages;
                     const int f = f_cur;
                     f_cur = f_nxt;
-                    f_nxt = j + 2 < n_ent ? __ldg(fl + entry(j + 2)) : 0;
+                    f_nxt = j + 2 < n_v ? flag_of(j + 2) : 0;
                     if (!wait_bounded(BAR(B_KFULL + s), (j / kStages) & 1, abort_flag, a.status)) break;
                     tc_fence_after();
                     const uint64_t k0 = dk0 + (s ? kTileDesc : 0);
@@ -771,24 +795,13 @@ int* status_ptr() {
     return static_cast<int*>(p);
 }
 
-}  // namespace
-
-extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache,
-                                 const void* v_cache, void* o, float* lse, float scale,
-                                 void* stream) {
+// Tensor maps, arguments and launches of one forward pass (the attention kernel for the plan's
+// head_dim and mode, then the split merge when the plan splits key ranges). ws_o / ws_lse: the
+// split scratch (unused without a split).
+int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
+                     void* o, float* lse, float scale, float* ws_o, float* ws_lse,
+                     const vdit::RopeTables& tabs, cudaStream_t st, int dev) {
     using vdit::fail;
-    if (!p) return fail(VDIT_ERR_INVALID_ARG, "NULL plan");
-    if (!p->d_buf) return fail(VDIT_ERR_NOT_UPLOADED, "plan not uploaded (vdit_plan_upload)");
-    if (!q || !k_cache || !v_cache || !o) return fail(VDIT_ERR_INVALID_ARG, "NULL tensor");
-    auto al = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
-    if (!al(q) || !al(k_cache) || !al(v_cache) || !al(o) || (reinterpret_cast<uintptr_t>(lse) & 3))
-        return fail(VDIT_ERR_MISALIGNED, "tensor not aligned");
-    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(VDIT_ERR_INVALID_ARG, "scale must be > 0");
-    int dev = 0;
-    if (int rc = vdit::cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
-    if (dev != p->device) return fail(VDIT_ERR_INVALID_ARG, "plan was uploaded to another device");
-    vdit::RopeTables tabs;
-    if (int rc = vdit::get_rope_tables(&p->g, &tabs)) return rc;
     CUtensorMap mk, mv;
     const int d = p->g.head_dim;
     if (int rc = make_cache_map(&mk, k_cache, p->kv_tokens, p->g.heads, d)) return rc;
@@ -796,13 +809,12 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_fwd_kernel<128>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)Layout<128>::kSmemBytes);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(attn_fwd_kernel<64>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)Layout<64>::kSmemBytes);
+        const void* fns[4] = {(const void*)attn_fwd_kernel<128, false>, (const void*)attn_fwd_kernel<64, false>,
+                              (const void*)attn_fwd_kernel<128, true>, (const void*)attn_fwd_kernel<64, true>};
+        const int bytes[4] = {(int)Layout<128>::kSmemBytes, (int)Layout<64>::kSmemBytes,
+                              (int)Layout<128>::kSmemBytes, (int)Layout<64>::kSmemBytes};
+        for (int i = 0; i < 4 && attr_err == cudaSuccess; ++i)
+            attr_err = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]);
     });
     if (int rc = vdit::cuda_check(attr_err, "cudaFuncSetAttribute")) return rc;
     int* status = status_ptr();
@@ -813,8 +825,8 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.u_col = p->d_u_col;
     a.u_flags = p->d_u_flags;
     a.unit_order = p->d_unit_order;
-    a.ws_o = p->d_ws_o;
-    a.ws_lse = p->d_ws_lse;
+    a.ws_o = ws_o;
+    a.ws_lse = ws_lse;
     a.n_qb = p->n_qb;
     a.n_split = p->n_split;
     a.masks = p->d_masks;
@@ -837,28 +849,55 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     a.grid_w = p->g.grid_w;
     a.q_start = p->q_start;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    a.tau_log2 = (float)(p->m.tau * 1.4426950408889634);
+    const bool dyn = p->m.kind & VDIT_MASK_DYNAMIC;
     dim3 grid(p->n_qb * p->n_split, p->g.heads);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128)
-        attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
+    if (d == 128 && !dyn)
+        attn_fwd_kernel<128, false><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
+    else if (d == 64 && !dyn)
+        attn_fwd_kernel<64, false><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
+    else if (d == 128)
+        attn_fwd_kernel<128, true><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
     else
-        attn_fwd_kernel<64><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
+        attn_fwd_kernel<64, true><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
+    if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
     if (p->n_split > 1) {
-        if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
         int sms = 148;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const long long rows = (long long)p->q_tokens * p->g.heads;
         const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)sms * 8);
         auto* ob = static_cast<__nv_bfloat16*>(o);
         if (d == 128)
-            split_combine_kernel<128><<<blocks, 256, 0, st>>>(p->d_ws_o, p->d_ws_lse, p->n_split,
-                                                              p->q_tokens, p->g.heads, ob, lse);
+            split_combine_kernel<128><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
+                                                              p->g.heads, ob, lse);
         else
-            split_combine_kernel<64><<<blocks, 256, 0, st>>>(p->d_ws_o, p->d_ws_lse, p->n_split,
-                                                             p->q_tokens, p->g.heads, ob, lse);
+            split_combine_kernel<64><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
+                                                             p->g.heads, ob, lse);
         return vdit::cuda_check(cudaGetLastError(), "split merge launch");
     }
-    return vdit::cuda_check(cudaGetLastError(), "attention kernel launch");
+    return VDIT_OK;
+}
+
+}  // namespace
+
+extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache,
+                                 const void* v_cache, void* o, float* lse, float scale,
+                                 void* stream) {
+    using vdit::fail;
+    if (!p) return fail(VDIT_ERR_INVALID_ARG, "NULL plan");
+    if (!p->d_buf) return fail(VDIT_ERR_NOT_UPLOADED, "plan not uploaded (vdit_plan_upload)");
+    if (!q || !k_cache || !v_cache || !o) return fail(VDIT_ERR_INVALID_ARG, "NULL tensor");
+    auto al = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
+    if (!al(q) || !al(k_cache) || !al(v_cache) || !al(o) || (reinterpret_cast<uintptr_t>(lse) & 3))
+        return fail(VDIT_ERR_MISALIGNED, "tensor not aligned");
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(VDIT_ERR_INVALID_ARG, "scale must be > 0");
+    int dev = 0;
+    if (int rc = vdit::cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    if (dev != p->device) return fail(VDIT_ERR_INVALID_ARG, "plan was uploaded to another device");
+    vdit::RopeTables tabs;
+    if (int rc = vdit::get_rope_tables(&p->g, &tabs)) return rc;
+    return launch_attention(p, q, k_cache, v_cache, o, lse, scale, p->d_ws_o, p->d_ws_lse, tabs,
+                            static_cast<cudaStream_t>(stream), dev);
 }
 
 extern "C" void vdit_debug_skip_loads(int on) { g_skip_loads.store(on ? 1 : 0); }
@@ -949,76 +988,10 @@ extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, cons
     if (int rc = noalloc_scratch_address(dev, &scratch)) return rc;
     vdit::RopeTables tabs;
     if (int rc = vdit::find_rope_tables(&p->g, &tabs)) return rc;
-    CUtensorMap mk, mv;
-    if (int rc = make_cache_map(&mk, k_cache, p->kv_tokens, p->g.heads, d)) return rc;
-    if (int rc = make_cache_map(&mv, v_cache, p->kv_tokens, p->g.heads, d)) return rc;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_fwd_kernel<128>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)Layout<128>::kSmemBytes);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(attn_fwd_kernel<64>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)Layout<64>::kSmemBytes);
-    });
-    if (int rc = vdit::cuda_check(attr_err, "cudaFuncSetAttribute")) return rc;
-    int* status = status_ptr();
-    if (!status) return fail(VDIT_ERR_CUDA, "cannot resolve status word");
-
     float* ws_o = p->n_split > 1 ? static_cast<float*>(scratch) : nullptr;
     float* ws_lse = p->n_split > 1
                         ? reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + o_bytes_al)
                         : nullptr;
-    AttnArgs a{};
-    a.u_row_ptr = p->d_u_row_ptr;
-    a.u_col = p->d_u_col;
-    a.u_flags = p->d_u_flags;
-    a.unit_order = p->d_unit_order;
-    a.ws_o = ws_o;
-    a.ws_lse = ws_lse;
-    a.n_qb = p->n_qb;
-    a.n_split = p->n_split;
-    a.masks = p->d_masks;
-    a.u_mask = p->d_u_mask;
-    a.q = static_cast<const uint4*>(q);
-    a.o = static_cast<uint4*>(o);
-    a.lse = lse;
-    a.tt = static_cast<const float2*>(tabs.t);
-    a.th = static_cast<const float2*>(tabs.h);
-    a.tw = static_cast<const float2*>(tabs.w);
-    a.status = status;
-    a.bt2 = p->g.band_t / 2;
-    a.bh2 = p->g.band_h / 2;
-    a.bw2 = p->g.band_w / 2;
-    a.q_tokens = p->q_tokens;
-    a.kv_tokens = p->kv_tokens;
-    a.heads = p->g.heads;
-    a.grid_h = p->g.grid_h;
-    a.grid_w = p->g.grid_w;
-    a.q_start = p->q_start;
-    a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    dim3 grid(p->n_qb * p->n_split, p->g.heads);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128)
-        attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
-    else
-        attn_fwd_kernel<64><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
-    if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
-    if (p->n_split > 1) {
-        int sms = 148;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const long long rows = (long long)p->q_tokens * p->g.heads;
-        const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)sms * 8);
-        auto* ob = static_cast<__nv_bfloat16*>(o);
-        if (d == 128)
-            split_combine_kernel<128><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
-                                                              p->g.heads, ob, lse);
-        else
-            split_combine_kernel<64><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
-                                                             p->g.heads, ob, lse);
-        return vdit::cuda_check(cudaGetLastError(), "split merge launch");
-    }
-    return VDIT_OK;
+    return launch_attention(p, q, k_cache, v_cache, o, lse, scale, ws_o, ws_lse, tabs,
+                            static_cast<cudaStream_t>(stream), dev);
 }

@@ -146,8 +146,10 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
     *out = nullptr;
     if (int rc = vdit::check_geom(g)) return rc;
     if (!m) return fail(VDIT_ERR_INVALID_ARG, "mask is NULL");
-    if (m->kind & ~(VDIT_MASK_BLOCK_CAUSAL | VDIT_MASK_RADIAL))
+    if (m->kind & ~(VDIT_MASK_BLOCK_CAUSAL | VDIT_MASK_RADIAL | VDIT_MASK_DYNAMIC))
         return fail(VDIT_ERR_INVALID_ARG, "unknown mask kind bits");
+    if ((m->kind & VDIT_MASK_DYNAMIC) && !(m->tau > 0.0 && m->tau < 1e30))
+        return fail(VDIT_ERR_INVALID_ARG, "dynamic threshold needs a finite tau > 0");
     if ((m->kind & VDIT_MASK_BLOCK_CAUSAL) && m->chunk_frames < 1)
         return fail(VDIT_ERR_INVALID_ARG, "chunk_frames must be >= 1");
     if ((m->kind & VDIT_MASK_RADIAL) && (m->w0 < 0 || m->gamma_shift < 0 || m->lambda < 0))
@@ -328,7 +330,9 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const long long units = (long long)p->n_qb * p->g.heads;
     int best = 1;
     double best_eff = 0.0;
-    for (int sp = 1; sp <= 8; ++sp) {
+    // the dynamic threshold needs each row's maximum over all its candidates: no key split
+    const int max_split = (p->m.kind & VDIT_MASK_DYNAMIC) ? 1 : 8;
+    for (int sp = 1; sp <= max_split; ++sp) {
         if (sp > 1 && max_len / sp < 8) break;
         const long long ctas = units * sp;
         const double eff = (double)ctas / (double)(((ctas + sms - 1) / sms) * sms);

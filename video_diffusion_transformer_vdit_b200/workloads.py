@@ -22,7 +22,7 @@ class Workload:
     heads: int
     head_dim: int
     bands: Tuple[int, int, int]
-    mask_kind: int            # bit 0 block-causal, bit 1 radial
+    mask_kind: int            # bit 0 block-causal, bit 1 radial, bit 2 dynamic threshold
     q_start: int              # global frame of the first query token
     q_frames: int
     capacity_frames: int      # KV ring capacity
@@ -32,6 +32,7 @@ class Workload:
     w0: int = 52
     gamma_shift: int = 1
     lam: int = 8
+    tau: float = 0.0          # dynamic threshold: logit margin below each row's maximum
     theta: float = 10000.0
 
     @property
@@ -83,4 +84,7 @@ WORKLOADS = {
                 mask_kind=3, q_start=396, q_frames=3, capacity_frames=21,
                 appends=tuple((s, 3) for s in range(378, 399, 3)), kv_stream_first_frame=378,
                 **_WAN),
+    6: Workload(6, "wan2.1-1.3b radial + dynamic threshold tau=2 21x30x52 h12", heads=12,
+                mask_kind=6, q_start=0, q_frames=21, capacity_frames=21, appends=((0, 21),),
+                kv_stream_first_frame=0, tau=2.0, **_WAN),
 }
