@@ -353,6 +353,27 @@ def run_gpu(args, w):
     del xs, ys
     rope_bytes = 2 * q.numel() * 2
 
+    # sequence-to-head pack (vdit_seq_pack) of Q as one of two sequence-parallel ranks would:
+    # RoPE at the global positions into the [2, tokens, heads / 2, d] all-to-all layout; back to
+    # back over two input / output pairs (400 MB in all)
+    pack = None
+    if g.heads % 2 == 0:
+        xs = [q, torch.empty_like(q).copy_(q)]
+        ss = [torch.empty(2, q.shape[0], g.heads // 2, g.head_dim, dtype=q.dtype, device=q.device)
+              for _ in range(2)]
+        for i in range(2):
+            vdit.seq_pack(xs[i], ss[i], g, w.q_start, q.shape[0], 2)
+        torch.cuda.synchronize()
+        r0.record(stream)
+        for i in range(20):
+            vdit.seq_pack(xs[i % 2], ss[i % 2], g, w.q_start, q.shape[0], 2)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        pack_ms = r0.elapsed_time(r1) / 20
+        pack = {"ms": pack_ms, "gbs": rope_bytes / (pack_ms * 1e-3) / 1e9,
+                "frac_hbm": rope_bytes / (pack_ms * 1e-3) / 1e9 / peaks()[0]["hbm_gbs"]}
+        del xs, ss
+
     # fused QKV projection + RoPE + cache append (vdit_qkv_rope) of the step's newest frames,
     # d_model = heads * head_dim (as in Wan2.1), random bf16 weights, its own cache
     qkv = None
@@ -486,6 +507,9 @@ def run_gpu(args, w):
                 "rope3d_apply_ms": rope_ms, "rope3d_apply_gbs": rope_bytes / (rope_ms * 1e-3) / 1e9,
                 "rope3d_apply_frac_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "hbm_peak_gbs": pk["hbm_gbs"],
+                "seq_pack": None if pack is None else dict(
+                    pack, how="vdit_seq_pack of Q for 2 ranks (RoPE + all-to-all layout), read + "
+                              "write bytes, not part of the step"),
                 "qkv_rope": None if qkv is None else dict(
                     qkv, frac_of_sustained_peak=qkv["tflops"] / peak,
                     frac_of_burst_peak=qkv["tflops"] / pk["bf16_tflops"],

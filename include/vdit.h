@@ -227,6 +227,18 @@ VDIT_API int vdit_qkv_rope(const vdit_geom* g, const void* x, const void* w, int
                            int start_frame, int n_frames, void* q_out, void* k_cache, void* v_cache,
                            int capacity_frames, void* stream);
 
+/* Sequence-to-head pack of the Ulysses-style exchange ([CRoPE] 2.A sequence split over ranks,
+ * 2.B global time index, 2.C one fused all-to-all that gathers the sequence and splits the heads,
+ * with the RoPE fused in). x: this rank's tokens, device bf16 [n_tokens, heads, head_dim], chunk-
+ * local tokens tok0 .. tok0 + n_tokens - 1 of a chunk whose first frame is start_frame. send:
+ * device bf16 [n_ranks][n_tokens][heads / n_ranks][head_dim]: block r holds heads
+ * r * heads / n_ranks .. (r + 1) * heads / n_ranks - 1, rotated at their global positions when
+ * rotate != 0 (as vdit_rope3d_apply), copied unchanged otherwise (V). An all-to-all of the n_ranks
+ * equal blocks then leaves every rank its heads for all tokens in sequence order. n_ranks must
+ * divide heads; x and send must not overlap. */
+VDIT_API int vdit_seq_pack(const vdit_geom* g, const void* x, void* send, int start_frame,
+                           long long tok0, long long n_tokens, int n_ranks, int rotate, void* stream);
+
 /* Reads and clears the current device's kernel status word: *status = VDIT_OK, or
  * VDIT_ERR_TIMEOUT when a bounded wait in a kernel gave up since the last read. Synchronises the
  * device. */

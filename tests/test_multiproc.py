@@ -49,3 +49,59 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.aggregate_tflops(1, 1e12, 1.0) == pytest.approx(1000.0)
+
+
+# ----------------------------------------------------------------------------- sequence -> heads
+
+def _oracle_pack(x, send, g, start_frame, tok0, n_ranks, rotate=True, stream=None):
+    """CPU stand-in of vdit_seq_pack for the gloo test (test infrastructure: the oracle's RoPE
+    at the tokens' global positions, then the [ranks, tokens, heads / ranks, D] layout)."""
+    import numpy as np
+    import oracle
+    n = x.shape[0]
+    y = x.double().numpy()
+    if rotate:
+        pos = oracle.positions(tok0 + n, g.grid_h, g.grid_w, start_frame)
+        og = oracle.Geometry(g.grid_h, g.grid_w, g.heads, g.head_dim, *g.bands, g.theta)
+        y = oracle.rope3d(y, tuple(p[tok0:] for p in pos), og)
+    hpr = g.heads // n_ranks
+    send.copy_(torch.from_numpy(np.ascontiguousarray(
+        y.reshape(n, n_ranks, hpr, g.head_dim).transpose(1, 0, 2, 3))).to(send.dtype))
+    return send
+
+
+def _seq_worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import numpy as np
+    import oracle
+    import synth
+    import video_diffusion_transformer_vdit_b200 as vdit
+    vdit.seq_pack = _oracle_pack  # the pack kernel needs a GPU; the exchange logic does not
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        g = vdit.Geometry(3, 5, 4, 64, (24, 20, 20))
+        n_all = 2 * 15 + 6                       # a chunk of 36 tokens (2.4 frames of 3 x 5)
+        full = synth.bf16_bits_to_f64(synth.qkv_bf16(7, n_all, 4, 64, "q"))
+        n = n_all // world
+        x = torch.from_numpy(full[rank * n:(rank + 1) * n]).float()
+        got = vdit.seq_to_heads(x, g, 9, rotate=True)
+        # the oracle's whole-chunk RoPE, this rank's heads
+        og = oracle.Geometry(3, 5, 4, 64, 24, 20, 20, 10000.0)
+        ref = oracle.rope3d(full, oracle.positions(n_all, 3, 5, 9), og)[:, rank * 2:(rank + 1) * 2]
+        out[rank] = float(np.abs(got.double().numpy() - ref).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_seq_to_heads_exchange_gloo_two_ranks():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as man:
+        out = man.dict()
+        mp.spawn(_seq_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    # float32 transport of float64 values: exact up to float32 rounding
+    assert res[0] < 1e-5 and res[1] < 1e-5

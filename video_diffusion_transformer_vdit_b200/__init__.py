@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_export.argtypes = [P, P, P, P]
         L.vdit_plan_export_masks.argtypes = [P, P, P]
         L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
+        L.vdit_seq_pack.argtypes = [P, P, P, I, ctypes.c_longlong, ctypes.c_longlong, I, I, P]
         L.vdit_plan_destroy.argtypes = [P]
         L.vdit_plan_destroy.restype = None
         L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
@@ -221,6 +222,41 @@ def qkv_rope(x: torch.Tensor, w: torch.Tensor, g: Geometry, start_frame: int,
                                _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
                                int(capacity_frames), _stream(stream)))
     return q
+
+
+def seq_pack(x: torch.Tensor, send: torch.Tensor, g: Geometry, start_frame: int, tok0: int,
+             n_ranks: int, rotate: bool = True, stream=None) -> torch.Tensor:
+    """x [n, heads, head_dim] (chunk-local tokens tok0 ..) -> send [n_ranks, n, heads / n_ranks,
+    head_dim], rotated at the global positions when rotate (vdit_seq_pack)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or x.shape[1:] != (g.heads, g.head_dim):
+        raise ValueError("x must be bf16 [n_tokens, heads, head_dim]")
+    if g.heads % n_ranks or tuple(send.shape) != (n_ranks, x.shape[0], g.heads // n_ranks, g.head_dim):
+        raise ValueError("send must be [n_ranks, n_tokens, heads / n_ranks, head_dim]")
+    gc = g.c()
+    _check(lib().vdit_seq_pack(ctypes.byref(gc), _dev_ptr(x, "x"), _dev_ptr(send, "send"),
+                               int(start_frame), int(tok0), x.shape[0], int(n_ranks), int(bool(rotate)),
+                               _stream(stream)))
+    return send
+
+
+def seq_to_heads(x: torch.Tensor, g: Geometry, start_frame: int, group=None, rotate: bool = True,
+                 stream=None) -> torch.Tensor:
+    """Sequence-parallel to head-parallel exchange of one chunk: rank r of the group holds tokens
+    [r n, (r + 1) n) (x [n, heads, head_dim]); returns [world * n, heads / world, head_dim], all
+    tokens of this rank's heads, rotated at their global positions when rotate. One pack
+    (vdit_seq_pack) and one all-to-all of equal blocks (NCCL on GPUs)."""
+    import torch.distributed as dist
+    on = dist.is_available() and dist.is_initialized()
+    world = dist.get_world_size(group) if on else 1
+    rank = dist.get_rank(group) if on else 0
+    n = x.shape[0]
+    send = torch.empty(world, n, g.heads // world, g.head_dim, dtype=x.dtype, device=x.device)
+    seq_pack(x, send, g, start_frame, rank * n, world, rotate, stream)
+    if world == 1:
+        return send[0]
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.view(world * n, g.heads // world, g.head_dim)
 
 
 class KVCache:

@@ -256,6 +256,59 @@ int launch_stream(bool append, StreamArgs& a, cudaStream_t s) {
     return vdit::cuda_check(cudaGetLastError(), "rope kernel launch");
 }
 
+// Sequence-to-head pack of the Ulysses-style exchange ("Accelerating Video Generation Inference
+// with Sequential-Parallel 3D Positional Encoding Using a Global Time Index", sections 2.A-2.C: the
+// sequence is split over the ranks; QKV, the causal RoPE and one fused all-to-all that gathers the
+// sequence and splits the heads). This rank's tokens x [n_tok, heads, D] (chunk-local tokens
+// tok0 .. tok0 + n_tok - 1) go to send [ranks][n_tok][heads / ranks][D]: block r holds the heads
+// rank r receives, so an all-to-all of equal blocks leaves every rank [ranks * n_tok, heads /
+// ranks, D] in sequence order. With ROTATE the rows are rotated at their global positions (the
+// time index needs only start_frame and tok0: no rank asks another for its positions).
+struct PackArgs {
+    StreamArgs s;       // x, y (= send), tables, geometry, n_tokens, cpt, cpr_log2
+    int tok0;
+    int heads_per_rank;
+    FastDiv by_hpr;
+};
+
+template <bool ROTATE>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) rope_pack_kernel(PackArgs pa) {
+    const StreamArgs& a = pa.s;
+    const int lane = threadIdx.x & 31;
+    const int n_warps = gridDim.x * kWarpsPerBlock;
+    const int c8 = lane & ((1 << a.cpr_log2) - 1);
+    const int ft = a.grid_h * a.grid_w;
+    for (int n = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); n < a.n_tokens; n += n_warps) {
+        float2 cs[4];
+        if (ROTATE) {
+            const int tok = pa.tok0 + n;
+            const uint32_t f = fdiv((uint32_t)tok, a.by_ft);
+            const int rem = tok - (int)f * ft;
+            const int h = (int)fdiv((uint32_t)rem, a.by_w);
+            chunk_angles(cs, c8 * 4, a.start_frame + (int)f, h, rem - h * a.grid_w, a);
+        }
+        const size_t src0 = (size_t)n * a.cpt;
+        for (int j0 = 0; j0 < a.cpt; j0 += 32 * kBatch) {
+            uint4 xin[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) xin[u] = __ldcs(a.x + src0 + j);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) {
+                    const int head = j >> a.cpr_log2;
+                    const int r = (int)fdiv((uint32_t)head, pa.by_hpr), hh = head - r * pa.heads_per_rank;
+                    const size_t row = ((size_t)r * a.n_tokens + n) * pa.heads_per_rank + hh;
+                    __stcs(a.y + (row << a.cpr_log2) + c8, ROTATE ? rotate_chunk(xin[u], cs) : xin[u]);
+                }
+            }
+        }
+    }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int fill_common(const vdit_geom* g, StreamArgs& a) {
@@ -345,4 +398,46 @@ extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
     a.cap_tok = ft * capacity_frames;
     a.by_cap = make_fastdiv((uint32_t)capacity_frames);
     return launch_stream(true, a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int vdit_seq_pack(const vdit_geom* g, const void* x, void* send, int start_frame,
+                             long long tok0, long long n_tokens, int n_ranks, int rotate, void* stream) {
+    using vdit::fail;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (n_tokens < 0 || tok0 < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens and tok0 must be >= 0");
+    if (n_tokens == 0) return VDIT_OK;
+    if (!x || !send) return fail(VDIT_ERR_INVALID_ARG, "x or send is NULL");
+    if (!aligned16(x) || !aligned16(send)) return fail(VDIT_ERR_MISALIGNED, "x/send not 16-byte aligned");
+    if (n_ranks < 1 || g->heads % n_ranks != 0)
+        return fail(VDIT_ERR_INVALID_ARG, "n_ranks must divide heads");
+    const long long ft = (long long)g->grid_h * g->grid_w;
+    const long long last = tok0 + n_tokens - 1;
+    if (start_frame < 0 || start_frame + last / ft > VDIT_MAX_FRAME)
+        return fail(VDIT_ERR_INVALID_ARG, "frames outside [0, VDIT_MAX_FRAME]");
+    const long long bytes = n_tokens * g->heads * g->head_dim * 2;
+    const char* xb = static_cast<const char*>(x);
+    const char* yb = static_cast<const char*>(send);
+    if (xb < yb + bytes && yb < xb + bytes) return fail(VDIT_ERR_INVALID_ARG, "x and send overlap");
+    if ((unsigned long long)n_tokens * g->heads * (g->head_dim / 8) >= (1ull << 31) || last >= (1ll << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "shard larger than 2^31 16-byte chunks");
+    PackArgs pa{};
+    if (int rc = fill_common(g, pa.s)) return rc;
+    pa.s.x = static_cast<const uint4*>(x);
+    pa.s.y = static_cast<uint4*>(send);
+    pa.s.n_tokens = (int)n_tokens;
+    pa.s.start_frame = start_frame;
+    pa.tok0 = (int)tok0;
+    pa.heads_per_rank = g->heads / n_ranks;
+    pa.by_hpr = make_fastdiv((uint32_t)pa.heads_per_rank);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long want = (n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int blocks = (int)std::min<long long>(want, (long long)sms * 4);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rotate)
+        rope_pack_kernel<true><<<blocks, kWarpsPerBlock * 32, 0, st>>>(pa);
+    else
+        rope_pack_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, st>>>(pa);
+    return vdit::cuda_check(cudaGetLastError(), "pack kernel launch");
 }
