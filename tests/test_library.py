@@ -185,3 +185,18 @@ def test_calls_reject_null_and_misaligned_pointers_before_device_work():
     assert L.vdit_attn_forward(h, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
                                ctypes.c_void_p(16), None, ctypes.c_float(0.1), None) == vdit.ERR_NOT_UPLOADED
     L.vdit_plan_destroy(h)
+
+
+def test_plan_and_masks_bit_exact_on_the_gpu_edge_workloads():
+    # the degenerate grids and masks of the GPU edge tests: 1 x 1 grid, lambda 1, w0 0, chunks of
+    # one frame, the last frames of the time table, a 2 x 1024 grid
+    from test_gpu_edges import EDGES
+    for name, w in EDGES.items():
+        first, last = w.window()
+        plan = vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                         kv_first_frame=first, kv_last_frame=last, upload=False)
+        ref = _oracle_tiles(w.grid_h, w.grid_w, w.q_start, w.q_frames, w.capacity_frames, first, last,
+                            w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
+        _compare(plan, ref)
+        _check_masks(plan, w.grid_h, w.grid_w, w.q_start, w.q_frames, w.capacity_frames, first, last,
+                     w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam)
