@@ -105,3 +105,60 @@ def test_seq_to_heads_exchange_gloo_two_ranks():
         res = dict(out)
     # float32 transport of float64 values: exact up to float32 rounding
     assert res[0] < 1e-5 and res[1] < 1e-5
+
+
+# ----------------------------------------------------------------------------- K/V push
+
+def _oracle_append(k_cache, v_cache, g, capacity_frames, k, v, start_frame, stream=None):
+    """CPU stand-in of vdit_kv_append for the gloo test (test infrastructure: the oracle's
+    append, in float64, on CPU caches)."""
+    import numpy as np
+    import oracle
+    og = oracle.Geometry(g.grid_h, g.grid_w, g.heads, g.head_dim, *g.bands, g.theta)
+    kc, vc = k_cache.numpy(), v_cache.numpy()
+    oracle.kv_append(kc, vc, capacity_frames, og, k.double().numpy(), v.double().numpy(),
+                     start_frame, k.shape[0] // g.frame_tokens)
+
+
+def _push_worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import numpy as np
+    import synth
+    import video_diffusion_transformer_vdit_b200 as vdit
+    vdit.kv_append = _oracle_append  # the append kernel needs a GPU; the push protocol does not
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        g = vdit.Geometry(3, 4, 2, 64, (24, 20, 20))
+        cache = vdit.KVCache(g, 5, device="cpu")
+        cache.k, cache.v = cache.k.double(), cache.v.double()
+        for start in (0, 3, 6):  # three chunks of 3 frames into a 5-frame ring (wraps)
+            if rank == 0:
+                k = torch.from_numpy(synth.bf16_bits_to_f64(synth.qkv_bf16(5, 36, 2, 64, "k", token_offset=12 * start)))
+                v = torch.from_numpy(synth.bf16_bits_to_f64(synth.qkv_bf16(5, 36, 2, 64, "v", token_offset=12 * start)))
+                cache.append(k, v, start)
+                for wk in cache.push(k, v, 1):
+                    wk.wait()
+            else:
+                cache.receive(start, 3, 0)
+        out[rank] = (cache.k.double().numpy().copy(), cache.v.double().numpy().copy(),
+                     cache.first_frame, cache.last_frame)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kv_push_gloo_two_ranks():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as man:
+        out = man.dict()
+        mp.spawn(_push_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    k0, v0, f0, l0 = res[0]
+    k1, v1, f1, l1 = res[1]
+    assert (f0, l0) == (f1, l1) == (4, 8)
+    # the receiver appended exactly what the sender appended
+    assert (k0 == k1).all() and (v0 == v1).all()
+    assert abs(k0).max() > 0

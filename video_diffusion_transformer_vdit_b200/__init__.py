@@ -291,6 +291,25 @@ class KVCache:
         kv_append(self.k, self.v, self.g, self.capacity_frames, k, v, start_frame, stream)
         self._note(start_frame, k.shape[0] // self.g.frame_tokens)
 
+    def push(self, k: torch.Tensor, v: torch.Tensor, dst: int, group=None) -> list:
+        """Wave Parallelism's K/V forward push (Wave Forcing / WaveRT): send a chunk's K and V (as
+        given to append, before RoPE) one way to rank dst, which appends them to its own cache
+        with receive(). The sends are asynchronous (isend; NCCL on GPUs), so they overlap the
+        attention that follows; returns the work handles to wait on before k, v are reused."""
+        import torch.distributed as dist
+        return [dist.isend(k.contiguous(), dst, group=group), dist.isend(v.contiguous(), dst, group=group)]
+
+    def receive(self, start_frame: int, n_frames: int, src: int, group=None, stream=None) -> None:
+        """Receive a chunk pushed by rank src and append it here (RoPE at its global frames, ring
+        write), as the sender appended it to its own cache."""
+        import torch.distributed as dist
+        shape = (n_frames * self.g.frame_tokens, self.g.heads, self.g.head_dim)
+        k = torch.empty(shape, dtype=self.k.dtype, device=self.k.device)
+        v = torch.empty_like(k)
+        dist.recv(k, src, group=group)
+        dist.recv(v, src, group=group)
+        self.append(k, v, start_frame, stream)
+
     def project_append(self, x: torch.Tensor, w: torch.Tensor, start_frame: int,
                        q_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """Fused QKV projection of the chunk x (vdit_qkv_rope): K', V into the ring; returns the
