@@ -90,7 +90,9 @@ enum {
     B_KFULL = 0, B_KEMPTY = B_KFULL + kStages, B_VFULL = B_KEMPTY + kStages,
     B_VEMPTY = B_VFULL + kStages, B_IFULL = B_VEMPTY + kStages, B_IEMPTY = B_IFULL + kStages,
     B_SFULL = B_IEMPTY + kStages, B_SFREE = B_SFULL + kQTiles, B_PFULL = B_SFREE + 1,
-    B_PVDONE = B_PFULL + kQTiles, B_DRAIN = B_PVDONE + kQTiles, B_COUNT
+    B_PVDONE = B_PFULL + kQTiles, B_DRAIN = B_PVDONE + kQTiles,
+    B_SFREE1 = B_DRAIN + 1,  // dynamic-threshold logit pass: the second score buffer
+    B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier area too small");
 // Stage of the keep masks, one per K stage: a 16-byte header {tile, flags} and, for each query
@@ -256,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(B_PVDONE + h), 1);
         }
         mbar_init(BAR(B_SFREE), 128);
+        mbar_init(BAR(B_SFREE1), 128);
         mbar_init(BAR(B_DRAIN), 2);  // one commit from each MMA-issuing thread
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -312,6 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(BAR(B_IFULL + s), (j / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
             const uint8_t* info = smem + L::OFF_KINFO + s * kKinfoBytes;
             const uint32_t flags = (uint32_t)reinterpret_cast<const int*>(info)[1];
+            // dynamic-threshold logit pass: each query tile's score tiles have a buffer of their own
+            const uint32_t sbuf = pass0 ? (uint32_t)h : 0u;
             if (!(flags & f_in)) {
                 mbar_arrive(BAR(B_IEMPTY + s));
                 continue;
@@ -320,14 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             uint32_t sr[128];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(t_s + q4 * 32, sr + q4 * 32);
+            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(t_s + 128u * sbuf + q4 * 32, sr + q4 * 32);
             tmem_ld_wait(sr);
             reg_touch32(sr + 32);
             reg_touch32(sr + 64);
             reg_touch32(sr + 96);
             // S is in registers: the shared S columns may take the next score tile
             tc_fence_before();
-            mbar_arrive(BAR(B_SFREE));
+            mbar_arrive(BAR(sbuf ? B_SFREE1 : B_SFREE));
             float* sv = reinterpret_cast<float*>(sr);
             if (!(flags & f_full)) {
                 // this row's keep bits for the 128 keys of the tile, from the plan's mask block
@@ -632,6 +637,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // S_h(j) = Q_h K(j)^T into the shared S columns, in list order, each after the
                 // previous score tile has been read out of TMEM by its softmax group
                 int ns = 0;
+                // dynamic-threshold logit pass: the P columns are idle, so each query tile's score
+                // tiles get a buffer of their own (group h: [128 h, 128 h + 128)); a group's next
+                // score tile waits only for its previous one to be read (never two unread, so a
+                // group's SFULL phases cannot run two ahead of its waits). Uses of each buffer so
+                // far, and whether buffer 1 has been drained before the first attention-pass tile
+                int uses0 = 0, uses1 = 0;
+                bool drained1 = false;
                 for (int j = 0; j < n_v; ++j) {  // both passes in the dynamic-threshold mode
                     const int s = j % kStages;
                     const int f = f_cur;
@@ -644,7 +656,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int h = 0; h < kQTiles; ++h) {
                         if (!(f & (h ? 4 : 1))) continue;
-                        if (ns > 0) {
+                        uint32_t sbuf = 0;
+                        if (DYN) {
+                            // the buffer's previous score tile has been read out
+                            sbuf = j < n_ent ? (uint32_t)h : 0u;
+                            const int uses = sbuf ? uses1 : uses0;
+                            if (uses > 0) {
+                                if (!wait_bounded(BAR(sbuf ? B_SFREE1 : B_SFREE), (uses - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                            }
+                            if (j >= n_ent && !drained1) {
+                                // attention pass: the P columns must hold no unread score tile
+                                if (uses1 > 0 &&
+                                    !wait_bounded(BAR(B_SFREE1), (uses1 - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                                drained1 = true;
+                            }
+                            if (sbuf) ++uses1; else ++uses0;
+                            tc_fence_after();
+                        } else if (ns > 0) {
                             if (!wait_bounded(BAR(B_SFREE), (ns - 1) & 1, abort_flag, a.status)) { ok = false; break; }
                             tc_fence_after();
                         }
@@ -652,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint64_t off = (uint64_t)((((kk >> 2) * kSlabBytes) + (kk & 3) * 32) >> 4);
-                            tc_mma(tmem, q0 + off, k0 + off, idesc_qk, kk > 0);
+                            tc_mma(tmem + 128u * sbuf, q0 + off, k0 + off, idesc_qk, kk > 0);
                         }
                         tc_commit(BAR(B_SFULL + h));
                         ++ns;
