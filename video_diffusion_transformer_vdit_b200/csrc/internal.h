@@ -48,7 +48,6 @@ struct vdit_plan {
     std::vector<unsigned char> full;
     std::vector<int> slot_frame;  // global frame held by each frame slot, -1 if empty
     std::vector<int> radius;      // per dt in [0, dt_max]: largest kept Chebyshev distance
-    std::vector<int> qtile_order; // q-tiles sorted by descending tile count (longest first)
     // Blocks of two consecutive q-tiles (2b, 2b+1), the unit one attention CTA works on: the
     // ascending union of the two tiles' key-tile lists, with per entry
     //   bit0: listed for q-tile 2b, bit1: full for 2b, bit2: listed for 2b+1, bit3: full for 2b+1.
@@ -68,12 +67,6 @@ struct vdit_plan {
     // device copy
     int device = -1;
     void* d_buf = nullptr;
-    const int* d_row_ptr = nullptr;
-    const int* d_col_idx = nullptr;
-    const unsigned char* d_full = nullptr;
-    const int* d_slot_frame = nullptr;
-    const int* d_radius = nullptr;
-    const int* d_qtile_order = nullptr;
     const int* d_u_row_ptr = nullptr;
     const int* d_u_col = nullptr;
     const unsigned char* d_u_flags = nullptr;

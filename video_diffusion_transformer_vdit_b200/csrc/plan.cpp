@@ -265,13 +265,6 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
     std::stable_sort(p->unit_order.begin(), p->unit_order.end(), [&](int a, int b) {
         return p->u_row_ptr[a + 1] - p->u_row_ptr[a] > p->u_row_ptr[b + 1] - p->u_row_ptr[b];
     });
-    // longest rows first: a persistent kernel that takes q-tiles in this order finishes its
-    // longest work items early and fills the tail with short ones
-    p->qtile_order.resize(p->n_qt);
-    for (int i = 0; i < p->n_qt; ++i) p->qtile_order[i] = i;
-    std::stable_sort(p->qtile_order.begin(), p->qtile_order.end(), [&](int a, int b) {
-        return p->row_ptr[a + 1] - p->row_ptr[a] > p->row_ptr[b + 1] - p->row_ptr[b];
-    });
     *out = p;
     return VDIT_OK;
 }
@@ -340,14 +333,11 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
         if (eff >= 0.9) break;
     }
     p->n_split = best;
-    // one allocation: row_ptr | qtile_order | slot_frame | radius | u_row_ptr | col_idx | full |
-    // u_col | u_flags | unit_order | u_mask | masks | (split workspace: partial O | partial lse)
+    // one allocation of what the kernels read: u_row_ptr | u_col | u_flags | unit_order | u_mask |
+    // masks | (split workspace: partial O | partial lse); the per-q-tile lists, the slot frames
+    // and the radius table stay on the host (exports, mask construction)
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
-    const size_t n_rp = sizeof(int) * p->row_ptr.size(), n_qo = sizeof(int) * p->qtile_order.size();
-    const size_t n_sf = sizeof(int) * p->slot_frame.size(), n_ra = sizeof(int) * p->radius.size();
     const size_t n_urp = sizeof(int) * p->u_row_ptr.size();
-    const size_t n_ci = sizeof(int) * std::max<size_t>(1, p->col_idx.size());
-    const size_t n_fu = std::max<size_t>(1, p->full.size());
     const size_t n_uc = sizeof(int) * std::max<size_t>(1, p->u_col.size());
     const size_t n_uf = std::max<size_t>(1, p->u_flags.size());
     const size_t n_uo = sizeof(int) * std::max<size_t>(1, p->unit_order.size());
@@ -356,36 +346,22 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t n_wo = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
                                              p->g.heads * p->g.head_dim : 0;
     const size_t n_wl = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads * p->q_tokens : 0;
-    const size_t meta = up(n_rp) + up(n_qo) + up(n_sf) + up(n_ra) + up(n_urp) + up(n_ci) +
-                        up(n_fu) + up(n_uc) + up(n_uf) + up(n_uo) + up(n_um) + up(n_mk);
+    const size_t meta = up(n_urp) + up(n_uc) + up(n_uf) + up(n_uo) + up(n_um) + up(n_mk);
     const size_t total = meta + up(n_wo) + up(n_wl);
     std::vector<unsigned char> host(total, 0);
     size_t off = 0;
-    auto put = [&](const void* src, size_t n) {
+    auto put = [&](const void* src, size_t n, size_t reserved) {
         size_t at = off;
         if (n) std::memcpy(host.data() + off, src, n);
-        off += up(n);
+        off += up(reserved);
         return at;
     };
-    const size_t o_rp = put(p->row_ptr.data(), n_rp);
-    const size_t o_qo = put(p->qtile_order.data(), n_qo);
-    const size_t o_sf = put(p->slot_frame.data(), n_sf);
-    const size_t o_ra = put(p->radius.data(), n_ra);
-    const size_t o_urp = put(p->u_row_ptr.data(), n_urp);
-    const size_t o_ci = put(p->col_idx.data(), sizeof(int) * p->col_idx.size());
-    off = o_ci + up(n_ci);
-    const size_t o_fu = put(p->full.data(), p->full.size());
-    off = o_fu + up(n_fu);
-    const size_t o_uc = put(p->u_col.data(), sizeof(int) * p->u_col.size());
-    off = o_uc + up(n_uc);
-    const size_t o_uf = put(p->u_flags.data(), p->u_flags.size());
-    off = o_uf + up(n_uf);
-    const size_t o_uo = put(p->unit_order.data(), sizeof(int) * p->unit_order.size());
-    off = o_uo + up(n_uo);
-    const size_t o_um = put(p->u_mask.data(), sizeof(int) * p->u_mask.size());
-    off = o_um + up(n_um);
-    const size_t o_mk = put(p->masks.data(), sizeof(uint32_t) * p->masks.size());
-    off = o_mk + up(n_mk);
+    const size_t o_urp = put(p->u_row_ptr.data(), n_urp, n_urp);
+    const size_t o_uc = put(p->u_col.data(), sizeof(int) * p->u_col.size(), n_uc);
+    const size_t o_uf = put(p->u_flags.data(), p->u_flags.size(), n_uf);
+    const size_t o_uo = put(p->unit_order.data(), sizeof(int) * p->unit_order.size(), n_uo);
+    const size_t o_um = put(p->u_mask.data(), sizeof(int) * p->u_mask.size(), n_um);
+    const size_t o_mk = put(p->masks.data(), sizeof(uint32_t) * p->masks.size(), n_mk);
     if (off != meta) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
     host.resize(meta);  // the workspace is not initialised: every entry is written before use
     void* d = nullptr;
@@ -400,12 +376,6 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     unsigned char* b = static_cast<unsigned char*>(d);
     p->device = dev;
     p->d_buf = d;
-    p->d_row_ptr = reinterpret_cast<const int*>(b + o_rp);
-    p->d_qtile_order = reinterpret_cast<const int*>(b + o_qo);
-    p->d_slot_frame = reinterpret_cast<const int*>(b + o_sf);
-    p->d_radius = reinterpret_cast<const int*>(b + o_ra);
-    p->d_col_idx = reinterpret_cast<const int*>(b + o_ci);
-    p->d_full = b + o_fu;
     p->d_u_row_ptr = reinterpret_cast<const int*>(b + o_urp);
     p->d_u_col = reinterpret_cast<const int*>(b + o_uc);
     p->d_u_flags = b + o_uf;
