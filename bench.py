@@ -173,7 +173,7 @@ def run_reference(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic N(0,1), seeded SplitMix64 + Box-Muller, bf16-rounded",
             "config": config_of(w, {"parallelism": "host cores (OpenMP)"}),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": arm.oracle.threads(),
                              "kind": "oracle", "sample": arm.describe(rows)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -460,7 +460,7 @@ def run_gpu(args, w):
         if world == 1 and not args.no_cpu_baseline:
             arm = OracleArm(w)
             val, dt, n = arm.sample(args.cpu_budget)
-            cpu = {"value": val, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            cpu = {"value": val, "unit": "TFLOP/s", "cores": arm.oracle.threads(), "kind": "oracle",
                    "sample": arm.describe(n), "seconds": dt}
         info = plan.info
         line = {

@@ -57,8 +57,14 @@ def lib() -> ctypes.CDLL:
         L.vo_cache_positions.argtypes = [_I, _I, _I, _I, _I, _i32p, _i32p, _i32p, _u8p]
         L.vo_kv_append.argtypes = [_f64p, _f64p, _I, _I, _I, _I, _I, _I, _I, _I, _D,
                                    _f64p, _f64p, _I, _I]
+        L.vo_threads.restype = _I
         _lib = L
     return _lib
+
+
+def threads() -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int(lib().vo_threads())
 
 
 @dataclass(frozen=True)

@@ -43,6 +43,7 @@
  * list == reshape/any of the explicit mask; ring placement of the KV cache.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -287,3 +288,6 @@ void vo_kv_append(double *k_cache, double *v_cache, int capacity_frames,
     }
     free(t); free(h); free(w); free(kr);
 }
+
+/* Number of OpenMP threads the parallel loops above run on (for reporting). */
+int vo_threads(void) { return omp_get_max_threads(); }
