@@ -76,10 +76,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemP = 128, kTmemO = 256;
 constexpr float kRescaleTau = 8.0f;              // rescale O only when the max grows by > 2^8
 // Which of every 8 consecutive P pairs of a row take the FMA-pipe exp2 instead of the MUFU unit
-// (bit i set: pair i mod 8). Measured on the dense 32,760-token workload: none 1073, two of
-// eight 1028, three of eight 997 TFLOP/s, so by default every exponential uses MUFU; the
-// software path stays available for other shapes (it passed the GPU parity tests with 0x88
-// and 0xA8).
+// (bit i set: pair i mod 8). Measured on the dense 32,760-token workload: none 1297 - 1300,
+// one of eight 1259 - 1270, two of eight 1247 - 1255, three of eight 1218 TFLOP/s (the XU pipe
+// is not the bound; the extra FMA work lengthens the softmax), so by default every exponential
+// uses MUFU; the software path stays available for other shapes (it passed the GPU parity
+// tests with 0x88 and 0xA8).
 #ifndef VDIT_POLY_PAIRS
 #define VDIT_POLY_PAIRS 0x00u
 #endif
