@@ -159,8 +159,9 @@ VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask
  * the forward pass from the device's SM count: when the (query block, head) units alone would
  * leave most of a wave of SMs idle, each unit's key tiles are cut into kv_splits pieces whose
  * normalised fp32 partial outputs and log-sum-exps go to a scratch workspace held by the plan
- * and are merged by a second kernel. Forward calls that share one plan must therefore not run
- * concurrently on different streams. */
+ * and are merged by a second kernel (never in the dynamic-threshold mode, whose threshold needs
+ * each row's maximum over all its candidates). Forward calls that share one plan must therefore
+ * not run concurrently on different streams. */
 VDIT_API int vdit_plan_upload(vdit_plan* p, void* stream);
 
 VDIT_API int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info);
@@ -184,7 +185,8 @@ VDIT_API void vdit_plan_destroy(vdit_plan* p);
  * ring layout above. o: device bf16 [q_tokens, heads, head_dim]. lse: optional device fp32
  * [heads, q_tokens] (natural-log sum of exp of the kept scaled scores) or NULL. scale > 0
  * (1/sqrt(head_dim) for the Wan2.1 shapes). Rows with no kept key get o = 0, lse = -inf.
- * head_dim must be 128 for this kernel (VDIT_ERR_UNSUPPORTED otherwise). */
+ * head_dim 64 or 128 (the plan accepts no other). With VDIT_MASK_DYNAMIC the output is the
+ * softmax over the kept candidates only, and lse their log-sum-exp. */
 VDIT_API int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
                       void* o, float* lse, float scale, void* stream);
 
