@@ -156,11 +156,12 @@ VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask
 
 /* Copies the plan's schedule and tables to the current device (allocates; the copy is ordered on
  * stream). Idempotent. Required before vdit_attn_forward. It also fixes the key-range split of
- * the forward pass from the device's SM count: when the (query block, head) units alone would
- * leave most of a wave of SMs idle, each unit's key tiles are cut into kv_splits pieces whose
- * normalised fp32 partial outputs and log-sum-exps go to a scratch workspace held by the plan
- * and are merged by a second kernel (never in the dynamic-threshold mode, whose threshold needs
- * each row's maximum over all its candidates). Forward calls that share one plan must therefore
+ * the forward pass from the device's SM count: when cutting each (query block, head) unit's key
+ * tiles into kv_splits pieces shortens the estimated time (the CTAs' makespan over the SMs plus
+ * the cost of the partial results), the pieces' normalised fp32 partial outputs and
+ * log-sum-exps go to a scratch workspace held by the plan and are merged by a second kernel
+ * (never in the dynamic-threshold mode, whose threshold needs each row's maximum over all its
+ * candidates). Forward calls that share one plan must therefore
  * not run concurrently on different streams. */
 VDIT_API int vdit_plan_upload(vdit_plan* p, void* stream);
 
