@@ -165,6 +165,10 @@ VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask
  * not run concurrently on different streams. */
 VDIT_API int vdit_plan_upload(vdit_plan* p, void* stream);
 
+/* Host only: the key split vdit_plan_upload would choose for this plan on a device with
+ * sm_count SMs (the rule above), without touching any device. */
+VDIT_API int vdit_plan_split_for(const vdit_plan* p, int sm_count, int* kv_splits);
+
 VDIT_API int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info);
 
 /* Host copy of the schedule: row_ptr [q_tiles + 1], col_idx [tiles], full [tiles] (0/1). */

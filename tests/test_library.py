@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import video_diffusion_transformer_vdit_b200 as vdit
-from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS
+from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS, Workload
 
 
 def test_library_exports_every_declared_symbol():
@@ -153,6 +153,25 @@ def test_plan_masks_bit_exact_vs_oracle_random_geometries():
         plan = vdit.Plan(g, vdit.Mask(kind, chunk, w0, gs, lam), q_start, q_frames,
                          capacity_frames=cap, kv_first_frame=first, kv_last_frame=last, upload=False)
         _check_masks(plan, gh, gw, q_start, q_frames, cap, first, last, kind, chunk, w0, gs, lam)
+
+
+def test_key_split_rule_picks_the_measured_best_counts():
+    """vdit_plan_upload's key split (host-only twin vdit_plan_split_for) on a 148-SM B200: on the
+    causal chunk forced splits 2 / 3 / 4 / 5 / 6 measured 1 018 / 1 133 / 1 068 / 1 088 / 1 038
+    TFLOP/s and on the 14B rollout chunk 1 / 2 / 4 measured 556 / 518 / 456, so the rule must
+    pick 3 and 1; the dense and radial shapes fill 10 waves unsplit; the dynamic threshold
+    never splits; one head of the causal chunk (19 CTAs unsplit) splits, within the 32 MiB the
+    no-allocation forward holds."""
+    def plan(w):
+        first, last = w.window()
+        return vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                         kv_first_frame=first, kv_last_frame=last, upload=False)
+    assert {k: plan(w).split_for(148) for k, w in WORKLOADS.items()} == {1: 1, 2: 1, 3: 3, 4: 1, 5: 1, 6: 1}
+    one = Workload(**{**WORKLOADS[3].__dict__, "id": 95, "heads": 1})
+    sp = plan(one).split_for(148)
+    assert sp > 1 and sp * one.q_tokens * (one.head_dim + 1) * 4 <= 32 << 20
+    with pytest.raises(vdit.VditError):
+        plan(one).split_for(0)
 
 
 def test_plan_rejects_bad_arguments():

@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_info.argtypes = [P, ctypes.POINTER(_PlanInfo)]
         L.vdit_plan_export.argtypes = [P, P, P, P]
         L.vdit_plan_export_masks.argtypes = [P, P, P]
+        L.vdit_plan_split_for.argtypes = [P, I, ctypes.POINTER(I)]
         L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
         L.vdit_seq_pack.argtypes = [P, P, P, I, ctypes.c_longlong, ctypes.c_longlong, I, I, P]
         L.vdit_plan_destroy.argtypes = [P]
@@ -372,6 +373,12 @@ class Plan:
         _check(lib().vdit_plan_export_masks(self._h, ctypes.c_void_p(idx.ctypes.data),
                                             ctypes.c_void_p(words.ctypes.data)))
         return idx[:inf["tiles"]], words[:inf["mask_bytes"] // 4].reshape(-1, 128, 4)
+
+    def split_for(self, sm_count: int) -> int:
+        """The key split vdit_plan_upload would choose on a device with sm_count SMs."""
+        out = ctypes.c_int()
+        _check(lib().vdit_plan_split_for(self._h, int(sm_count), ctypes.byref(out)))
+        return out.value
 
     def flops(self) -> float:
         """Unmasked-entry FLOPs of one forward: 4 * head_dim per kept (query, key, head)."""

@@ -270,6 +270,58 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
     return VDIT_OK;
 }
 
+namespace {
+
+// Key-range split of every (q-block, head) unit for a device with `sms` SMs: the count (1 .. 8,
+// at least 8 key tiles a piece) with the least estimated time. The attention kernel's time is
+// the makespan of its CTAs, dispatched in launch order (per head, piece-major, units longest
+// first) each to the SM that frees first, a CTA costing its key tiles plus kPieceTiles for its
+// prologue, pipeline fill and epilogue; a split adds its fp32 partial results, written and read
+// back by the merge. Constants measured on a B200 (one CTA per SM runs a union-list entry of two
+// 128-query tiles in ~1.44 us); they reproduce the measured order of split counts on the causal
+// chunk (3 best, then 5, 4, 6, 2) and on the 14B rollout chunk (1, then 2, then 4).
+int choose_split(const vdit_plan& p, int sms) {
+    constexpr double kPieceTiles = 12.0, kTileSeconds = 1.44e-6, kBytesPerSecond = 6.5e12;
+    int max_len = 0;
+    for (int b = 0; b < p.n_qb; ++b) max_len = std::max(max_len, p.u_row_ptr[b + 1] - p.u_row_ptr[b]);
+    int best = 1;
+    double best_t = 0.0;
+    // the dynamic threshold needs each row's maximum over all its candidates: no key split
+    const int max_split = (p.m.kind & VDIT_MASK_DYNAMIC) ? 1 : 8;
+    std::vector<double> sm_free;
+    for (int sp = 1; sp <= max_split; ++sp) {
+        if (sp > 1 && max_len / sp < 8) break;
+        sm_free.assign(std::max(1, sms), 0.0);
+        std::make_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
+        double span = 0.0;
+        for (int h = 0; h < p.g.heads; ++h)
+            for (int piece = 0; piece < sp; ++piece)
+                for (int i = 0; i < p.n_qb; ++i) {
+                    const int u = p.unit_order[i];
+                    const long long n = p.u_row_ptr[u + 1] - p.u_row_ptr[u];
+                    const double cost = (double)(n * (piece + 1) / sp - n * piece / sp) + kPieceTiles;
+                    std::pop_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
+                    sm_free.back() += cost;
+                    span = std::max(span, sm_free.back());
+                    std::push_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
+                }
+        double t = span * kTileSeconds;
+        if (sp > 1)
+            t += 2.0 * sp * (double)p.q_tokens * p.g.heads * (p.g.head_dim + 1) * 4.0 / kBytesPerSecond;
+        if (sp == 1 || t < best_t) { best_t = t; best = sp; }
+    }
+    return best;
+}
+
+}  // namespace
+
+extern "C" int vdit_plan_split_for(const vdit_plan* p, int sm_count, int* kv_splits) {
+    if (!p || !kv_splits || sm_count < 1)
+        return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or output, or sm_count < 1");
+    *kv_splits = choose_split(*p, sm_count);
+    return VDIT_OK;
+}
+
 extern "C" int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info) {
     if (!p || !info) return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or info");
     info->q_tokens = p->q_tokens;
@@ -315,46 +367,9 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
         if (p->device == dev) return VDIT_OK;
         return vdit::fail(VDIT_ERR_INVALID_ARG, "plan already uploaded to another device");
     }
-    // Key-range split: the count (1 .. 8, at least 8 key tiles a piece) with the least estimated
-    // time. The attention kernel's time is the makespan of its CTAs, dispatched in launch order
-    // (per head, piece-major, units longest first) each to the SM that frees first, a CTA costing
-    // its key tiles plus kPieceTiles for its prologue, pipeline fill and epilogue; a split adds
-    // its fp32 partial results, written and read back by the merge. Constants measured on a
-    // B200 (one CTA per SM runs a union-list entry of two 128-query tiles in ~1.44 us); they
-    // reproduce the measured order of split counts on the causal chunk (3 best, then 5, 4, 6, 2)
-    // and on the 14B rollout chunk (1, then 2, then 4).
-    constexpr double kPieceTiles = 12.0, kTileSeconds = 1.44e-6, kBytesPerSecond = 6.5e12;
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int max_len = 0;
-    for (int b = 0; b < p->n_qb; ++b) max_len = std::max(max_len, p->u_row_ptr[b + 1] - p->u_row_ptr[b]);
-    int best = 1;
-    double best_t = 0.0;
-    // the dynamic threshold needs each row's maximum over all its candidates: no key split
-    const int max_split = (p->m.kind & VDIT_MASK_DYNAMIC) ? 1 : 8;
-    std::vector<double> sm_free;
-    for (int sp = 1; sp <= max_split; ++sp) {
-        if (sp > 1 && max_len / sp < 8) break;
-        sm_free.assign(std::max(1, sms), 0.0);
-        std::make_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
-        double span = 0.0;
-        for (int h = 0; h < p->g.heads; ++h)
-            for (int piece = 0; piece < sp; ++piece)
-                for (int i = 0; i < p->n_qb; ++i) {
-                    const int u = p->unit_order[i];
-                    const long long n = p->u_row_ptr[u + 1] - p->u_row_ptr[u];
-                    const double cost = (double)(n * (piece + 1) / sp - n * piece / sp) + kPieceTiles;
-                    std::pop_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
-                    sm_free.back() += cost;
-                    span = std::max(span, sm_free.back());
-                    std::push_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
-                }
-        double t = span * kTileSeconds;
-        if (sp > 1)
-            t += 2.0 * sp * (double)p->q_tokens * p->g.heads * (p->g.head_dim + 1) * 4.0 / kBytesPerSecond;
-        if (sp == 1 || t < best_t) { best_t = t; best = sp; }
-    }
-    p->n_split = best;
+    p->n_split = choose_split(*p, sms);
     // one allocation of what the kernels read: u_row_ptr | u_col | u_flags | unit_order | u_mask |
     // masks | (split workspace: partial O | partial lse); the per-q-tile lists, the slot frames
     // and the radius table stay on the host (exports, mask construction)
