@@ -56,7 +56,7 @@ extern "C" {
 enum {
     VDIT_OK = 0,
     VDIT_ERR_INVALID_ARG = -1,  /* null pointer, size out of range, inconsistent geometry     */
-    VDIT_ERR_UNSUPPORTED = -2,  /* valid request this build does not implement (head_dim,...) */
+    VDIT_ERR_UNSUPPORTED = -2,  /* valid request the library does not implement (head_dim,...) */
     VDIT_ERR_MISALIGNED = -3,   /* a tensor pointer is not 16-byte aligned                    */
     VDIT_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (message has the reason)  */
     VDIT_ERR_TIMEOUT = -5,      /* a bounded wait inside a kernel gave up (vdit_get_status)    */
