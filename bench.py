@@ -536,6 +536,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    world = dist_env()[1]
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} but {world} rank(s): launch one process per GPU "
+                 f"(python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py ...)")
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
