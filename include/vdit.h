@@ -191,7 +191,8 @@ VDIT_API void vdit_plan_destroy(vdit_plan* p);
  * [heads, q_tokens] (natural-log sum of exp of the kept scaled scores) or NULL. scale > 0
  * (1/sqrt(head_dim) for the Wan2.1 shapes). Rows with no kept key get o = 0, lse = -inf.
  * head_dim 64 or 128 (the plan accepts no other). With VDIT_MASK_DYNAMIC the output is the
- * softmax over the kept candidates only, and lse their log-sum-exp. */
+ * softmax over the kept candidates only, and lse their log-sum-exp. When vdit_get_status reports
+ * VDIT_ERR_TIMEOUT for a call, its o and lse are unspecified. */
 VDIT_API int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
                       void* o, float* lse, float scale, void* stream);
 
@@ -209,10 +210,14 @@ VDIT_API int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_
  * The call itself makes no cudaMalloc / cudaFree or other allocating call: the plan must already
  * be uploaded, and the RoPE tables for its bands must already exist on the device (any earlier
  * vdit_kv_append, vdit_rope3d_apply or vdit_attn_forward builds them; otherwise
- * VDIT_ERR_INVALID_ARG). The first call on each device looks up the buffer's device address
- * (cudaGetSymbolAddress), so make that first call before any stream capture. All calls share
- * the buffer and it keeps the last call's contents (nothing in it needs to start at zero): calls
- * whose kernels may overlap on the GPU, e.g. on two streams of one device, race on it. */
+ * VDIT_ERR_INVALID_ARG). The buffer lives in the library's attention module: under CUDA's lazy
+ * module loading that module, buffer included, is loaded on a device at its first use there, and
+ * vdit_plan_upload makes that first use (it also resolves the buffer's device address with
+ * cudaGetSymbolAddress), so this call, which needs a plan uploaded to the current device, only
+ * launches kernels. All calls share the buffer and it keeps the last call's contents (nothing in it
+ * needs to start at zero): calls whose kernels may overlap on the GPU, e.g. on two streams of one
+ * device, race on it. After a call whose kernel timed out (VDIT_ERR_TIMEOUT) o and lse are
+ * unspecified (the merge may have read an earlier call's partial results). */
 VDIT_API int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, const void* k_cache,
                                        const void* v_cache, void* o, float* lse, float scale,
                                        void* stream);

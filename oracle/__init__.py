@@ -6,7 +6,8 @@ reference leg of ``bench.py`` import this package. It shares no code with the pr
 
 Every function converts numpy arrays to contiguous C buffers and calls the C oracle; the
 arithmetic lives in ``vdit_oracle.c`` (see its header for the pages each step follows), except
-``qkv_project``, whose one step is numpy's float64 matrix product.
+``qkv_project`` and the logits of ``dynamic_keep``, whose one step is numpy's float64 matrix
+product.
 """
 from __future__ import annotations
 
@@ -58,6 +59,7 @@ def lib() -> ctypes.CDLL:
         L.vo_kv_append.argtypes = [_f64p, _f64p, _I, _I, _I, _I, _I, _I, _I, _I, _D,
                                    _f64p, _f64p, _I, _I]
         L.vo_threads.restype = _I
+        L.vo_round_bf16.argtypes = [_f64p, _L]
         _lib = L
     return _lib
 
@@ -161,27 +163,59 @@ def attention(q, k, v, mask, scale: float):
     return o, lse
 
 
-def attention_dynamic(q, k, v, cand, scale: float, tau: float):
-    """Attention in the dynamic-threshold mode of "DynamicRad: Content-Adaptive Sparse Attention
-    for Long Video Diffusion", section 2: the pre-softmax logits serve as importance proxies and
-    an adaptive threshold filters the structured candidate set. Reading taken: per head and query
-    row, with z = scale * q . k over the row's candidates (cand [nq, nk], from mask_rows) and
-    z_max their maximum, a candidate is kept iff z >= z_max - tau; then masked softmax attention
-    over the kept keys. The logits are numpy float64 matrix products (a library primitive), the
-    attention is the C oracle's. Returns (o [nq, heads, D], lse [heads, nq], keep [heads, nq, nk])."""
+def round_bf16(x) -> np.ndarray:
+    """x rounded to the nearest bfloat16 value (ties to even), returned as float64."""
+    y = np.array(x, dtype=np.float64, order="C", copy=True)
+    lib().vo_round_bf16(y.reshape(-1), y.size)
+    return y
+
+
+def dynamic_keep(q, k, cand, scale: float, tau: float, logits: str = "f64"):
+    """Keep decision of the dynamic-threshold mode of "DynamicRad: Content-Adaptive Sparse
+    Attention for Long Video Diffusion", section 2: the pre-softmax logits are the importance
+    proxies and an adaptive threshold filters the structured candidate set. Reading taken: per
+    head and query row, with z = scale * q . k over the row's candidates (cand [nq, nk], from
+    mask_rows) and z_max their maximum, a candidate is kept iff z >= z_max - tau.
+
+    logits selects the precision of the decision. "f64": q and k as given. "bf16": q and k are
+    first rounded to bfloat16 (round_bf16), the operand precision of the tensor-core kernel, and
+    the products are summed in float64: a threshold is a decision taken from floating point, and
+    both sides take it in the same precision. The logits are numpy float64 matrix products (a
+    library primitive). Returns (keep [heads, nq, nk] bool, z [heads, nq, nk] with -inf outside
+    the candidates, thr [heads, nq, 1] = z_max - tau)."""
+    if logits not in ("f64", "bf16"):
+        raise ValueError("logits must be 'f64' or 'bf16'")
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
-    v = np.asarray(v, np.float64)
+    if logits == "bf16":
+        q, k = round_bf16(q), round_bf16(k)
     cand = np.asarray(cand).astype(bool)
-    nq, heads, d = q.shape
-    o = np.empty((nq, heads, d))
-    lse = np.empty((heads, nq))
+    nq, heads, _ = q.shape
     keep = np.zeros((heads,) + cand.shape, bool)
+    z_all = np.full((heads,) + cand.shape, -np.inf)
+    thr = np.full((heads, nq, 1), -np.inf)
     for h in range(heads):
         z = scale * (q[:, h] @ k[:, h].T)
         zc = np.where(cand, z, -np.inf)
         zmax = zc.max(axis=1, keepdims=True) if cand.shape[1] else np.full((nq, 1), -np.inf)
         keep[h] = cand & (z >= zmax - tau)
+        z_all[h] = zc
+        thr[h] = zmax - tau
+    return keep, z_all, thr
+
+
+def attention_dynamic(q, k, v, cand, scale: float, tau: float, logits: str = "f64"):
+    """Attention in the dynamic-threshold mode (dynamic_keep's decision, in the precision
+    `logits` selects), then masked softmax attention over the kept keys with the float64 q, k and
+    v (the C oracle's attention). Returns (o [nq, heads, D], lse [heads, nq], keep [heads, nq, nk])."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    nq, heads, d = q.shape
+    keep, _, _ = dynamic_keep(q, k, cand, scale, tau, logits)
+    o = np.empty((nq, heads, d))
+    lse = np.empty((heads, nq))
+    for h in range(heads):
         oh, lh = attention(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], keep[h].astype(np.uint8), scale)
         o[:, h] = oh[:, 0]
         lse[h] = lh[0]

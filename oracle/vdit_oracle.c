@@ -291,3 +291,24 @@ void vo_kv_append(double *k_cache, double *v_cache, int capacity_frames,
 
 /* Number of OpenMP threads the parallel loops above run on (for reporting). */
 int vo_threads(void) { return omp_get_max_threads(); }
+
+/* Rounds each x[i] to the nearest bfloat16 value, ties to even, in place. bfloat16 keeps 8
+ * significant bits and float32's exponent range: for |x| >= 2^-126 the spacing of bfloat16
+ * values around x is 2^(e-7) with e = floor(log2 |x|); below that (subnormal) it is 2^-133.
+ * x / spacing is exact (a power-of-two scaling), and nearbyint rounds it to the nearest integer
+ * with ties to even under the default rounding mode. Results of magnitude 2^128 or more are
+ * infinite (the largest finite bfloat16 is (2 - 2^-7) 2^127). This is the precision in which
+ * the dynamic-threshold mode's keep decision is taken (the tensor core multiplies bfloat16
+ * operands); it is not a step of the attention itself. */
+void vo_round_bf16(double *x, long n)
+{
+    for (long i = 0; i < n; ++i) {
+        double a = x[i];
+        if (a == 0.0 || isnan(a) || isinf(a)) continue;
+        int e = ilogb(a);
+        int step_exp = e < -126 ? -133 : e - 7;
+        double r = ldexp(nearbyint(ldexp(a, -step_exp)), step_exp);
+        if (fabs(r) >= ldexp(1.0, 128)) r = a > 0 ? INFINITY : -INFINITY;
+        x[i] = r;
+    }
+}

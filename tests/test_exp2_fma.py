@@ -1,6 +1,9 @@
-"""Error bound of the FMA-pipe exp2 used for a quarter of the softmax exponentials.
+"""Error bound and provenance of the FMA-pipe exp2 the attention kernel can use for part of the
+softmax exponentials (off by default).
 
-The constants are read from the CUDA source and the device algorithm (Cody-Waite reduction
+The constants are this repository's own fitted cubic, parsed from csrc/attn_fwd.cu; the fit is
+reproduced below (float64 weighted least squares with Lawson's reweighting toward the minimax
+relative error on [-1/2, 1/2], constant term pinned to 1). The device algorithm (Cody-Waite reduction
 x = n + f with n = round(x), |f| <= 1/2; cubic for 2^f in Horner form; n added to the exponent
 field; inputs below -127 clamped) is replayed in float32 with numpy, then compared with the exact
 2^x. The kernel rounds P to bf16 (relative 2^-9), so a relative error below 1.5e-4 is far
@@ -32,6 +35,37 @@ def _exp2_fma(x):
     q = (q * f + c0).astype(np.float32)
     n = t.view(np.int32) - np.int32(0x4B400000)
     return (q.view(np.int32) + (n << 23)).view(np.float32)
+
+
+def _lawson_fit(iters=400):
+    """Cubic 1 + c1 f + c2 f^2 + c3 f^3 minimising the maximum relative error to 2^f on
+    [-1/2, 1/2]: Lawson's algorithm (C. L. Lawson, 1961) iterates weighted least squares,
+    multiplying each sample's weight by its current absolute error, which converges to the
+    minimax (equioscillating) solution."""
+    f = np.linspace(-0.5, 0.5, 4001)
+    e = np.exp2(f)
+    a = np.stack([f / e, f ** 2 / e, f ** 3 / e], axis=1)  # relative error = a c - (1 - 1/e)
+    b = 1.0 - 1.0 / e
+    wt = np.full(f.size, 1.0 / f.size)
+    c = None
+    for _ in range(iters):
+        sw = np.sqrt(wt)
+        c = np.linalg.lstsq(a * sw[:, None], b * sw, rcond=None)[0]
+        r = np.abs(a @ c - b)
+        wt = wt * r
+        wt /= wt.sum()
+    return c, float(np.abs(a @ c - b).max())
+
+
+def test_constants_are_the_minimax_fit():
+    c, best = _lawson_fit()
+    c0, c1, c2, c3 = (float(x) for x in _coeffs())
+    assert c0 == 1.0
+    # the kernel's constants are the fit rounded to float32
+    assert np.allclose([c1, c2, c3], c, rtol=1e-5, atol=0)
+    f = np.linspace(-0.5, 0.5, 4001)
+    mine = np.abs((1 + c1 * f + c2 * f ** 2 + c3 * f ** 3) / np.exp2(f) - 1).max()
+    assert best < 1.02e-4 and mine <= 1.001 * best
 
 
 def test_relative_error_over_the_softmax_range():

@@ -201,18 +201,14 @@ def test_attention_rows_without_keys(q_start, q_frames):
 
 # ----------------------------------------------------------------------------- dynamic threshold
 
-def _bf16(x):
-    return synth.bf16_bits_to_f64(synth.f32_to_bf16_bits(np.asarray(x, np.float32)))
-
-
 def _dynamic_check(w, rows=None, heads=None, q_scale=1.0):
     """Dynamic-threshold parity. The keep decision (logit within tau of the row maximum) is an
     integer decision taken from floating point, so the reference takes it in the kernel's
-    precision: logits of the bf16 rotated q and bf16 K' (fp64 sums; the tensor core's fp32 sums
-    of the same exact bf16 products differ by ~1e-6). Candidates within 2e-5 of their row's
-    threshold may fall either way: a row with one such key must match the reference with that
-    key kept or dropped (no row of these inputs has two). The values are the fp64 oracle's on
-    the decided set."""
+    precision: the oracle's dynamic_keep with logits="bf16" (bf16-rounded rotated q and K',
+    fp64 sums; the tensor core's fp32 sums of the same exact bf16 products differ by ~1e-6).
+    Candidates within 2e-5 of their row's threshold may fall either way: a row with one such key
+    must match the reference with that key kept or dropped (no row of these inputs has two). The
+    values are the fp64 oracle's attention on the decided set."""
     q, k, v = inputs(w, q_scale)
     o, lse, _, _ = run_product(w, q, k, v)
     rows = np.arange(w.q_tokens) if rows is None else rows
@@ -232,12 +228,11 @@ def _dynamic_check(w, rows=None, heads=None, q_scale=1.0):
     cand = oracle.mask_rows(qpos, kpos, kvalid, omask(w)).astype(bool)
     got = f64(o[rows][:, heads])
     n_amb_rows = 0
+    keep_all, z_all, thr_all = oracle.dynamic_keep(qrot, kc.transpose(1, 0, 2), cand, w.scale,
+                                                   w.tau, logits="bf16")
     for hi in range(len(heads)):
-        z = w.scale * (_bf16(qrot[:, hi]) @ _bf16(kc[hi]).T)
-        zmax = np.where(cand, z, -np.inf).max(axis=1, keepdims=True)
-        thr = zmax - w.tau
-        keep = cand & (z >= thr)
-        amb = cand & (np.abs(z - thr) < 2e-5)
+        keep = keep_all[hi]
+        amb = cand & (np.abs(z_all[hi] - thr_all[hi]) < 2e-5)
         assert (amb.sum(axis=1) <= 1).all()
         ref, ref_lse = oracle.attention(qrot[:, hi:hi + 1], kc[hi][:, None], vc[hi][:, None],
                                         keep.astype(np.uint8), w.scale)

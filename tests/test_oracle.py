@@ -471,3 +471,94 @@ def test_dynamic_threshold_kept_sets_grow_with_tau():
         if prev is not None:
             assert (prev <= keep).all()
         prev = keep
+
+
+# ----------------------------------------------------------------------------- bf16 decision rule
+
+def test_round_bf16_hand_worked_values():
+    # spacing 2^-7 on [1, 2): 1 + 2^-8 is a tie -> even (1.0); 1 + 3 * 2^-8 is a tie -> even
+    # (1 + 2^-6); 0.7509765625 = 192.25 * 2^-8 -> 0.75; subnormal spacing 2^-133; overflow -> inf
+    x = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 0.7509765625, -0.7490234375, 3 * 2 ** -135,
+                  2.0 ** 128, 0.0, -1.5])
+    want = np.array([1.0, 1 + 2 ** -6, 0.75, -0.75, 2.0 ** -133, np.inf, 0.0, -1.5])
+    assert np.array_equal(oracle.round_bf16(x), want)
+
+
+def test_round_bf16_equals_torch_float32_to_bfloat16():
+    # for float32 inputs, round-to-nearest-even to 8 significant bits is torch's own conversion
+    x = _rand(77, (20000,)).astype(np.float32) * np.float32(3.0)
+    x[:5] = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 2 ** -130, -2 ** -127, 65504.0], np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_bf16(x.astype(np.float64)), ref)
+
+
+def test_dynamic_keep_bf16_flips_a_decision_the_f64_rule_keeps():
+    # one query q = (1, 0), scale 1, d = 2: logits are the keys' first channels. k0 = 1 - 2^-10
+    # rounds up to 1.0 in bfloat16, k1 = 0.75 is exact. tau = 0.2495:
+    #   f64:  z1 - z0 = 0.75 - 0.9990234375 = -0.2490234375 >= -0.2495  -> both kept
+    #   bf16: z1 - z0 = 0.75 - 1.0 = -0.25 < -0.2495                    -> only k0 kept
+    q = np.array([1.0, 0.0]).reshape(1, 1, 2)
+    k = np.array([[1 - 2 ** -10, 0.0], [0.75, 0.0]]).reshape(2, 1, 2)
+    v = np.array([[2.0, -1.0], [5.0, 3.0]]).reshape(2, 1, 2)
+    cand = np.ones((1, 2), np.uint8)
+    o64, l64, keep64 = oracle.attention_dynamic(q, k, v, cand, 1.0, 0.2495, logits="f64")
+    ob, lb, keepb = oracle.attention_dynamic(q, k, v, cand, 1.0, 0.2495, logits="bf16")
+    assert keep64[0, 0].tolist() == [True, True]
+    assert keepb[0, 0].tolist() == [True, False]
+    # bf16 rule: only key 0 is kept, so o = v0 and lse = its (unrounded) logit
+    assert np.array_equal(ob[0, 0], [2.0, -1.0]) and lse_close(lb[0, 0], 1 - 2 ** -10)
+    # f64 rule: softmax over the two unrounded logits, written out by hand
+    e0, e1 = math.exp(1 - 2 ** -10), math.exp(0.75)
+    assert np.allclose(o64[0, 0], [(2 * e0 + 5 * e1) / (e0 + e1), (-e0 + 3 * e1) / (e0 + e1)], rtol=1e-14)
+    assert lse_close(l64[0, 0], math.log(e0 + e1))
+    # the logits and threshold it returns are the rounded ones
+    _, z, thr = oracle.dynamic_keep(q, k, cand, 1.0, 0.2495, logits="bf16")
+    assert z[0, 0].tolist() == [1.0, 0.75] and thr[0, 0, 0] == 1.0 - 0.2495
+
+
+def lse_close(a, b):
+    return abs(a - b) <= 1e-14 * max(1.0, abs(b))
+
+
+def test_dynamic_keep_rules_agree_on_bf16_exact_operands():
+    # operands that are already bfloat16 values round to themselves: both rules are identical
+    q, k, v, cand = _rand_case(4, nq=12, nk=64, d=16)
+    q, k = oracle.round_bf16(q), oracle.round_bf16(k)
+    for tau in (0.1, 0.7, 3.0):
+        o1, l1, k1 = oracle.attention_dynamic(q, k, v, cand, 0.25, tau, logits="f64")
+        o2, l2, k2 = oracle.attention_dynamic(q, k, v, cand, 0.25, tau, logits="bf16")
+        assert np.array_equal(k1, k2) and np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_dynamic_keep_rules_differ_only_inside_the_rounding_band():
+    # rounding q and k to bfloat16 moves each product q_i k_i by at most (2^-8 + 2^-16) |q_i k_i|
+    # (relative error 2^-8 of each operand), so a logit moves by at most
+    # eps = scale (2^-8 + 2^-16) sum_i |q_i k_i|; a decision can only flip for a candidate whose
+    # f64 logit lies within eps_j + eps_max of the f64 threshold (the row maximum moves too)
+    q, k, v, cand = _rand_case(5, nq=64, nk=400, d=32)
+    scale, tau = 0.3, 2.0
+    k64, z64, thr64 = oracle.dynamic_keep(q, k, cand, scale, tau, logits="f64")
+    kb, _, _ = oracle.dynamic_keep(q, k, cand, scale, tau, logits="bf16")
+    flips = 0
+    for h in range(q.shape[1]):
+        eps = scale * (2 ** -8 + 2 ** -16) * (np.abs(q[:, h]) @ np.abs(k[:, h]).T)
+        eps_max = np.where(cand.astype(bool), eps, 0).max(axis=1, keepdims=True)
+        band = np.abs(z64[h] - thr64[h]) <= eps + eps_max
+        diff = k64[h] != kb[h]
+        assert not (diff & ~band).any()
+        flips += int(diff.sum())
+    # the band is wide enough on these inputs that the two rules really do differ somewhere
+    assert flips > 0
+
+
+def test_dynamic_keep_bf16_limits_in_tau():
+    q, k, v, cand = _rand_case(6)
+    keep, _, _ = oracle.dynamic_keep(q, k, cand, 0.35, 1e9, logits="bf16")
+    assert (keep == cand.astype(bool)[None]).all()
+    keep, _, _ = oracle.dynamic_keep(q, k, cand, 0.35, 1e-12, logits="bf16")
+    qb, kb = oracle.round_bf16(q), oracle.round_bf16(k)
+    for h in range(2):
+        z = np.where(cand.astype(bool), qb[:, h] @ kb[:, h].T, -np.inf)
+        for r in range(1, z.shape[0]):
+            assert keep[h, r].sum() == 1 and keep[h, r, int(np.argmax(z[r]))]
+    assert not keep[:, 0].any()

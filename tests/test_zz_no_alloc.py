@@ -1,5 +1,6 @@
 """The attention entry point that allocates nothing (vdit_attn_forward_noalloc), called through
-the C ABI and checked against vdit_attn_forward on the same inputs.
+the C ABI and checked against vdit_attn_forward on the same inputs (bit-identical: the same
+kernels run on the same plan) and against the fp64 oracle.
 
 It exists for callers that cannot allocate device memory when they run attention (another
 framework owns the GPU's memory through its own pool, or a latency-critical loop must not enter
@@ -14,10 +15,11 @@ import numpy as np
 import pytest
 import torch
 
+import synth
 import video_diffusion_transformer_vdit_b200 as vdit
 from video_diffusion_transformer_vdit_b200.workloads import WORKLOADS, Workload
 
-from _parity import MAX_ABS, REL_RMS, assert_close, dev, f64, geom, inputs, mask
+from _parity import MAX_ABS, REL_RMS, assert_close, dev, f64, geom, inputs, mask, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -59,13 +61,26 @@ def test_noalloc_forward_matches_forward_twice_in_a_row():
     L = vdit.lib()
     rc, o_ref, lse_ref = _call(L.vdit_attn_forward, plan, q, cache, w)
     assert rc == vdit.OK
-    for _ in range(2):  # the second call finds the first call's contents in the buffer
+    # another query between the two calls leaves different partial results in the shared buffer,
+    # so a call that read stale entries instead of its own would not match
+    q_other = dev(synth.qkv_bf16(96, w.q_tokens, w.heads, w.head_dim, "q"))
+    for i in range(2):
         rc, o, lse = _call(L.vdit_attn_forward_noalloc, plan, q, cache, w)
         assert rc == vdit.OK, L.vdit_last_error()
-        assert torch.isfinite(o.float()).all()
-        assert_close(f64(o), f64(o_ref), max_abs=MAX_ABS, rel_rms=REL_RMS)
-        assert torch.max(torch.abs(lse - lse_ref)).item() < 2e-2
+        # the same kernels on the same inputs and plan: bit-identical to vdit_attn_forward
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+        if i == 0:
+            rc, o_x, _ = _call(L.vdit_attn_forward_noalloc, plan, q_other, cache, w)
+            assert rc == vdit.OK and not torch.equal(o_x, o_ref)
     assert vdit.get_status() == vdit.OK
+    # and against the fp64 oracle on sampled rows (first tile, random rows, the ragged last tile)
+    qb, kb, vb = inputs(w)
+    rng = np.random.default_rng(95)
+    rows = np.unique(np.r_[np.arange(0, 64), rng.integers(0, w.q_tokens, 96),
+                           np.arange((w.q_tokens - 1) // 128 * 128, w.q_tokens)])
+    ro, rl = run_oracle(w, qb, kb, vb, rows, [0])
+    assert_close(f64(o[rows]), ro, max_abs=MAX_ABS, rel_rms=REL_RMS)
+    assert np.max(np.abs(lse[0][rows].cpu().numpy() - rl[0])) < 2e-2
 
 
 def test_noalloc_forward_rejects_a_split_larger_than_its_buffer():

@@ -23,9 +23,8 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-# the in-tree build; VDIT_LIBRARY names another build of the same library (e.g. a variant under
-# test) — there is no fallback either way: a missing library is an error
-LIB_PATH = os.environ.get("VDIT_LIBRARY") or os.path.join(_PKG, "libvdit.so")
+# the in-tree build; there is no fallback: a missing library is an error
+LIB_PATH = os.path.join(_PKG, "libvdit.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "vdit.h")
 
 OK = 0

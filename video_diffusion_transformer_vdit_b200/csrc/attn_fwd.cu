@@ -818,10 +818,57 @@ int make_cache_map(CUtensorMap* map, const void* base, int kv_tokens, int heads,
     return VDIT_OK;
 }
 
-int* status_ptr() {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-    return static_cast<int*>(p);
+// Per-device state of this file's kernels, set up once per device with that device current:
+// the dynamic shared-memory opt-in of every attention kernel instance (a function attribute
+// belongs to the function in one device's context), the device addresses of the status word and
+// of the no-allocation scratch buffer (cudaGetSymbolAddress; in host code a __device__ variable's
+// name is only a host-side stand-in), and the SM count. vdit_plan_upload runs this set-up for its
+// device, so the forward calls on an uploaded plan find it done.
+struct DeviceState {
+    bool ready = false;
+    int* status = nullptr;
+    void* noalloc = nullptr;
+    int sms = 148;
+};
+constexpr int kMaxDevices = 256;
+std::mutex g_dev_mu;
+DeviceState g_dev[kMaxDevices];
+
+}  // namespace
+// the no-allocation scratch buffer (its declaration and rules are with the entry point below)
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+namespace {
+
+int device_state(int dev, const DeviceState** out) {
+    if (dev < 0 || dev >= kMaxDevices) return vdit::fail(VDIT_ERR_INVALID_ARG, "device index too large");
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        const void* fns[4] = {(const void*)attn_fwd_kernel<128, false>, (const void*)attn_fwd_kernel<64, false>,
+                              (const void*)attn_fwd_kernel<128, true>, (const void*)attn_fwd_kernel<64, true>};
+        const int bytes[4] = {(int)Layout<128>::kSmemBytes, (int)Layout<64>::kSmemBytes,
+                              (int)Layout<128>::kSmemBytes, (int)Layout<64>::kSmemBytes};
+        for (int i = 0; i < 4; ++i)
+            if (int rc = vdit::cuda_check(cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                               bytes[i]),
+                                          "cudaFuncSetAttribute(attention)"))
+                return rc;
+        void* p = nullptr;
+        if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&p, g_status), "cudaGetSymbolAddress(status)")) return rc;
+        st.status = static_cast<int*>(p);
+        p = nullptr;
+        if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scratch),
+                                      "cudaGetSymbolAddress(no-alloc scratch)"))
+            return rc;
+        st.noalloc = p;
+        if (int rc = vdit::cuda_check(cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev),
+                                      "cudaDeviceGetAttribute"))
+            return rc;
+        st.ready = true;
+    }
+    *out = &st;
+    return VDIT_OK;
 }
 
 // Tensor maps, arguments and launches of one forward pass (the attention kernel for the plan's
@@ -835,19 +882,8 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     const int d = p->g.head_dim;
     if (int rc = make_cache_map(&mk, k_cache, p->kv_tokens, p->g.heads, d)) return rc;
     if (int rc = make_cache_map(&mv, v_cache, p->kv_tokens, p->g.heads, d)) return rc;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        const void* fns[4] = {(const void*)attn_fwd_kernel<128, false>, (const void*)attn_fwd_kernel<64, false>,
-                              (const void*)attn_fwd_kernel<128, true>, (const void*)attn_fwd_kernel<64, true>};
-        const int bytes[4] = {(int)Layout<128>::kSmemBytes, (int)Layout<64>::kSmemBytes,
-                              (int)Layout<128>::kSmemBytes, (int)Layout<64>::kSmemBytes};
-        for (int i = 0; i < 4 && attr_err == cudaSuccess; ++i)
-            attr_err = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]);
-    });
-    if (int rc = vdit::cuda_check(attr_err, "cudaFuncSetAttribute")) return rc;
-    int* status = status_ptr();
-    if (!status) return fail(VDIT_ERR_CUDA, "cannot resolve status word");
+    const DeviceState* ds = nullptr;
+    if (int rc = device_state(dev, &ds)) return rc;
 
     AttnArgs a{};
     a.u_row_ptr = p->d_u_row_ptr;
@@ -866,7 +902,7 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     a.tt = static_cast<const float2*>(tabs.t);
     a.th = static_cast<const float2*>(tabs.h);
     a.tw = static_cast<const float2*>(tabs.w);
-    a.status = status;
+    a.status = ds->status;
     a.skip_loads = g_skip_loads.load(std::memory_order_relaxed);
     a.bt2 = p->g.band_t / 2;
     a.bh2 = p->g.band_h / 2;
@@ -891,10 +927,8 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
         attn_fwd_kernel<64, true><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
     if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
     if (p->n_split > 1) {
-        int sms = 148;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const long long rows = (long long)p->q_tokens * p->g.heads;
-        const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)sms * 8);
+        const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)ds->sms * 8);
         auto* ob = static_cast<__nv_bfloat16*>(o);
         if (d == 128)
             split_combine_kernel<128><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
@@ -945,6 +979,13 @@ extern "C" int vdit_get_status(int* status) {
     return VDIT_OK;
 }
 
+namespace vdit {
+int attn_prepare_device(int dev) {
+    const DeviceState* ds = nullptr;
+    return device_state(dev, &ds);
+}
+}  // namespace vdit
+
 // ------------------------------------------------------------------------------ no-allocation
 // variant of the forward pass
 //
@@ -953,39 +994,18 @@ extern "C" int vdit_get_status(int* status) {
 // fragments that pool), latency-critical loops that must not touch the allocator, and code that
 // must not synchronise the device. vdit_attn_forward takes its key-split scratch from the plan
 // (allocated by vdit_plan_upload); this variant instead writes the partial results into the
-// fixed buffer below, so the call itself allocates nothing.
+// fixed buffer g_noalloc_scratch, so the call itself allocates nothing.
 //
-// The buffer is a file-scope device array: every GPU that loads this library holds its
-// kNoAllocScratchBytes until the process exits, whether or not the variant is used. In host code
-// its name is only a host-side stand-in, so its device address is resolved with
-// cudaGetSymbolAddress once per device (with that device current) on the variant's first call
-// there; that first call should therefore come before any stream capture. All calls share the
-// buffer and it keeps the last call's contents: every partial entry a call reads is written by
-// the same call first, so nothing has to start at zero, but two calls whose kernels overlap on
-// the GPU (different streams, same device) race on it.
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-namespace {
-std::mutex g_noalloc_mu;
-constexpr int kMaxDevices = 256;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-int noalloc_scratch_address(int dev, void** out) {
-    if (dev < 0 || dev >= kMaxDevices) return vdit::fail(VDIT_ERR_INVALID_ARG, "device index too large");
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* ptr = nullptr;
-        if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&ptr, g_noalloc_scratch),
-                                      "cudaGetSymbolAddress(no-alloc scratch)"))
-            return rc;
-        g_noalloc_ptr[dev] = ptr;
-    }
-    *out = g_noalloc_ptr[dev];
-    return VDIT_OK;
-}
-}  // namespace
-
+// The buffer is a file-scope device array: every GPU on which this file's module is loaded holds
+// its kNoAllocScratchBytes until the process exits. Under CUDA's lazy module loading the module
+// (code and buffer) is loaded on first use on each device; vdit_plan_upload, which allocates
+// anyway, makes that first use (it resolves the buffer's device address with
+// cudaGetSymbolAddress, with the device current), so the variant itself, which needs an uploaded
+// plan, only launches. All calls share the buffer and it keeps the last call's contents: every
+// partial entry a successful call reads is written by the same call first, so nothing has to
+// start at zero, but two calls whose kernels overlap on the GPU (different streams, same device)
+// race on it. A call whose kernel timed out (VDIT_ERR_TIMEOUT from vdit_get_status) leaves o and
+// lse unspecified: the merge may have read an earlier call's partials.
 extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, const void* k_cache,
                                          const void* v_cache, void* o, float* lse, float scale,
                                          void* stream) {
@@ -1013,8 +1033,9 @@ extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, cons
                     "this plan's key split needs " + std::to_string(o_bytes_al + l_bytes) +
                         " bytes of scratch; the no-allocation variant's static buffer holds " +
                         std::to_string(kNoAllocScratchBytes) + " (use vdit_attn_forward)");
-    void* scratch = nullptr;
-    if (int rc = noalloc_scratch_address(dev, &scratch)) return rc;
+    const DeviceState* ds = nullptr;
+    if (int rc = device_state(dev, &ds)) return rc;
+    void* scratch = ds->noalloc;
     vdit::RopeTables tabs;
     if (int rc = vdit::find_rope_tables(&p->g, &tabs)) return rc;
     float* ws_o = p->n_split > 1 ? static_cast<float*>(scratch) : nullptr;

@@ -33,6 +33,10 @@ int find_rope_tables(const vdit_geom* g, RopeTables* out);
 // Reads and clears the device status word of the fused QKV projection kernel.
 int qkv_status_take(int* out);
 
+// One-time set-up of the attention kernels on device dev (current): shared-memory opt-in of every
+// kernel instance, device addresses of the status word and of the no-allocation scratch buffer.
+int attn_prepare_device(int dev);
+
 }  // namespace vdit
 
 // Plan object (host schedule + optional device copy).

@@ -369,6 +369,9 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     }
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // the attention kernels' per-device set-up happens here, in a call that allocates anyway, so
+    // that the forward calls on this plan (the no-allocation one included) only launch
+    if (int rc = vdit::attn_prepare_device(dev)) return rc;
     p->n_split = choose_split(*p, sms);
     // one allocation of what the kernels read: u_row_ptr | u_col | u_flags | unit_order | u_mask |
     // masks | (split workspace: partial O | partial lse); the per-q-tile lists, the slot frames

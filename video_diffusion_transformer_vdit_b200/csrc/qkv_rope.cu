@@ -356,11 +356,45 @@ int encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
     return r == CUDA_SUCCESS ? VDIT_OK : vdit::fail(VDIT_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 }
 
+// Per-device set-up, once per device with that device current: the kernel's dynamic shared-memory
+// opt-in (a function attribute belongs to one device's context), the status word's device
+// address and the SM count.
+struct QkvDeviceState {
+    bool ready = false;
+    int* status = nullptr;
+    int sms = 148;
+};
+constexpr int kMaxDevices = 256;
+std::mutex g_qkv_dev_mu;
+QkvDeviceState g_qkv_dev[kMaxDevices];
+
+int qkv_device_state(int dev, QkvDeviceState* out) {
+    if (dev < 0 || dev >= kMaxDevices) return vdit::fail(VDIT_ERR_INVALID_ARG, "device index too large");
+    std::lock_guard<std::mutex> lk(g_qkv_dev_mu);
+    QkvDeviceState& st = g_qkv_dev[dev];
+    if (!st.ready) {
+        if (int rc = vdit::cuda_check(cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                           (int)kGSmemBytes),
+                                      "cudaFuncSetAttribute(qkv_rope)"))
+            return rc;
+        void* sp = nullptr;
+        if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&sp, g_qkv_status), "cudaGetSymbolAddress(status)"))
+            return rc;
+        st.status = static_cast<int*>(sp);
+        if (int rc = vdit::cuda_check(cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev),
+                                      "cudaDeviceGetAttribute"))
+            return rc;
+        st.ready = true;
+    }
+    *out = st;
+    return VDIT_OK;
+}
+
 // One launch over `n_tok` consecutive tokens of the chunk (chunk-local first token tok0) whose K
 // and V rows go to consecutive cache rows starting at cache_row0.
 int launch_part(const vdit_geom* g, const vdit::RopeTables& tabs, const uint8_t* x, const void* w,
                 int d_model, int start_frame, int tok0, int n_tok, uint8_t* q, void* k_cache, void* v_cache,
-                long long cap_tok, long long cache_row0, cudaStream_t st) {
+                long long cap_tok, long long cache_row0, const QkvDeviceState& ds, cudaStream_t st) {
     const int hd = g->heads * g->head_dim, d = g->head_dim;
     CUtensorMap mx, mw, mq, mk, mv;
     {
@@ -406,14 +440,9 @@ int launch_part(const vdit_geom* g, const vdit::RopeTables& tabs, const uint8_t*
     a.bt2 = g->band_t / 2;
     a.bh2 = g->band_h / 2;
     a.bw2 = g->band_w / 2;
-    void* sp = nullptr;
-    if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&sp, g_qkv_status), "status word")) return rc;
-    a.status = static_cast<int*>(sp);
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    a.status = ds.status;
     const int tiles = a.n_tiles_m * a.n_tiles_n;
-    const int grid = std::min(tiles, sms);
+    const int grid = std::min(tiles, ds.sms);
     qkv_rope_kernel<<<grid, kGThreads, kGSmemBytes, st>>>(mx, mw, mq, mk, mv, a);
     return vdit::cuda_check(cudaGetLastError(), "qkv_rope kernel launch");
 }
@@ -451,13 +480,10 @@ extern "C" int vdit_qkv_rope(const vdit_geom* g, const void* x, const void* w, i
     if (ft * n_frames > (1 << 30)) return fail(VDIT_ERR_UNSUPPORTED, "chunk too large");
     vdit::RopeTables tabs;
     if (int rc = vdit::get_rope_tables(g, &tabs)) return rc;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)kGSmemBytes);
-    });
-    if (int rc = vdit::cuda_check(attr_err, "cudaFuncSetAttribute")) return rc;
+    int dev = 0;
+    if (int rc = vdit::cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    QkvDeviceState ds;
+    if (int rc = qkv_device_state(dev, &ds)) return rc;
     // frames of the chunk go to slots (frame mod capacity): one launch per run of consecutive
     // slots (two when the chunk wraps around the end of the ring)
     const long long cap_tok = ft * capacity_frames;
@@ -468,7 +494,7 @@ extern "C" int vdit_qkv_rope(const vdit_geom* g, const void* x, const void* w, i
         const int run = std::min(n_frames - f, capacity_frames - slot);
         if (int rc = launch_part(g, tabs, static_cast<const uint8_t*>(x), w, d_model, start_frame, (int)(f * ft),
                                  (int)(run * ft), static_cast<uint8_t*>(q), k_cache, v_cache, cap_tok,
-                                 (long long)slot * ft, st))
+                                 (long long)slot * ft, ds, st))
             return rc;
         f += run;
     }
