@@ -254,6 +254,97 @@ def traffic_per_launch(w):
         return None, None
 
 
+def _nvtx(name):
+    """NVTX range around a timed region (visible to Nsight tools; a no-op otherwise)."""
+    import contextlib
+    try:
+        return torch.cuda.nvtx.range(name)
+    except Exception:  # pragma: no cover - NVTX unavailable
+        return contextlib.nullcontext()
+
+
+def _time_back_to_back(fn, n, stream):
+    """Mean device time (ms) of fn() over n back-to-back calls on `stream` (CUDA events)."""
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def time_append(vdit, g, capacity_frames, n_frames, start_frame, dev, stream, n=20):
+    """vdit_kv_append of one n_frames chunk, timed back to back over distinct (source, cache)
+    sets whose total exceeds L2, so no launch finds its input in L2 and each pays for the
+    write-back its predecessor left there. Returns (ms, algorithmic bytes: read K, V + write K',
+    V)."""
+    ft = g.grid_h * g.grid_w
+    shape = (n_frames * ft, g.heads, g.head_dim)
+    per_set = 4 * int(np.prod(shape)) * 2
+    n_sets = max(2, min(8, -(-400_000_000 // per_set)))
+    gen = torch.Generator(device=dev).manual_seed(11)
+    sets = []
+    for _ in range(n_sets):
+        k = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        v = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        cs = (g.heads, capacity_frames * ft, g.head_dim)
+        sets.append((k, v, torch.zeros(cs, dtype=torch.bfloat16, device=dev),
+                     torch.zeros(cs, dtype=torch.bfloat16, device=dev)))
+
+    def one(i):
+        k, v, kc, vc = sets[i % n_sets]
+        vdit.kv_append(kc, vc, g, capacity_frames, k, v, start_frame)
+
+    for i in range(n_sets):
+        one(i)
+    with _nvtx(f"kv_append {n_frames} frames x {g.heads} heads"):
+        ms = _time_back_to_back(one, n, stream)
+    return ms, per_set
+
+
+def time_workload(vdit, w, dev, stream, burst_peak, n=10):
+    """Attention forward (plus the split merge, when the plan splits) of workload w on seeded
+    device-generated N(0, 1) bf16 inputs: its KV history appended first, then n timed launches
+    after 3 warm-up launches. Inputs exceed L2 (cache K and V, Q, O)."""
+    g = vdit.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, w.bands, w.theta)
+    m = vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, w.tau)
+    ft = w.frame_tokens
+    gen = torch.Generator(device=dev).manual_seed(1000 + w.id)
+    cache = vdit.KVCache(g, w.capacity_frames, device=dev)
+    for s, nf in w.appends:
+        shape = (nf * ft, w.heads, w.head_dim)
+        k = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        v = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        cache.append(k, v, s)
+        del k, v
+    q = torch.randn((w.q_tokens, w.heads, w.head_dim), device=dev, generator=gen).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    t0 = time.perf_counter()
+    plan = vdit.Plan(g, m, w.q_start, w.q_frames, cache=cache)
+    t_plan = time.perf_counter() - t0
+    for _ in range(3):
+        vdit.attn_forward(plan, q, cache, out=o, scale=w.scale)
+    with _nvtx(f"attention workload {w.id}"):
+        ms = _time_back_to_back(lambda i: vdit.attn_forward(plan, q, cache, out=o, scale=w.scale), n, stream)
+    info = plan.info
+    flops = plan.flops()
+    tf = flops / (ms * 1e-3) / 1e12
+    status = vdit.get_status()
+    return {"workload": w.name, "mask": MASK_NAMES[w.mask_kind],
+            "q_tokens": w.q_tokens, "kv_tokens": w.kv_tokens, "heads": w.heads,
+            "attn_fwd_ms": ms, "tflops": tf, "frac_of_burst_peak": tf / burst_peak,
+            "kept_fraction": info["kept_pairs"] / (w.q_tokens * w.kv_tokens),
+            "tiles": info["tiles"], "full_tiles": info["full_tiles"],
+            "kv_splits": info["kv_splits"],
+            "launches": 1 + (1 if info["kv_splits"] > 1 else 0),
+            "plan_host_ms": 1e3 * t_plan, "status": status,
+            "how": "%d back-to-back launches after 3 warm-up, CUDA events; ms includes the "
+                   "split merge kernel when kv_splits > 1; TFLOP/s counts 4*d per kept pair"
+                   % n}
+
+
 def run_gpu(args, w):
     import video_diffusion_transformer_vdit_b200 as vdit
 
@@ -321,11 +412,12 @@ def run_gpu(args, w):
         time.sleep(0.3)
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    t1.record(stream)
-    barrier()
+    with _nvtx("timed steps"):
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        barrier()
     clk = clocks.stop() if clocks else None
     ms = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms / args.steps
@@ -344,35 +436,44 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
     r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_rope = 20
-    r0.record(stream)
-    for i in range(n_rope):
-        vdit.rope3d_apply(xs[i % 4], g, w.q_start, out=ys[i % 4])
-    r1.record(stream)
+    with _nvtx("rope3d_apply"):
+        r0.record(stream)
+        for i in range(n_rope):
+            vdit.rope3d_apply(xs[i % 4], g, w.q_start, out=ys[i % 4])
+        r1.record(stream)
     torch.cuda.synchronize()
     rope_ms = r0.elapsed_time(r1) / n_rope
     del xs, ys
     rope_bytes = 2 * q.numel() * 2
 
-    # sequence-to-head pack (vdit_seq_pack) of Q as one of two sequence-parallel ranks would:
-    # RoPE at the global positions into the [2, tokens, heads / 2, d] all-to-all layout; back to
-    # back over two input / output pairs (400 MB in all)
+    # sequence-to-head pack (vdit_seq_pack) as rank 0 of two sequence-parallel ranks: RoPE of Q and K
+    # at the global positions, Q, K and V of half the tokens into the all-to-all layout (the block
+    # of the other rank) and the own head-sharded buffers, in one launch; back to back over two
+    # distinct input / output sets (1.2 GB in all)
     pack = None
     if g.heads % 2 == 0:
-        xs = [q, torch.empty_like(q).copy_(q)]
-        ss = [torch.empty(2, q.shape[0], g.heads // 2, g.head_dim, dtype=q.dtype, device=q.device)
-              for _ in range(2)]
+        n_half = q.shape[0] // 2
+        hg = g.heads // 2
+        sets = []
+        for _ in range(2):
+            ins = [q[:n_half].clone() for _ in range(3)]
+            send = torch.empty(2, 3, n_half, hg, g.head_dim, dtype=q.dtype, device=q.device)
+            full = tuple(torch.empty(2 * n_half, hg, g.head_dim, dtype=q.dtype, device=q.device)
+                         for _ in range(3))
+            sets.append((ins, send, full))
+
+        def one_pack(i):
+            ins, send, full = sets[i % 2]
+            vdit.seq_pack(ins[0], ins[1], ins[2], g, w.q_start, 0, 2, send, full)
+
         for i in range(2):
-            vdit.seq_pack(xs[i], ss[i], g, w.q_start, q.shape[0], 2)
-        torch.cuda.synchronize()
-        r0.record(stream)
-        for i in range(20):
-            vdit.seq_pack(xs[i % 2], ss[i % 2], g, w.q_start, q.shape[0], 2)
-        r1.record(stream)
-        torch.cuda.synchronize()
-        pack_ms = r0.elapsed_time(r1) / 20
-        pack = {"ms": pack_ms, "gbs": rope_bytes / (pack_ms * 1e-3) / 1e9,
-                "frac_hbm": rope_bytes / (pack_ms * 1e-3) / 1e9 / peaks()[0]["hbm_gbs"]}
-        del xs, ss
+            one_pack(i)
+        with _nvtx("seq_pack"):
+            pack_ms = _time_back_to_back(one_pack, 20, stream)
+        pack_bytes = 3 * 2 * n_half * g.heads * g.head_dim * 2
+        pack = {"ms": pack_ms, "bytes": pack_bytes, "gbs": pack_bytes / (pack_ms * 1e-3) / 1e9,
+                "frac_hbm": pack_bytes / (pack_ms * 1e-3) / 1e9 / peaks()[0]["hbm_gbs"]}
+        del sets
 
     # fused QKV projection + RoPE + cache append (vdit_qkv_rope) of the step's newest frames,
     # d_model = heads * head_dim (as in Wan2.1), random bf16 weights, its own cache
@@ -398,6 +499,31 @@ def run_gpu(args, w):
         qkv = {"ms": qkv_ms, "tflops": 2.0 * n_tok * dm * 3 * dm / (qkv_ms * 1e-3) / 1e12,
                "shape": f"[{n_tok}, {dm}] x [{3 * dm}, {dm}]^T"}
         del xq, wq, qc, qo
+
+    # KV append on its own, over distinct buffers (no deferred write-back into the next
+    # kernel): the clip-sized append of this workload and the 3-frame chunks of the Wan2.1-1.3B
+    # (12 heads) and Wan2.1-14B (40 heads) decode
+    appends = {}
+    pk0 = peaks()[0]
+    for name, heads, nf, start in (("clip", g.heads, n_last, s_last),
+                                   ("chunk_1.3b_h12", 12, 3, 18), ("chunk_14b_h40", 40, 3, 396)):
+        ga = vdit.Geometry(g.grid_h, g.grid_w, heads, g.head_dim, g.bands, g.theta)
+        a_ms, a_bytes = time_append(vdit, ga, w.capacity_frames if name == "clip" else 21, nf,
+                                    start, dev, stream)
+        gbs = a_bytes / (a_ms * 1e-3) / 1e9
+        appends[name] = {"frames": nf, "heads": heads, "ms": a_ms, "bytes": a_bytes, "gbs": gbs,
+                         "frac_hbm": gbs / pk0["hbm_gbs"]}
+    torch.cuda.synchronize()
+
+    # the other attention configurations, timed in the same run (not part of the step)
+    per_workload = {}
+    if not args.no_per_workload:
+        for wid in (2, 3, 4, 5, 6):
+            if wid == w.id:
+                continue
+            per_workload[str(wid)] = time_workload(vdit, WORKLOADS[wid], dev, stream,
+                                                   pk0["bf16_tflops"])
+            torch.cuda.empty_cache()
 
     # End to end through the public API: every step copies its Q, K, V from pinned host memory
     # and its O back to pinned host memory. Inputs and outputs are double-buffered and the copies
@@ -453,7 +579,16 @@ def run_gpu(args, w):
 
     if rank == 0:
         pk, src = peaks()
-        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        # the attention kernel is timed in a short region: the burst peak applies unless the
+        # region ran for a second or more, or the SM clock sat well below its maximum
+        # (power-capped), where the sustained peak (measured under the cap) does
+        timed_s = ms * 1e-3
+        clk_ok = bool(clk and clk.get("sm_mhz") and clk.get("sm_max_mhz")
+                      and clk["sm_mhz"] >= 0.95 * clk["sm_max_mhz"])
+        burst = timed_s < 1.0 and (clk_ok or not clk or not clk.get("sm_mhz"))
+        peak = pk["bf16_tflops"] if burst else pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        peak_kind = ("bf16 dense, burst (%s): timed region %.2f s at full clock" % (src, timed_s)
+                     if burst else "bf16 dense, sustained (%s): timed region %.2f s" % (src, timed_s))
         achieved = flops / (attn_ms * 1e-3) / 1e12
         traffic, tnote = traffic_per_launch(w)
         cpu = None
@@ -482,8 +617,10 @@ def run_gpu(args, w):
                 "kept_fraction": info["kept_pairs"] / (w.q_tokens * w.kv_tokens)}),
             "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_kind": f"bf16 dense, sustained ({src})",
+                         "peak_kind": peak_kind,
                          "frac_of_burst_peak": achieved / pk["bf16_tflops"],
+                         "frac_of_sustained_peak": achieved / pk.get("bf16_tflops_sustained",
+                                                                     pk["bf16_tflops"]),
                          "traffic": traffic, "traffic_note": tnote,
                          "algorithmic": "4*head_dim FLOP per kept (query, key, head): %.4g per launch" % flops},
             "cpu_baseline": cpu,
@@ -502,19 +639,26 @@ def run_gpu(args, w):
             "clocks": clk,
             "kernels": {
                 "attn_fwd_ms": attn_ms, "attn_fwd_tflops": achieved,
-                "kv_append_ms": app_ms, "kv_append_gbs": append_bytes / (app_ms * 1e-3) / 1e9,
-                "kv_append_frac_hbm": append_bytes / (app_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "kv_append_ms": appends["clip"]["ms"], "kv_append_gbs": appends["clip"]["gbs"],
+                "kv_append_frac_hbm": appends["clip"]["frac_hbm"],
+                "kv_append": dict(appends, how="vdit_kv_append alone, 20 launches back to back "
+                                  "over distinct source and cache buffers (> 400 MB in all); "
+                                  "bytes = read K, V + write K', V"),
+                "kv_append_in_step_ms": app_ms,
+                "kv_append_in_step_gbs": append_bytes / (app_ms * 1e-3) / 1e9,
                 "rope3d_apply_ms": rope_ms, "rope3d_apply_gbs": rope_bytes / (rope_ms * 1e-3) / 1e9,
                 "rope3d_apply_frac_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "hbm_peak_gbs": pk["hbm_gbs"],
                 "seq_pack": None if pack is None else dict(
-                    pack, how="vdit_seq_pack of Q for 2 ranks (RoPE + all-to-all layout), read + "
-                              "write bytes, not part of the step"),
+                    pack, how="vdit_seq_pack of Q, K, V of one of 2 sequence-parallel ranks (RoPE "
+                              "of Q and K + all-to-all layout, one launch), read + write bytes, "
+                              "not part of the step"),
                 "qkv_rope": None if qkv is None else dict(
                     qkv, frac_of_sustained_peak=qkv["tflops"] / peak,
                     frac_of_burst_peak=qkv["tflops"] / pk["bf16_tflops"],
                     how="vdit_qkv_rope: X W^T on tcgen05, RoPE of Q and K, K' and V into the "
                         "ring cache; 10 launches back to back, not part of the step")},
+            "per_workload": per_workload,
             "status": status,
         }
         print(json.dumps(line), flush=True)
@@ -533,6 +677,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip timing the other attention configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -143,6 +143,13 @@ VDIT_API int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int s
 VDIT_API int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache, int capacity_frames,
                    const void* k, const void* v, int start_frame, int n_frames, void* stream);
 
+/* Ring write of an already rotated chunk ([CRoPE] 2.A cache of past chunks; 2.C, when the RoPE
+ * ran in the producer, e.g. vdit_seq_pack with rotate): as vdit_kv_append, but K' is k_rotated
+ * copied unchanged (bit-exact) instead of RoPE(k). Same arguments, layout and checks. */
+VDIT_API int vdit_kv_write(const vdit_geom* g, void* k_cache, void* v_cache, int capacity_frames,
+                           const void* k_rotated, const void* v, int start_frame, int n_frames,
+                           void* stream);
+
 /* Tile schedule (host only; [DR] sec. 2 and [WF] masks): queries are q_frames frames starting at
  * global frame q_start_frame; keys are the capacity_frames-frame ring cache holding global frames
  * kv_first_frame .. kv_last_frame (at most capacity_frames of them; other slots empty).
@@ -196,6 +203,13 @@ VDIT_API void vdit_plan_destroy(vdit_plan* p);
 VDIT_API int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
                       void* o, float* lse, float scale, void* stream);
 
+/* vdit_attn_forward with queries that are already rotated at the plan's query positions
+ * ([CRoPE] 2.C: the RoPE runs in the producer of Q, e.g. vdit_seq_pack with rotate or
+ * vdit_qkv_rope): the Q tile is loaded as given. Same arguments, results and error codes. */
+VDIT_API int vdit_attn_forward_rotated(const vdit_plan* p, const void* q_rotated, const void* k_cache,
+                                       const void* v_cache, void* o, float* lse, float scale,
+                                       void* stream);
+
 /* Attention forward that allocates nothing. No passage of the source pages has a counterpart:
  * this is a service for callers that cannot allocate device memory when they run attention,
  * for instance code running while another framework owns the GPU's memory through its own
@@ -239,17 +253,36 @@ VDIT_API int vdit_qkv_rope(const vdit_geom* g, const void* x, const void* w, int
                            int start_frame, int n_frames, void* q_out, void* k_cache, void* v_cache,
                            int capacity_frames, void* stream);
 
-/* Sequence-to-head pack of the Ulysses-style exchange ([CRoPE] 2.A sequence split over ranks,
- * 2.B global time index, 2.C one fused all-to-all that gathers the sequence and splits the heads,
- * with the RoPE fused in). x: this rank's tokens, device bf16 [n_tokens, heads, head_dim], chunk-
- * local tokens tok0 .. tok0 + n_tokens - 1 of a chunk whose first frame is start_frame. send:
- * device bf16 [n_ranks][n_tokens][heads / n_ranks][head_dim]: block r holds heads
- * r * heads / n_ranks .. (r + 1) * heads / n_ranks - 1, rotated at their global positions when
- * rotate != 0 (as vdit_rope3d_apply), copied unchanged otherwise (V). An all-to-all of the n_ranks
- * equal blocks then leaves every rank its heads for all tokens in sequence order. n_ranks must
- * divide heads; x and send must not overlap. */
-VDIT_API int vdit_seq_pack(const vdit_geom* g, const void* x, void* send, int start_frame,
-                           long long tok0, long long n_tokens, int n_ranks, int rotate, void* stream);
+/* Sequence-to-head pack of the Ulysses-style exchange ([CRoPE] 2.A: the sequence is split over
+ * the ranks; 2.B: the global time index, so each rank rotates its own tokens without asking
+ * another for positions; 2.C: one fused all-to-all that gathers the sequence and splits the
+ * heads, for Q, K and V together). Rank `rank` of n_ranks holds the chunk-local tokens
+ * rank * n_tokens .. (rank + 1) * n_tokens - 1 of a chunk whose first frame is start_frame:
+ * q, k, v: device bf16 [n_tokens, heads, head_dim] (g->heads = all heads; n_ranks divides it).
+ * Writes, in one launch:
+ *   send: device bf16 [n_ranks][3][n_tokens][heads / n_ranks][head_dim]; block r (r != rank) holds
+ *     Q, K, V of the heads rank r owns (heads r * heads / n_ranks ..), ready to be sent to rank r
+ *     as three contiguous messages; block `rank` is not written (may be NULL when n_ranks == 1);
+ *   q_full, k_full, v_full: device bf16 [n_ranks * n_tokens][heads / n_ranks][head_dim], the
+ *     head-sharded buffers of this rank: rows rank * n_tokens .. get this rank's own block; the
+ *     exchange fills the other rows with the blocks the other ranks send.
+ * With rotate != 0, Q and K are rotated at their global positions (as vdit_rope3d_apply); V is
+ * always a bit-exact copy. The consumers of rotated data are vdit_kv_write (K', V into the ring)
+ * and vdit_attn_forward_rotated. No output may overlap an input or another output. */
+VDIT_API int vdit_seq_pack(const vdit_geom* g, const void* q, const void* k, const void* v, void* send,
+                           void* q_full, void* k_full, void* v_full, int rank, int n_ranks,
+                           int start_frame, long long n_tokens, int rotate, void* stream);
+
+/* Head-to-sequence unpack of the return exchange after attention ([CRoPE] 2.A-2.C, the second
+ * all-to-all of the sequence-parallel step). Rank `rank` computed attention for heads
+ * rank * heads / n_ranks .. of all n_ranks * n_tokens tokens; rank r sent it the output rows of
+ * the rank's own tokens for r's heads. recv: device bf16 [n_ranks][n_tokens][heads / n_ranks]
+ * [head_dim] (block r from rank r; block `rank` unused, recv may be NULL when n_ranks == 1);
+ * own: device bf16 [n_tokens][heads / n_ranks][head_dim], this rank's own output rows for its
+ * tokens; out: device bf16 [n_tokens, heads, head_dim], out[n, r * heads / n_ranks + j, :] =
+ * block r row n head j. A copy (bit-exact); out must not overlap recv or own. */
+VDIT_API int vdit_seq_unpack(const vdit_geom* g, const void* recv, const void* own, void* out, int rank,
+                             int n_ranks, long long n_tokens, void* stream);
 
 /* Reads and clears the current device's kernel status word: *status = VDIT_OK, or
  * VDIT_ERR_TIMEOUT when a bounded wait in a kernel gave up since the last read. Synchronises the

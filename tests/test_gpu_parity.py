@@ -141,18 +141,21 @@ def test_attention_medium_full(name):
     _full_check(MEDIUM[name])
 
 
-def test_attention_sharp_softmax():
+@pytest.mark.parametrize("name", ["causal_radial", "dense"])
+def test_attention_sharp_softmax(name):
     # Q scaled by 4: logits of standard deviation ~4 and a peaked softmax (|o| ~ 1), where the
     # relative-RMS bound is the binding one. The kernel multiplies bf16 operands, so the rotated
     # q and k carry a relative rounding of up to 2^-9 per element; on 128-term dot products with
     # |q_i k_i| * scale ~ 0.35 that moves a logit by ~0.015 typically (a few times that at the
     # tail), i.e. a softmax weight by a few percent, so single outputs near 1 can move by several
-    # 1e-2. Bound: max-abs 0.1 (5x the dense bound), relative RMS 1e-2 unchanged.
-    w = MEDIUM["causal_radial"]
+    # 1e-2. Observed on B200 for these inputs: max-abs 0.044 (causal_radial) and 0.026 (dense),
+    # relative RMS 5.1e-3 and 4.9e-3, lse 0.022 and 0.025. Bounds: max-abs 0.09 and lse 0.05 (about
+    # twice the larger observation), relative RMS 1e-2 unchanged.
+    w = MEDIUM[name]
     q, k, v = inputs(w, 4.0)
     o, lse, _, _ = run_product(w, q, k, v)
     ro, rl = run_oracle(w, q, k, v, np.arange(w.q_tokens), range(w.heads))
-    assert_close(f64(o), ro, max_abs=0.1, rel_rms=1e-2)
+    assert_close(f64(o), ro, max_abs=0.09, rel_rms=1e-2)
     assert np.max(np.abs(lse.cpu().numpy() - rl)) < 5e-2
 
 

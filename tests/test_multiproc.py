@@ -1,9 +1,12 @@
-"""The multi-GPU bench path runs one independent replica per rank (weak scaling); its only
-collective is the max-over-ranks step time. This checks that reduction and the whole-job
-throughput formula with two gloo ranks on CPU."""
+"""Multi-process host logic on gloo ranks (CPU): the bench's max-over-ranks step time and
+whole-job throughput (its replicas share no data-path collective); the sequence-parallel
+attention step (pack, one batched exchange of Q, K and V, ring write, attention of the rank's
+heads, return exchange, unpack) with the oracle standing in for the device kernels; and Wave
+Parallelism's K/V push."""
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -51,60 +54,131 @@ def test_single_rank_needs_no_process_group():
     assert bench.aggregate_tflops(1, 1e12, 1.0) == pytest.approx(1000.0)
 
 
-# ----------------------------------------------------------------------------- sequence -> heads
+# ----------------------------------------------------------------------------- sequence parallel
 
-def _oracle_pack(x, send, g, start_frame, tok0, n_ranks, rotate=True, stream=None):
-    """CPU stand-in of vdit_seq_pack for the gloo test (test infrastructure: the oracle's RoPE
-    at the tokens' global positions, then the [ranks, tokens, heads / ranks, D] layout)."""
-    import numpy as np
+def _oracle_pack(q, k, v, g, start_frame, rank, n_ranks, send, full, rotate=True, stream=None):
+    """CPU stand-in of vdit_seq_pack for the gloo test (test infrastructure: the oracle's RoPE of
+    q and k at the shard's global positions, then the [ranks, 3, tokens, heads / ranks, D] send
+    layout and the own block into the head-sharded buffers)."""
     import oracle
-    n = x.shape[0]
-    y = x.double().numpy()
+    n = q.shape[0]
+    tok0 = rank * n
+    og = oracle.Geometry(g.grid_h, g.grid_w, g.heads, g.head_dim, *g.bands, g.theta)
+    pos = tuple(p[tok0:] for p in oracle.positions(tok0 + n, g.grid_h, g.grid_w, start_frame))
+    xs = [t.double().numpy() for t in (q, k, v)]
     if rotate:
-        pos = oracle.positions(tok0 + n, g.grid_h, g.grid_w, start_frame)
-        og = oracle.Geometry(g.grid_h, g.grid_w, g.heads, g.head_dim, *g.bands, g.theta)
-        y = oracle.rope3d(y, tuple(p[tok0:] for p in pos), og)
-    hpr = g.heads // n_ranks
-    send.copy_(torch.from_numpy(np.ascontiguousarray(
-        y.reshape(n, n_ranks, hpr, g.head_dim).transpose(1, 0, 2, 3))).to(send.dtype))
-    return send
+        xs[0], xs[1] = oracle.rope3d(xs[0], pos, og), oracle.rope3d(xs[1], pos, og)
+    hg = g.heads // n_ranks
+    for x in range(3):
+        blocks = torch.from_numpy(xs[x].reshape(n, n_ranks, hg, g.head_dim).transpose(1, 0, 2, 3).copy())
+        for r in range(n_ranks):
+            if r == rank:
+                full[x][rank * n:(rank + 1) * n] = blocks[r]
+            else:
+                send[r, x] = blocks[r]
 
 
-def _seq_worker(rank, world, port, out):
+def _oracle_unpack(recv, own, out, g, rank, n_ranks, stream=None):
+    """CPU stand-in of vdit_seq_unpack (a copy)."""
+    hg = g.heads // n_ranks
+    for r in range(n_ranks):
+        out[:, r * hg:(r + 1) * hg] = own if r == rank else recv[r]
+    return out
+
+
+SP_GRID = (3, 4)        # 12 tokens per latent frame
+SP_HEADS, SP_D = 6, 64
+# the chunk is frames 9..11 (36 tokens); the ring (10 frames) also holds frames 3..8
+
+
+def _sp_inputs():
+    import synth
+    ft = SP_GRID[0] * SP_GRID[1]
+    n_kv = 9 * ft  # frames 3..11
+    k = synth.bf16_bits_to_f64(synth.qkv_bf16(31, n_kv, SP_HEADS, SP_D, "k"))
+    v = synth.bf16_bits_to_f64(synth.qkv_bf16(31, n_kv, SP_HEADS, SP_D, "v"))
+    q = synth.bf16_bits_to_f64(synth.qkv_bf16(31, 3 * ft, SP_HEADS, SP_D, "q"))
+    return q, k, v
+
+
+def _sp_reference():
+    """Single-process oracle: the chunk's block-causal attention over frames 3..11, all heads."""
+    import oracle
+    q, k, v = _sp_inputs()
+    gh, gw = SP_GRID
+    ft = gh * gw
+    og = oracle.Geometry(gh, gw, SP_HEADS, SP_D, 24, 20, 20, 10000.0)
+    kc = np.zeros((SP_HEADS, 10 * ft, SP_D))
+    vc = np.zeros_like(kc)
+    for s in (3, 6, 9):
+        off = (s - 3) * ft
+        oracle.kv_append(kc, vc, 10, og, k[off:off + 3 * ft], v[off:off + 3 * ft], s, 3)
+    kpos, kvalid = oracle.cache_positions(10, 3, 11, gh, gw)
+    qpos = oracle.positions(3 * ft, gh, gw, 9)
+    qrot = oracle.rope3d(q, qpos, og)
+    m = oracle.mask_rows(qpos, kpos, kvalid, oracle.Mask(block_causal=True, chunk_frames=3))
+    o, _ = oracle.attention(qrot, kc.transpose(1, 0, 2), vc.transpose(1, 0, 2), m, SP_D ** -0.5)
+    return o
+
+
+def _sp_worker(rank, world, port, out):
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     sys.path.insert(0, root)
-    import numpy as np
     import oracle
-    import synth
     import video_diffusion_transformer_vdit_b200 as vdit
-    vdit.seq_pack = _oracle_pack  # the pack kernel needs a GPU; the exchange logic does not
+    # the pack / unpack kernels need a GPU; the exchange and the composition do not
+    vdit.seq_pack = _oracle_pack
+    vdit.seq_unpack = _oracle_unpack
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
                             world_size=world)
     try:
-        g = vdit.Geometry(3, 5, 4, 64, (24, 20, 20))
-        n_all = 2 * 15 + 6                       # a chunk of 36 tokens (2.4 frames of 3 x 5)
-        full = synth.bf16_bits_to_f64(synth.qkv_bf16(7, n_all, 4, 64, "q"))
-        n = n_all // world
-        x = torch.from_numpy(full[rank * n:(rank + 1) * n]).float()
-        got = vdit.seq_to_heads(x, g, 9, rotate=True)
-        # the oracle's whole-chunk RoPE, this rank's heads
-        og = oracle.Geometry(3, 5, 4, 64, 24, 20, 20, 10000.0)
-        ref = oracle.rope3d(full, oracle.positions(n_all, 3, 5, 9), og)[:, rank * 2:(rank + 1) * 2]
-        out[rank] = float(np.abs(got.double().numpy() - ref).max())
+        q, k, v = _sp_inputs()
+        gh, gw = SP_GRID
+        ft = gh * gw
+        g = vdit.Geometry(gh, gw, SP_HEADS, SP_D, (24, 20, 20))
+        n = 3 * ft // world
+        sl = slice(rank * n, (rank + 1) * n)
+        hg = SP_HEADS // world
+        hs = slice(rank * hg, (rank + 1) * hg)
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+        qf, kf, vf = vdit.seq_to_heads(t(q[sl]), t(k[6 * ft:][sl]), t(v[6 * ft:][sl]), g, 9)
+        # this rank's cache holds its heads: the history (frames 3..8) appended by the oracle,
+        # then the exchanged, already rotated chunk written into the ring as is
+        og = oracle.Geometry(gh, gw, hg, SP_D, 24, 20, 20, 10000.0)
+        kc = np.zeros((hg, 10 * ft, SP_D))
+        vc = np.zeros_like(kc)
+        for s in (3, 6):
+            off = (s - 3) * ft
+            oracle.kv_append(kc, vc, 10, og, k[off:off + 3 * ft][:, hs], v[off:off + 3 * ft][:, hs], s, 3)
+        for f in range(3):  # kv_write: frame 9 + f -> slot (9 + f) mod 10
+            slot = (9 + f) % 10
+            kc[:, slot * ft:(slot + 1) * ft] = kf.numpy()[f * ft:(f + 1) * ft].transpose(1, 0, 2)
+            vc[:, slot * ft:(slot + 1) * ft] = vf.numpy()[f * ft:(f + 1) * ft].transpose(1, 0, 2)
+        kpos, kvalid = oracle.cache_positions(10, 3, 11, gh, gw)
+        qpos = oracle.positions(3 * ft, gh, gw, 9)
+        m = oracle.mask_rows(qpos, kpos, kvalid, oracle.Mask(block_causal=True, chunk_frames=3))
+        o_full, _ = oracle.attention(qf.numpy(), kc.transpose(1, 0, 2), vc.transpose(1, 0, 2), m, SP_D ** -0.5)
+        o = vdit.heads_to_seq(t(o_full), g)
+        out[rank] = o.numpy().copy()
     finally:
         dist.destroy_process_group()
 
 
-def test_seq_to_heads_exchange_gloo_two_ranks():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_parallel_attention_composition_gloo(world):
+    # pack (RoPE at global positions) -> one batched exchange of Q, K, V -> ring write of the
+    # rotated K', V -> attention of this rank's heads -> return exchange -> unpack, on `world`
+    # gloo ranks; together the ranks' outputs equal the single-process attention of the chunk
     port = _free_port()
     with mp.Manager() as man:
         out = man.dict()
-        mp.spawn(_seq_worker, args=(world, port, out), nprocs=world, join=True)
+        mp.spawn(_sp_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
-    # float32 transport of float64 values: exact up to float32 rounding
-    assert res[0] < 1e-5 and res[1] < 1e-5
+    got = np.concatenate([res[r] for r in range(world)], axis=0)
+    ref = _sp_reference()
+    assert got.shape == ref.shape
+    assert np.abs(got - ref).max() < 1e-12
 
 
 # ----------------------------------------------------------------------------- K/V push

@@ -89,7 +89,10 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_export_masks.argtypes = [P, P, P]
         L.vdit_plan_split_for.argtypes = [P, I, ctypes.POINTER(I)]
         L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
-        L.vdit_seq_pack.argtypes = [P, P, P, I, ctypes.c_longlong, ctypes.c_longlong, I, I, P]
+        L.vdit_seq_pack.argtypes = [gp, P, P, P, P, P, P, P, I, I, I, LL, I, P]
+        L.vdit_seq_unpack.argtypes = [gp, P, P, P, I, I, LL, P]
+        L.vdit_kv_write.argtypes = [gp, P, P, I, P, P, I, I, P]
+        L.vdit_attn_forward_rotated.argtypes = [P, P, P, P, P, P, F, P]
         L.vdit_plan_destroy.argtypes = [P]
         L.vdit_plan_destroy.restype = None
         L.vdit_attn_forward.argtypes = [P, P, P, P, P, P, F, P]
@@ -224,39 +227,145 @@ def qkv_rope(x: torch.Tensor, w: torch.Tensor, g: Geometry, start_frame: int,
     return q
 
 
-def seq_pack(x: torch.Tensor, send: torch.Tensor, g: Geometry, start_frame: int, tok0: int,
-             n_ranks: int, rotate: bool = True, stream=None) -> torch.Tensor:
-    """x [n, heads, head_dim] (chunk-local tokens tok0 ..) -> send [n_ranks, n, heads / n_ranks,
-    head_dim], rotated at the global positions when rotate (vdit_seq_pack)."""
-    if x.dtype != torch.bfloat16 or x.dim() != 3 or x.shape[1:] != (g.heads, g.head_dim):
-        raise ValueError("x must be bf16 [n_tokens, heads, head_dim]")
-    if g.heads % n_ranks or tuple(send.shape) != (n_ranks, x.shape[0], g.heads // n_ranks, g.head_dim):
-        raise ValueError("send must be [n_ranks, n_tokens, heads / n_ranks, head_dim]")
+def kv_write(k_cache: torch.Tensor, v_cache: torch.Tensor, g: Geometry, capacity_frames: int,
+             k_rotated: torch.Tensor, v: torch.Tensor, start_frame: int, stream=None) -> None:
+    """Write already rotated K' and V into ring slots f mod capacity_frames (vdit_kv_write)."""
+    ft = g.frame_tokens
+    if k_rotated.shape != v.shape or k_rotated.shape[0] % ft or k_rotated.shape[1:] != (g.heads, g.head_dim):
+        raise ValueError("k, v must be [n_frames * frame_tokens, heads, head_dim]")
+    for t in (k_rotated, v, k_cache, v_cache):
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bf16")
     gc = g.c()
-    _check(lib().vdit_seq_pack(ctypes.byref(gc), _dev_ptr(x, "x"), _dev_ptr(send, "send"),
-                               int(start_frame), int(tok0), x.shape[0], int(n_ranks), int(bool(rotate)),
-                               _stream(stream)))
-    return send
+    _check(lib().vdit_kv_write(ctypes.byref(gc), _dev_ptr(k_cache, "k_cache"),
+                               _dev_ptr(v_cache, "v_cache"), int(capacity_frames),
+                               _dev_ptr(k_rotated, "k"), _dev_ptr(v, "v"), int(start_frame),
+                               k_rotated.shape[0] // ft, _stream(stream)))
 
 
-def seq_to_heads(x: torch.Tensor, g: Geometry, start_frame: int, group=None, rotate: bool = True,
-                 stream=None) -> torch.Tensor:
-    """Sequence-parallel to head-parallel exchange of one chunk: rank r of the group holds tokens
-    [r n, (r + 1) n) (x [n, heads, head_dim]); returns [world * n, heads / world, head_dim], all
-    tokens of this rank's heads, rotated at their global positions when rotate. One pack
-    (vdit_seq_pack) and one all-to-all of equal blocks (NCCL on GPUs)."""
+def seq_pack(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, start_frame: int,
+             rank: int, n_ranks: int, send: Optional[torch.Tensor], full, rotate: bool = True,
+             stream=None) -> None:
+    """vdit_seq_pack: this rank's q, k, v [n, heads, head_dim] (chunk-local tokens rank * n ..)
+    -> send [n_ranks, 3, n, heads / n_ranks, head_dim] (blocks for the other ranks) and the own
+    block into full = (q_full, k_full, v_full), each [n_ranks * n, heads / n_ranks, head_dim];
+    Q and K rotated at their global positions when rotate."""
+    n = q.shape[0]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.dim() != 3 or tuple(t.shape) != (n, g.heads, g.head_dim):
+            raise ValueError(f"{name} must be bf16 [n_tokens, heads, head_dim]")
+    if n_ranks < 1 or g.heads % n_ranks:
+        raise ValueError("n_ranks must divide heads")
+    hg = g.heads // n_ranks
+    for t in full:
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (n_ranks * n, hg, g.head_dim):
+            raise ValueError("full buffers must be bf16 [n_ranks * n_tokens, heads / n_ranks, head_dim]")
+    if n_ranks > 1 and (send is None or tuple(send.shape) != (n_ranks, 3, n, hg, g.head_dim)):
+        raise ValueError("send must be [n_ranks, 3, n_tokens, heads / n_ranks, head_dim]")
+    gc = g.c()
+    sp = _dev_ptr(send, "send") if send is not None else ctypes.c_void_p(0)
+    _check(lib().vdit_seq_pack(ctypes.byref(gc), _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                               sp, _dev_ptr(full[0], "q_full"), _dev_ptr(full[1], "k_full"),
+                               _dev_ptr(full[2], "v_full"), int(rank), int(n_ranks), int(start_frame),
+                               n, int(bool(rotate)), _stream(stream)))
+
+
+def seq_unpack(recv: Optional[torch.Tensor], own: torch.Tensor, out: torch.Tensor, g: Geometry,
+               rank: int, n_ranks: int, stream=None) -> torch.Tensor:
+    """vdit_seq_unpack: out [n, heads, head_dim] from recv [n_ranks, n, heads / n_ranks,
+    head_dim] (block r from rank r) and own [n, heads / n_ranks, head_dim] (block rank)."""
+    n = out.shape[0]
+    hg = g.heads // n_ranks
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (n, g.heads, g.head_dim):
+        raise ValueError("out must be bf16 [n_tokens, heads, head_dim]")
+    if tuple(own.shape) != (n, hg, g.head_dim):
+        raise ValueError("own must be [n_tokens, heads / n_ranks, head_dim]")
+    if n_ranks > 1 and (recv is None or tuple(recv.shape) != (n_ranks, n, hg, g.head_dim)):
+        raise ValueError("recv must be [n_ranks, n_tokens, heads / n_ranks, head_dim]")
+    gc = g.c()
+    rp = _dev_ptr(recv, "recv") if recv is not None else ctypes.c_void_p(0)
+    _check(lib().vdit_seq_unpack(ctypes.byref(gc), rp, _dev_ptr(own, "own"), _dev_ptr(out, "out"),
+                                 int(rank), int(n_ranks), n, _stream(stream)))
+    return out
+
+
+def _group_info(group):
     import torch.distributed as dist
-    on = dist.is_available() and dist.is_initialized()
-    world = dist.get_world_size(group) if on else 1
-    rank = dist.get_rank(group) if on else 0
-    n = x.shape[0]
-    send = torch.empty(world, n, g.heads // world, g.head_dim, dtype=x.dtype, device=x.device)
-    seq_pack(x, send, g, start_frame, rank * n, world, rotate, stream)
-    if world == 1:
-        return send[0]
-    recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
-    return recv.view(world * n, g.heads // world, g.head_dim)
+    if not (dist.is_available() and dist.is_initialized()):
+        return 1, 0
+    return dist.get_world_size(group), dist.get_rank(group)
+
+
+def exchange(sends: dict, recvs: dict, group=None) -> None:
+    """One batched point-to-point exchange: sends[r] (a list of tensors) go to group rank r, and
+    recvs[r] (a list of tensors, the same sizes in the same order as rank r's sends here) are
+    filled from group rank r, all posted together (batch_isend_irecv; one grouped NCCL launch on
+    GPUs). Backends without device-tensor point-to-point (gloo) stage device tensors through host
+    memory."""
+    import torch.distributed as dist
+    peers = sorted(set(sends) | set(recvs))
+    if not peers:
+        return
+    staged = dist.get_backend(group) != "nccl"
+
+    def host(t):
+        return t.detach().cpu() if (staged and t.is_cuda) else t
+
+    def glob(r):
+        return r if group is None else dist.get_global_rank(group, r)
+
+    ops, back = [], []
+    for r in peers:
+        for t in sends.get(r, ()):
+            ops.append(dist.P2POp(dist.isend, host(t).contiguous(), glob(r), group))
+        for t in recvs.get(r, ()):
+            buf = torch.empty(t.shape, dtype=t.dtype) if (staged and t.is_cuda) else t
+            ops.append(dist.P2POp(dist.irecv, buf, glob(r), group))
+            if buf is not t:
+                back.append((t, buf))
+    for req in dist.batch_isend_irecv(ops):
+        req.wait()
+    for t, buf in back:
+        t.copy_(buf)
+
+
+def seq_to_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, start_frame: int,
+                 group=None, rotate: bool = True, stream=None):
+    """Sequence-parallel to head-parallel exchange of one chunk ("Accelerating Video Generation
+    Inference with Sequential-Parallel 3D Positional Encoding Using a Global Time Index", sections
+    2.A-2.C): rank r of the group holds tokens [r n, (r + 1) n) of q, k, v [n, heads, head_dim];
+    returns (q_full, k_full, v_full), each [world * n, heads / world, head_dim]: all tokens of
+    this rank's heads, Q and K rotated at their global positions when rotate. One pack launch
+    (vdit_seq_pack) and one batched exchange of Q, K and V together."""
+    world, rank = _group_info(group)
+    n = q.shape[0]
+    hg = g.heads // world
+    full = tuple(torch.empty(world * n, hg, g.head_dim, dtype=q.dtype, device=q.device) for _ in range(3))
+    send = torch.empty(world, 3, n, hg, g.head_dim, dtype=q.dtype, device=q.device) if world > 1 else None
+    seq_pack(q, k, v, g, start_frame, rank, world, send, full, rotate, stream)
+    if world > 1:
+        exchange({r: [send[r, x] for x in range(3)] for r in range(world) if r != rank},
+                 {r: [full[x][r * n:(r + 1) * n] for x in range(3)] for r in range(world) if r != rank},
+                 group)
+    return full
+
+
+def heads_to_seq(o_full: torch.Tensor, g: Geometry, group=None, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Return exchange after attention: o_full [world * n, heads / world, head_dim] (this rank's
+    heads, all tokens) -> out [n, heads, head_dim] (this rank's tokens, all heads): one batched
+    exchange and one unpack launch (vdit_seq_unpack)."""
+    world, rank = _group_info(group)
+    n = o_full.shape[0] // world
+    hg = g.heads // world
+    if out is None:
+        out = torch.empty(n, g.heads, g.head_dim, dtype=o_full.dtype, device=o_full.device)
+    recv = None
+    if world > 1:
+        recv = torch.empty(world, n, hg, g.head_dim, dtype=o_full.dtype, device=o_full.device)
+        exchange({r: [o_full[r * n:(r + 1) * n]] for r in range(world) if r != rank},
+                 {r: [recv[r]] for r in range(world) if r != rank}, group)
+    return seq_unpack(recv, o_full[rank * n:(rank + 1) * n], out, g, rank, world, stream)
 
 
 class KVCache:
@@ -291,23 +400,40 @@ class KVCache:
         kv_append(self.k, self.v, self.g, self.capacity_frames, k, v, start_frame, stream)
         self._note(start_frame, k.shape[0] // self.g.frame_tokens)
 
+    def write(self, k_rotated: torch.Tensor, v: torch.Tensor, start_frame: int, stream=None) -> None:
+        """Write an already rotated chunk (K' and V) into the ring (vdit_kv_write)."""
+        self._check_next(start_frame)
+        kv_write(self.k, self.v, self.g, self.capacity_frames, k_rotated, v, start_frame, stream)
+        self._note(start_frame, k_rotated.shape[0] // self.g.frame_tokens)
+
     def push(self, k: torch.Tensor, v: torch.Tensor, dst: int, group=None) -> list:
-        """Wave Parallelism's K/V forward push (Wave Forcing / WaveRT): send a chunk's K and V (as
-        given to append, before RoPE) one way to rank dst, which appends them to its own cache
-        with receive(). The sends are asynchronous (isend; NCCL on GPUs), so they overlap the
-        attention that follows; returns the work handles to wait on before k, v are reused."""
+        """Wave Parallelism's K/V forward push (Wave Forcing / WaveRT): send a chunk's K and V as
+        given to append (before RoPE: one contiguous message each; the receiver's append rotates
+        K at the same global frames in the same pass that places it in its ring, so sending K'
+        would save no work) one way to rank dst, which appends them to its own cache with
+        receive(). The sends are asynchronous (isend; NCCL on GPUs), so they overlap the attention
+        that follows; returns the work handles to wait on before k, v are reused. Backends
+        without device-tensor point-to-point (gloo) stage through host memory."""
         import torch.distributed as dist
-        return [dist.isend(k.contiguous(), dst, group=group), dist.isend(v.contiguous(), dst, group=group)]
+        glob = dst if group is None else dist.get_global_rank(group, dst)
+        staged = dist.get_backend(group) != "nccl"
+        bufs = [t.detach().cpu() if (staged and t.is_cuda) else t.contiguous() for t in (k, v)]
+        return [dist.isend(b, glob, group=group) for b in bufs]
 
     def receive(self, start_frame: int, n_frames: int, src: int, group=None, stream=None) -> None:
         """Receive a chunk pushed by rank src and append it here (RoPE at its global frames, ring
         write), as the sender appended it to its own cache."""
         import torch.distributed as dist
+        glob = src if group is None else dist.get_global_rank(group, src)
+        staged = dist.get_backend(group) != "nccl"
         shape = (n_frames * self.g.frame_tokens, self.g.heads, self.g.head_dim)
-        k = torch.empty(shape, dtype=self.k.dtype, device=self.k.device)
+        dev = torch.device("cpu") if staged else self.k.device
+        k = torch.empty(shape, dtype=self.k.dtype, device=dev)
         v = torch.empty_like(k)
-        dist.recv(k, src, group=group)
-        dist.recv(v, src, group=group)
+        dist.recv(k, glob, group=group)
+        dist.recv(v, glob, group=group)
+        if staged and self.k.is_cuda:
+            k, v = k.to(self.k.device), v.to(self.k.device)
         self.append(k, v, start_frame, stream)
 
     def project_append(self, x: torch.Tensor, w: torch.Tensor, start_frame: int,
@@ -393,8 +519,9 @@ class Plan:
 def attn_forward(plan: Plan, q: torch.Tensor, cache: Optional[KVCache] = None,
                  k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                 scale: Optional[float] = None, stream=None) -> torch.Tensor:
-    """o = masked softmax(RoPE(q) . K'^T * scale) V over the plan; q is unrotated."""
+                 scale: Optional[float] = None, stream=None, q_rotated: bool = False) -> torch.Tensor:
+    """o = masked softmax(RoPE(q) . K'^T * scale) V over the plan; q is unrotated (RoPE fused into
+    the Q load, vdit_attn_forward) unless q_rotated (vdit_attn_forward_rotated)."""
     if cache is not None:
         k_cache, v_cache = cache.k, cache.v
     g = plan.g
@@ -410,9 +537,9 @@ def attn_forward(plan: Plan, q: torch.Tensor, cache: Optional[KVCache] = None,
         if lse.dtype != torch.float32 or lse.shape != (g.heads, q.shape[0]) or not lse.is_contiguous():
             raise ValueError("lse must be fp32 [heads, q_tokens]")
         lse_ptr = ctypes.c_void_p(lse.data_ptr())
-    _check(lib().vdit_attn_forward(plan._h, _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
-                                   _dev_ptr(v_cache, "v_cache"), _dev_ptr(o, "out"), lse_ptr,
-                                   float(scale), _stream(stream)))
+    fn = lib().vdit_attn_forward_rotated if q_rotated else lib().vdit_attn_forward
+    _check(fn(plan._h, _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+              _dev_ptr(o, "out"), lse_ptr, float(scale), _stream(stream)))
     return o
 
 

@@ -135,6 +135,7 @@ struct AttnArgs {
     const float2* th;
     const float2* tw;
     int* status;
+    int q_rotated;         // q already rotated at the plan's query positions: plain load
     int skip_loads;        // test hook: the producer issues nothing, so every wait runs out
     int bt2, bh2, bw2;
     int q_tokens, kv_tokens, heads;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = qi / ft, rm = qi - f * ft;
             const int hh = rm / a.grid_w, ww = rm - hh * a.grid_w;
             const uint4 x = __ldg(a.q + ((size_t)qi * a.heads + head) * kC16 + c16);
-            v = rope_chunk(x, c16 * 4, a.q_start + f, hh, ww, a);
+            v = a.q_rotated ? x : rope_chunk(x, c16 * 4, a.q_start + f, hh, ww, a);
         }
         *reinterpret_cast<uint4*>(smem + L::OFF_Q + h * kTileBytes + sw128_offset(r, c16)) = v;
     }
@@ -876,7 +877,7 @@ int device_state(int dev, const DeviceState** out) {
 // split scratch (unused without a split).
 int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
                      void* o, float* lse, float scale, float* ws_o, float* ws_lse,
-                     const vdit::RopeTables& tabs, cudaStream_t st, int dev) {
+                     const vdit::RopeTables& tabs, cudaStream_t st, int dev, bool q_rotated = false) {
     using vdit::fail;
     CUtensorMap mk, mv;
     const int d = p->g.head_dim;
@@ -903,6 +904,7 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     a.th = static_cast<const float2*>(tabs.h);
     a.tw = static_cast<const float2*>(tabs.w);
     a.status = ds->status;
+    a.q_rotated = q_rotated ? 1 : 0;
     a.skip_loads = g_skip_loads.load(std::memory_order_relaxed);
     a.bt2 = p->g.band_t / 2;
     a.bh2 = p->g.band_h / 2;
@@ -943,9 +945,9 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
 
 }  // namespace
 
-extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache,
-                                 const void* v_cache, void* o, float* lse, float scale,
-                                 void* stream) {
+namespace {
+int attn_forward_impl(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache, void* o,
+                      float* lse, float scale, void* stream, bool q_rotated) {
     using vdit::fail;
     if (!p) return fail(VDIT_ERR_INVALID_ARG, "NULL plan");
     if (!p->d_buf) return fail(VDIT_ERR_NOT_UPLOADED, "plan not uploaded (vdit_plan_upload)");
@@ -960,7 +962,20 @@ extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* 
     vdit::RopeTables tabs;
     if (int rc = vdit::get_rope_tables(&p->g, &tabs)) return rc;
     return launch_attention(p, q, k_cache, v_cache, o, lse, scale, p->d_ws_o, p->d_ws_lse, tabs,
-                            static_cast<cudaStream_t>(stream), dev);
+                            static_cast<cudaStream_t>(stream), dev, q_rotated);
+}
+}  // namespace
+
+extern "C" int vdit_attn_forward(const vdit_plan* p, const void* q, const void* k_cache,
+                                 const void* v_cache, void* o, float* lse, float scale,
+                                 void* stream) {
+    return attn_forward_impl(p, q, k_cache, v_cache, o, lse, scale, stream, false);
+}
+
+extern "C" int vdit_attn_forward_rotated(const vdit_plan* p, const void* q_rotated, const void* k_cache,
+                                         const void* v_cache, void* o, float* lse, float scale,
+                                         void* stream) {
+    return attn_forward_impl(p, q_rotated, k_cache, v_cache, o, lse, scale, stream, true);
 }
 
 extern "C" void vdit_debug_skip_loads(int on) { g_skip_loads.store(on ? 1 : 0); }

@@ -190,8 +190,9 @@ template <bool APPEND>
 constexpr int blocks_per_sm() { return APPEND ? 2 : 4; }
 
 // APPEND = false: y = RoPE(x) at t = start_frame + local frame.
-// APPEND = true:  K' = RoPE(k) and V (unchanged) go to frame slot t mod capacity of the caches.
-template <bool APPEND>
+// APPEND = true:  K' = RoPE(k) (ROTATE) or K' = k (already rotated, !ROTATE) and V (unchanged) go
+//                 to frame slot t mod capacity of the caches.
+template <bool APPEND, bool ROTATE = true>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, blocks_per_sm<APPEND>())
     rope_stream_kernel(StreamArgs a) {
     const int lane = threadIdx.x & 31;
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, blocks_per_sm<APPEND>())
         const int w = rem - h * a.grid_w;
         const int t = a.start_frame + (int)f;
         float2 cs[4];
-        chunk_angles(cs, c8 * 4, t, h, w, a);
+        if (ROTATE) chunk_angles(cs, c8 * 4, t, h, w, a);
         const size_t src0 = (size_t)tok * a.cpt;
         size_t dst_tok = 0;  // append: chunk index of (head 0, chunk 0) of this token's cache row
         if (APPEND) {
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, blocks_per_sm<APPEND>())
             for (int u = 0; u < kBatch; ++u) {
                 const int j = j0 + 32 * u + lane;
                 if (j < a.cpt) {
-                    const uint4 r = rotate_chunk(xin[u], cs);
+                    const uint4 r = ROTATE ? rotate_chunk(xin[u], cs) : xin[u];
                     if (APPEND) {
                         const int head = j >> a.cpr_log2;
                         const size_t d = dst_tok + (((size_t)head * a.cap_tok) << a.cpr_log2) + c8;
@@ -241,31 +242,53 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, blocks_per_sm<APPEND>())
     }
 }
 
-int launch_stream(bool append, StreamArgs& a, cudaStream_t s) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+// SM count of the current device, looked up once per device.
+int sm_count() {
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+    cache[dev] = sms;
+    return sms;
+}
+
+// append: 0 = RoPE only, 1 = RoPE + ring write, 2 = ring write of already rotated K
+int launch_stream(int append, StreamArgs& a, cudaStream_t s) {
     const long long want = ((long long)a.n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
     const int per_sm = append ? blocks_per_sm<true>() : blocks_per_sm<false>();
-    const int blocks = (int)std::min<long long>(want, (long long)sms * per_sm);
+    const int blocks = (int)std::min<long long>(want, (long long)sm_count() * per_sm);
     if (blocks == 0) return VDIT_OK;
-    if (append)
-        rope_stream_kernel<true><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
+    if (append == 1)
+        rope_stream_kernel<true, true><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
+    else if (append == 2)
+        rope_stream_kernel<true, false><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
     else
-        rope_stream_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
+        rope_stream_kernel<false, true><<<blocks, kWarpsPerBlock * 32, 0, s>>>(a);
     return vdit::cuda_check(cudaGetLastError(), "rope kernel launch");
 }
 
 // Sequence-to-head pack of the Ulysses-style exchange ("Accelerating Video Generation Inference
 // with Sequential-Parallel 3D Positional Encoding Using a Global Time Index", sections 2.A-2.C: the
-// sequence is split over the ranks; QKV, the causal RoPE and one fused all-to-all that gathers the
-// sequence and splits the heads). This rank's tokens x [n_tok, heads, D] (chunk-local tokens
-// tok0 .. tok0 + n_tok - 1) go to send [ranks][n_tok][heads / ranks][D]: block r holds the heads
-// rank r receives, so an all-to-all of equal blocks leaves every rank [ranks * n_tok, heads /
-// ranks, D] in sequence order. With ROTATE the rows are rotated at their global positions (the
-// time index needs only start_frame and tok0: no rank asks another for its positions).
+// sequence is split over the ranks; the causal RoPE at global positions, then one fused all-to-all
+// that gathers the sequence and splits the heads for Q, K and V together). Rank `rank` holds the
+// chunk-local tokens rank * n_tok .. (rank + 1) * n_tok - 1 of q, k, v [n_tok, heads, D]. Block r of
+// the send buffer, send [ranks][3][n_tok][heads / ranks][D], holds the heads rank r owns, Q then K
+// then V; the rank's own block goes straight to rows rank * n_tok .. of its head-sharded buffers
+// q_full, k_full, v_full [ranks * n_tok][heads / ranks][D], where the exchange leaves every other
+// rank's block too. With ROTATE, Q and K are rotated at their global positions (the time index
+// needs only start_frame and the shard's first token: no rank asks another for its positions);
+// V is copied. One warp streams one (token, tensor) row.
 struct PackArgs {
-    StreamArgs s;       // x, y (= send), tables, geometry, n_tokens, cpt, cpr_log2
+    StreamArgs s;       // tables, geometry, n_tokens (= n_tok), cpt, cpr_log2, start_frame
+    const uint4* src[3];
+    uint4* send;
+    uint4* full[3];
+    int rank;
     int tok0;
     int heads_per_rank;
     FastDiv by_hpr;
@@ -278,22 +301,25 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) rope_pack_kernel(PackA
     const int n_warps = gridDim.x * kWarpsPerBlock;
     const int c8 = lane & ((1 << a.cpr_log2) - 1);
     const int ft = a.grid_h * a.grid_w;
-    for (int n = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); n < a.n_tokens; n += n_warps) {
+    const int items = 3 * a.n_tokens;
+    for (int it = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); it < items; it += n_warps) {
+        const int x = it / a.n_tokens, n = it - x * a.n_tokens;
+        const bool rot = ROTATE && x < 2;
         float2 cs[4];
-        if (ROTATE) {
+        if (rot) {
             const int tok = pa.tok0 + n;
             const uint32_t f = fdiv((uint32_t)tok, a.by_ft);
             const int rem = tok - (int)f * ft;
             const int h = (int)fdiv((uint32_t)rem, a.by_w);
             chunk_angles(cs, c8 * 4, a.start_frame + (int)f, h, rem - h * a.grid_w, a);
         }
-        const size_t src0 = (size_t)n * a.cpt;
+        const uint4* src = pa.src[x] + (size_t)n * a.cpt;
         for (int j0 = 0; j0 < a.cpt; j0 += 32 * kBatch) {
             uint4 xin[kBatch];
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 const int j = j0 + 32 * u + lane;
-                if (j < a.cpt) xin[u] = __ldcs(a.x + src0 + j);
+                if (j < a.cpt) xin[u] = __ldcs(src + j);
             }
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
@@ -301,9 +327,54 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) rope_pack_kernel(PackA
                 if (j < a.cpt) {
                     const int head = j >> a.cpr_log2;
                     const int r = (int)fdiv((uint32_t)head, pa.by_hpr), hh = head - r * pa.heads_per_rank;
-                    const size_t row = ((size_t)r * a.n_tokens + n) * pa.heads_per_rank + hh;
-                    __stcs(a.y + (row << a.cpr_log2) + c8, ROTATE ? rotate_chunk(xin[u], cs) : xin[u]);
+                    uint4* dst = r == pa.rank
+                                     ? pa.full[x] + ((((size_t)pa.rank * a.n_tokens + n) * pa.heads_per_rank + hh)
+                                                     << a.cpr_log2)
+                                     : pa.send + (((((size_t)r * 3 + x) * a.n_tokens + n) * pa.heads_per_rank + hh)
+                                                  << a.cpr_log2);
+                    __stcs(dst + c8, rot ? rotate_chunk(xin[u], cs) : xin[u]);
                 }
+            }
+        }
+    }
+}
+
+// Head-to-sequence unpack after attention (the return all-to-all of the same exchange): this
+// rank's tokens of out [n_tok, heads, D] gather head block r from recv[r] = [n_tok][heads /
+// ranks][D] (sent by rank r, which computed those heads), block `rank` from `own` (this rank's
+// own attention output rows for its tokens). A copy: bit-exact.
+struct UnpackArgs {
+    const uint4* recv;
+    const uint4* own;
+    uint4* out;
+    int n_tokens, cpt, cpr_log2, rank, heads_per_rank;
+    FastDiv by_hpr;
+};
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) seq_unpack_kernel(UnpackArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int n_warps = gridDim.x * kWarpsPerBlock;
+    const int c8 = lane & ((1 << a.cpr_log2) - 1);
+    for (int n = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); n < a.n_tokens; n += n_warps) {
+        for (int j0 = 0; j0 < a.cpt; j0 += 32 * kBatch) {
+            uint4 xin[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) {
+                    const int head = j >> a.cpr_log2;
+                    const int r = (int)fdiv((uint32_t)head, a.by_hpr), hh = head - r * a.heads_per_rank;
+                    const uint4* src = r == a.rank
+                                           ? a.own + ((((size_t)n) * a.heads_per_rank + hh) << a.cpr_log2)
+                                           : a.recv + ((((size_t)r * a.n_tokens + n) * a.heads_per_rank + hh)
+                                                       << a.cpr_log2);
+                    xin[u] = __ldcs(src + c8);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) __stcs(a.out + (size_t)n * a.cpt + j, xin[u]);
             }
         }
     }
@@ -357,12 +428,12 @@ extern "C" int vdit_rope3d_apply(const vdit_geom* g, const void* x, void* y, int
     a.y = static_cast<uint4*>(y);
     a.n_tokens = (int)n_tokens;
     a.start_frame = start_frame;
-    return launch_stream(false, a, static_cast<cudaStream_t>(stream));
+    return launch_stream(0, a, static_cast<cudaStream_t>(stream));
 }
 
-extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
-                              int capacity_frames, const void* k, const void* v, int start_frame,
-                              int n_frames, void* stream) {
+namespace {
+int kv_ring_write(const vdit_geom* g, void* k_cache, void* v_cache, int capacity_frames, const void* k,
+                  const void* v, int start_frame, int n_frames, bool rotate, void* stream) {
     using vdit::fail;
     if (int rc = vdit::check_geom(g)) return rc;
     if (!k_cache || !v_cache || !k || !v) return fail(VDIT_ERR_INVALID_ARG, "NULL pointer");
@@ -397,47 +468,123 @@ extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
     a.cap_frames = capacity_frames;
     a.cap_tok = ft * capacity_frames;
     a.by_cap = make_fastdiv((uint32_t)capacity_frames);
-    return launch_stream(true, a, static_cast<cudaStream_t>(stream));
+    return launch_stream(rotate ? 1 : 2, a, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+extern "C" int vdit_kv_append(const vdit_geom* g, void* k_cache, void* v_cache,
+                              int capacity_frames, const void* k, const void* v, int start_frame,
+                              int n_frames, void* stream) {
+    return kv_ring_write(g, k_cache, v_cache, capacity_frames, k, v, start_frame, n_frames, true, stream);
 }
 
-extern "C" int vdit_seq_pack(const vdit_geom* g, const void* x, void* send, int start_frame,
-                             long long tok0, long long n_tokens, int n_ranks, int rotate, void* stream) {
+extern "C" int vdit_kv_write(const vdit_geom* g, void* k_cache, void* v_cache, int capacity_frames,
+                             const void* k_rotated, const void* v, int start_frame, int n_frames,
+                             void* stream) {
+    return kv_ring_write(g, k_cache, v_cache, capacity_frames, k_rotated, v, start_frame, n_frames, false,
+                         stream);
+}
+
+extern "C" int vdit_seq_pack(const vdit_geom* g, const void* q, const void* k, const void* v, void* send,
+                             void* q_full, void* k_full, void* v_full, int rank, int n_ranks, int start_frame,
+                             long long n_tokens, int rotate, void* stream) {
     using vdit::fail;
     if (int rc = vdit::check_geom(g)) return rc;
-    if (n_tokens < 0 || tok0 < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens and tok0 must be >= 0");
+    if (n_tokens < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens must be >= 0");
+    if (n_ranks < 1 || g->heads % n_ranks != 0) return fail(VDIT_ERR_INVALID_ARG, "n_ranks must divide heads");
+    if (rank < 0 || rank >= n_ranks) return fail(VDIT_ERR_INVALID_ARG, "rank outside [0, n_ranks)");
     if (n_tokens == 0) return VDIT_OK;
-    if (!x || !send) return fail(VDIT_ERR_INVALID_ARG, "x or send is NULL");
-    if (!aligned16(x) || !aligned16(send)) return fail(VDIT_ERR_MISALIGNED, "x/send not 16-byte aligned");
-    if (n_ranks < 1 || g->heads % n_ranks != 0)
-        return fail(VDIT_ERR_INVALID_ARG, "n_ranks must divide heads");
+    if (!q || !k || !v || !q_full || !k_full || !v_full || (n_ranks > 1 && !send))
+        return fail(VDIT_ERR_INVALID_ARG, "NULL pointer");
+    const void* ptrs[7] = {q, k, v, send, q_full, k_full, v_full};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(VDIT_ERR_MISALIGNED, "tensor not 16-byte aligned");
     const long long ft = (long long)g->grid_h * g->grid_w;
-    const long long last = tok0 + n_tokens - 1;
+    const long long tok0 = (long long)rank * n_tokens, last = tok0 + n_tokens - 1;
     if (start_frame < 0 || start_frame + last / ft > VDIT_MAX_FRAME)
         return fail(VDIT_ERR_INVALID_ARG, "frames outside [0, VDIT_MAX_FRAME]");
-    const long long bytes = n_tokens * g->heads * g->head_dim * 2;
-    const char* xb = static_cast<const char*>(x);
-    const char* yb = static_cast<const char*>(send);
-    if (xb < yb + bytes && yb < xb + bytes) return fail(VDIT_ERR_INVALID_ARG, "x and send overlap");
-    if ((unsigned long long)n_tokens * g->heads * (g->head_dim / 8) >= (1ull << 31) || last >= (1ll << 31))
-        return fail(VDIT_ERR_UNSUPPORTED, "shard larger than 2^31 16-byte chunks");
+    if ((unsigned long long)n_tokens * n_ranks * g->heads * (g->head_dim / 8) >= (1ull << 31) ||
+        (long long)n_tokens * n_ranks >= (1ll << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "exchange larger than 2^31 16-byte chunks");
+    // inputs (3 x n_tokens rows) against outputs (send: 3 x n_ranks x n_tokens rows; each full
+    // buffer: n_ranks x n_tokens rows of heads / n_ranks heads) must not overlap
+    const long long in_bytes = n_tokens * g->heads * g->head_dim * 2;
+    const long long full_bytes = in_bytes;  // n_ranks * n_tokens * (heads / n_ranks) * D * 2
+    const long long send_bytes = 3 * in_bytes;
+    const void* outs[4] = {send, q_full, k_full, v_full};
+    const long long out_n[4] = {n_ranks > 1 ? send_bytes : 0, full_bytes, full_bytes, full_bytes};
+    auto overlap = [](const void* a, long long na, const void* b, long long nb) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        return na > 0 && nb > 0 && x < y + nb && y < x + na;
+    };
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 3; ++j)
+            if (overlap(outs[i], out_n[i], ptrs[j], in_bytes))
+                return fail(VDIT_ERR_INVALID_ARG, "an output overlaps an input");
+        for (int j = i + 1; j < 4; ++j)
+            if (overlap(outs[i], out_n[i], outs[j], out_n[j]))
+                return fail(VDIT_ERR_INVALID_ARG, "outputs overlap each other");
+    }
     PackArgs pa{};
     if (int rc = fill_common(g, pa.s)) return rc;
-    pa.s.x = static_cast<const uint4*>(x);
-    pa.s.y = static_cast<uint4*>(send);
     pa.s.n_tokens = (int)n_tokens;
     pa.s.start_frame = start_frame;
+    pa.src[0] = static_cast<const uint4*>(q);
+    pa.src[1] = static_cast<const uint4*>(k);
+    pa.src[2] = static_cast<const uint4*>(v);
+    pa.send = static_cast<uint4*>(send);
+    pa.full[0] = static_cast<uint4*>(q_full);
+    pa.full[1] = static_cast<uint4*>(k_full);
+    pa.full[2] = static_cast<uint4*>(v_full);
+    pa.rank = rank;
     pa.tok0 = (int)tok0;
     pa.heads_per_rank = g->heads / n_ranks;
     pa.by_hpr = make_fastdiv((uint32_t)pa.heads_per_rank);
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long want = (n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    const int blocks = (int)std::min<long long>(want, (long long)sms * 4);
+    const long long want = (3 * n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int blocks = (int)std::min<long long>(want, (long long)sm_count() * 4);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (rotate)
         rope_pack_kernel<true><<<blocks, kWarpsPerBlock * 32, 0, st>>>(pa);
     else
         rope_pack_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, st>>>(pa);
     return vdit::cuda_check(cudaGetLastError(), "pack kernel launch");
+}
+
+extern "C" int vdit_seq_unpack(const vdit_geom* g, const void* recv, const void* own, void* out, int rank,
+                               int n_ranks, long long n_tokens, void* stream) {
+    using vdit::fail;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (n_tokens < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens must be >= 0");
+    if (n_ranks < 1 || g->heads % n_ranks != 0) return fail(VDIT_ERR_INVALID_ARG, "n_ranks must divide heads");
+    if (rank < 0 || rank >= n_ranks) return fail(VDIT_ERR_INVALID_ARG, "rank outside [0, n_ranks)");
+    if (n_tokens == 0) return VDIT_OK;
+    if (!own || !out || (n_ranks > 1 && !recv)) return fail(VDIT_ERR_INVALID_ARG, "NULL pointer");
+    if ((recv && !aligned16(recv)) || !aligned16(own) || !aligned16(out))
+        return fail(VDIT_ERR_MISALIGNED, "tensor not 16-byte aligned");
+    const long long out_bytes = n_tokens * g->heads * g->head_dim * 2;
+    const long long own_bytes = out_bytes / n_ranks, recv_bytes = n_ranks > 1 ? out_bytes : 0;
+    auto overlap = [](const void* a, long long na, const void* b, long long nb) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        return na > 0 && nb > 0 && x < y + nb && y < x + na;
+    };
+    if (overlap(out, out_bytes, own, own_bytes) || overlap(out, out_bytes, recv, recv_bytes))
+        return fail(VDIT_ERR_INVALID_ARG, "out overlaps an input");
+    if ((unsigned long long)n_tokens * g->heads * (g->head_dim / 8) >= (1ull << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "shard larger than 2^31 16-byte chunks");
+    UnpackArgs a{};
+    a.recv = static_cast<const uint4*>(recv);
+    a.own = static_cast<const uint4*>(own);
+    a.out = static_cast<uint4*>(out);
+    a.n_tokens = (int)n_tokens;
+    a.cpr_log2 = g->head_dim == 128 ? 4 : 3;
+    a.cpt = g->heads * (g->head_dim / 8);
+    a.rank = rank;
+    a.heads_per_rank = g->heads / n_ranks;
+    a.by_hpr = make_fastdiv((uint32_t)a.heads_per_rank);
+    const long long want = (n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int blocks = (int)std::min<long long>(want, (long long)sm_count() * 4);
+    seq_unpack_kernel<<<blocks, kWarpsPerBlock * 32, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return vdit::cuda_check(cudaGetLastError(), "unpack kernel launch");
 }
