@@ -118,8 +118,9 @@ typedef struct vdit_plan_info_t {
     int uploaded;        /* 1 after vdit_plan_upload */
     int kv_splits;       /* key-range pieces per (query block, head), set by vdit_plan_upload */
     long long workspace_bytes; /* device scratch the plan holds for kv_splits > 1 */
-    long long mask_bytes;      /* keep masks of the partial tiles: 2 KiB per listed tile that
-                                  is not full (see vdit_plan_export_masks) */
+    long long mask_bytes;      /* keep masks of the partial tiles: 2 KiB per distinct block
+                                  (identical blocks of several tiles are stored once; see
+                                  vdit_plan_export_masks) */
 } vdit_plan_info_t;
 
 /* 3-D RoPE ([CRoPE] 2.B, [TR] Metodologia 1) of n_tokens consecutive tokens of one chunk whose
@@ -183,7 +184,8 @@ VDIT_API int vdit_plan_export(const vdit_plan* p, int* row_ptr, int* col_idx, un
 
 /* Host copy of the per-row keep masks the kernel applies to partial tiles (listed, not full),
  * computed on the host from the mask predicate above. For schedule entry i (the col_idx order of
- * vdit_plan_export), mask_index[i] is its block number, or -1 for a full tile. Block b is
+ * vdit_plan_export), mask_index[i] is its block number, or -1 for a full tile; entries whose
+ * masks are identical share one block. Block b is
  * words[512 b .. 512 b + 511]: for row r (query q_tile * 128 + r) and key kt * 128 + k, the pair
  * is kept iff bit (k mod 32) of words[512 b + 4 r + k / 32] is set. Rows and keys past the token
  * counts are 0. mask_index: [tiles]; words: [mask_bytes / 4] (may be NULL when mask_bytes is 0). */

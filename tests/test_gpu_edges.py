@@ -87,8 +87,11 @@ def test_empty_calls_are_no_ops():
     x = torch.empty(0, 2, 64, dtype=torch.bfloat16, device="cuda")
     y = vdit.rope3d_apply(x, g, 0)
     assert y.shape == (0, 2, 64)
-    send = torch.empty(2, 0, 1, 64, dtype=torch.bfloat16, device="cuda")
-    vdit.seq_pack(x, send, g, 0, 0, 2)
+    send = torch.empty(2, 3, 0, 1, 64, dtype=torch.bfloat16, device="cuda")
+    full = tuple(torch.empty(0, 1, 64, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    vdit.seq_pack(x, x, x, g, 0, 1, 2, send, full)
+    out = torch.empty(0, 2, 64, dtype=torch.bfloat16, device="cuda")
+    vdit.seq_unpack(torch.empty(2, 0, 1, 64, dtype=torch.bfloat16, device="cuda"), full[0], out, g, 1, 2)
     torch.cuda.synchronize()
     assert vdit.get_status() == vdit.OK
 

@@ -229,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // work unit: q-block (longest lists first), head, and the piece `sp` of its key tiles
-    const int sp = blockIdx.x / a.n_qb, head = blockIdx.y;
-    const int qb = __ldg(a.unit_order + (blockIdx.x - sp * a.n_qb));
+    const int unit = blockIdx.x, head = blockIdx.y;
+    const int sp = unit / a.n_qb;
+    const int qb = __ldg(a.unit_order + (unit - sp * a.n_qb));
     const int u_first = __ldg(a.u_row_ptr + qb);
     const int n_all = __ldg(a.u_row_ptr + qb + 1) - u_first;
     const int e0 = (int)((long long)n_all * sp / a.n_split);
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every CTA walks its key tiles starting at a different position (the online softmax does
     // not depend on the order): CTAs of one head run concurrently, and starting them all at the
     // same tile makes them request the same 32 KiB of K / V from the same L2 slices at once.
-    const int rot = n_ent > 0 ? (int)(((unsigned)blockIdx.x * 97u + (unsigned)blockIdx.y * 31u) % (unsigned)n_ent) : 0;
+    const int rot = n_ent > 0 ? (int)(((unsigned)unit * 97u + (unsigned)head * 31u) % (unsigned)n_ent) : 0;
     auto entry = [&](int i) { const int e = i + rot; return e >= n_ent ? e - n_ent : e; };
     // visits of the entries: the dynamic-threshold mode walks the list twice
     const int n_v = DYN ? 2 * n_ent : n_ent;
@@ -918,7 +919,7 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
     a.tau_log2 = (float)(p->m.tau * 1.4426950408889634);
     const bool dyn = p->m.kind & VDIT_MASK_DYNAMIC;
-    dim3 grid(p->n_qb * p->n_split, p->g.heads);
+    const dim3 grid((unsigned)(p->n_qb * p->n_split), (unsigned)p->g.heads);
     if (d == 128 && !dyn)
         attn_fwd_kernel<128, false><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
     else if (d == 64 && !dyn)

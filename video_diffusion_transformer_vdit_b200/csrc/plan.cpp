@@ -14,6 +14,8 @@
 #include <cstring>
 #include <functional>
 #include <new>
+#include <unordered_map>
+#include <vector>
 
 #include <cuda_runtime.h>
 
@@ -200,6 +202,7 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
         segments(kt * VDIT_TILE, std::min(p->kv_tokens, (kt + 1) * VDIT_TILE), g->grid_h,
                  g->grid_w, [&](int slot) { return p->slot_frame[slot]; }, kseg[kt]);
     std::vector<Seg> qs;
+    std::unordered_map<uint64_t, std::vector<int>> seen;  // mask block hash -> block numbers
     p->row_ptr.assign(p->n_qt + 1, 0);
     p->kept_pairs = 0;
     p->n_full = 0;
@@ -234,8 +237,27 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
                 p->col_idx.push_back(kt);
                 p->full.push_back(all ? 1 : 0);
                 p->n_full += all;
-                p->mask_of.push_back(all ? -1 : (int)(p->masks.size() / 512));
-                if (!all) tile_mask(*p, q0, q1, kseg[kt], p->masks);
+                int block = -1;
+                if (!all) {
+                    // keep-mask block of this tile; identical blocks (tiles at the same offsets
+                    // within their frames with the same radii) are stored once, so the blocks the
+                    // kernel reads for all heads stay resident in L2
+                    const size_t at = p->masks.size();
+                    tile_mask(*p, q0, q1, kseg[kt], p->masks);
+                    uint64_t hsh = 1469598103934665603ull;  // FNV-1a over the 512 words
+                    for (size_t wi = at; wi < at + 512; ++wi) hsh = (hsh ^ p->masks[wi]) * 1099511628211ull;
+                    block = (int)(at / 512);
+                    auto& same = seen[hsh];
+                    for (int b : same)
+                        if (std::equal(p->masks.begin() + at, p->masks.begin() + at + 512,
+                                       p->masks.begin() + (size_t)b * 512)) {
+                            block = b;
+                            break;
+                        }
+                    if (block != (int)(at / 512)) p->masks.resize(at);
+                    else same.push_back(block);
+                }
+                p->mask_of.push_back(block);
             }
         }
         p->row_ptr[qt + 1] = (int)p->col_idx.size();
