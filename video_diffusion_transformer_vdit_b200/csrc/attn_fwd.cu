@@ -75,16 +75,7 @@ constexpr uint32_t kSlabBytes = kTile * 64 * 2;  // 16 KiB: 128 rows x 128 B (on
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemP = 128, kTmemO = 256;
 constexpr float kRescaleTau = 8.0f;              // rescale O only when the max grows by > 2^8
-// Which of every 8 consecutive P pairs of a row take the FMA-pipe exp2 instead of the MUFU unit
-// (bit i set: pair i mod 8). Measured on the dense 32,760-token workload: none 1297 - 1300,
-// one of eight 1259 - 1270, two of eight 1247 - 1255, three of eight 1218 TFLOP/s (the XU pipe
-// is not the bound; the extra FMA work lengthens the softmax), so by default every exponential
-// uses MUFU; the software path stays available for other shapes (it passed the GPU parity
-// tests with 0x88 and 0xA8).
-#ifndef VDIT_POLY_PAIRS
-#define VDIT_POLY_PAIRS 0x00u
-#endif
-constexpr uint32_t kPolyPairs = VDIT_POLY_PAIRS;
+
 
 // barrier indices (8 bytes each)
 enum {
@@ -147,37 +138,6 @@ struct AttnArgs {
 
 // ------------------------------------------------------------------------------ PTX wrappers
 
-
-// 2^x on the FMA pipe, for x <= 2^22 (x = -inf gives exactly 0). Cody-Waite range reduction
-// (Cody and Waite, "Software Manual for the Elementary Functions", 1980): x = n + f with
-// n = round(x) and |f| <= 1/2, so 2^x = 2^n * 2^f; 2^f comes from a cubic 1 + c1 f + c2 f^2 +
-// c3 f^3 fitted here for minimal relative error on [-1/2, 1/2] (weighted least squares with
-// Lawson reweighting in float64, coefficients rounded to float32; maximum relative error 1.0e-4
-// in float32 Horner form, far below the 2^-9 of the bf16 P it feeds). n is read from the low
-// mantissa bits of x + 1.5 * 2^23 and added to the exponent field. Inputs below -127 are clamped
-// to -127: there f = 0 and the cubic is exactly 1 (its constant term is pinned to 1 for this),
-// so the assembly gives exactly +0 for masked scores.
-constexpr float kExp2C0 = 1.0f, kExp2C1 = 0.6932829022407532f, kExp2C2 = 0.2422109693288803f,
-                kExp2C3 = 0.05500892922282219f;
-__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
-    float x0, x1;
-    unpack2(x2, x0, x1);
-    x0 = fmaxf(x0, -127.f);
-    x1 = fmaxf(x1, -127.f);
-    const uint64_t xc = pack2(x0, x1);
-    const uint64_t t = add2(xc, pack2(12582912.f, 12582912.f));
-    const uint64_t r = add2(t, pack2(-12582912.f, -12582912.f));
-    const uint64_t f = fma2(r, pack2(-1.f, -1.f), xc);
-    uint64_t q = fma2(pack2(kExp2C3, kExp2C3), f, pack2(kExp2C2, kExp2C2));
-    q = fma2(q, f, pack2(kExp2C1, kExp2C1));
-    q = fma2(q, f, pack2(kExp2C0, kExp2C0));
-    float t0, t1, q0, q1;
-    unpack2(t, t0, t1);
-    unpack2(q, q0, q1);
-    const int n0 = __float_as_int(t0) - 0x4B400000, n1 = __float_as_int(t1) - 0x4B400000;
-    return pack2(__int_as_float(__float_as_int(q0) + (n0 << 23)),
-                 __int_as_float(__float_as_int(q1) + (n1 << 23)));
-}
 
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
@@ -395,8 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st32(t_o + q4 * 32, orow);
                 }
             }
-            // P = 2^(s*c - m*c) as bf16 pairs into the P_h columns of this lane; the pairs
-            // selected by kPolyPairs take the FMA-pipe exp2 so the MUFU pipe is not the bound
+            // P = 2^(s*c - m*c) as bf16 pairs into the P_h columns of this lane (MUFU ex2)
             uint64_t rs2[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) rs2[i] = pack2(0.f, 0.f);
@@ -408,14 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 32; ++i) {
                     const uint64_t x2 =
                         fma2(pack2(sv[64 * half + 2 * i], sv[64 * half + 2 * i + 1]), c2, nmc2);
-                    uint64_t p2;
-                    if (kPolyPairs & (1u << (i & 7))) {
-                        p2 = exp2_fma2(x2);
-                    } else {
-                        float x0, x1;
-                        unpack2(x2, x0, x1);
-                        p2 = pack2(fast_exp2(x0), fast_exp2(x1));
-                    }
+                    float x0, x1;
+                    unpack2(x2, x0, x1);
+                    const uint64_t p2 = pack2(fast_exp2(x0), fast_exp2(x1));
                     rs2[i & 3] = add2(rs2[i & 3], p2);
                     float p0, p1;
                     unpack2(p2, p0, p1);
