@@ -68,9 +68,19 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 def aggregate_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
-    """Whole-job throughput: every rank does flops_per_rank per step (weak scaling), the step
-    time is the slowest rank's."""
+    """Whole-job throughput: every rank does flops_per_rank per step (replicas: weak scaling;
+    equal head shards of one step: strong scaling), the step time is the slowest rank's."""
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def head_shard(heads: int, world: int, rank: int):
+    """Heads [h0, h1) of `rank` when `world` ranks split one step's heads evenly (heads are
+    independent in attention, so each rank runs the same plan on its slice of Q and of the
+    cache, with no exchange)."""
+    if world < 1 or heads % world:
+        raise ValueError(f"{heads} heads do not split evenly over {world} ranks")
+    hg = heads // world
+    return rank * hg, (rank + 1) * hg
 
 
 def config_of(w, extra=None):
@@ -357,6 +367,11 @@ def run_gpu(args, w):
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
+    full_heads = w.heads
+    if args.shard == "heads":
+        import dataclasses
+        h0, h1 = head_shard(w.heads, world, rank)
+        w = dataclasses.replace(w, heads=h1 - h0)
     g = vdit.Geometry(w.grid_h, w.grid_w, w.heads, w.head_dim, w.bands, w.theta)
     m = vdit.Mask(w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, w.tau)
     ft = w.frame_tokens
@@ -365,9 +380,11 @@ def run_gpu(args, w):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
 
     n_kv = w.kv_stream_frames * ft
-    q_h = bf16(synth.qkv_bf16(w.id, w.q_tokens, w.heads, w.head_dim, "q"))
-    k_h = bf16(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "k"))
-    v_h = bf16(synth.qkv_bf16(w.id, n_kv, w.heads, w.head_dim, "v"))
+    q_h = bf16(synth.qkv_bf16(w.id, w.q_tokens, full_heads, w.head_dim, "q"))
+    k_h = bf16(synth.qkv_bf16(w.id, n_kv, full_heads, w.head_dim, "k"))
+    v_h = bf16(synth.qkv_bf16(w.id, n_kv, full_heads, w.head_dim, "v"))
+    if args.shard == "heads":  # this rank's heads of the same step
+        q_h, k_h, v_h = (t[:, h0:h1].contiguous() for t in (q_h, k_h, v_h))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     cache = vdit.KVCache(g, w.capacity_frames, device=dev)
     # history before the timed append (the earlier chunks of a causal rollout)
@@ -604,11 +621,14 @@ def run_gpu(args, w):
             "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic N(0,1), seeded SplitMix64 + Box-Muller, bf16-rounded",
             "config": config_of(w, {
-                "parallelism": f"{world} independent replicas (no collective)",
+                "parallelism": (f"{world} head shards of {w.heads} of {full_heads} heads (no collective)"
+                                if args.shard == "heads" else
+                                f"{world} independent replicas (no collective)"),
                 "l2": "inputs larger than L2: %.0f MB touched per step (Q, K/V chunk, caches, O)"
                       % ((q.numel() * 2 * 2 + append_bytes + cache.k.numel() * 4) / 1e6),
                 "step": "kv_append(newest chunk) + attn_forward (RoPE of Q fused); plan built "
@@ -630,10 +650,11 @@ def run_gpu(args, w):
                            "double-buffered on copy streams overlapping the previous step"},
             "attended": {
                 "pairs_per_s": world * g.heads * info["kept_pairs"] / (attn_ms * 1e-3),
-                "query_tokens_per_s": world * w.q_tokens / (ms_step * 1e-3),
+                "query_tokens_per_s": (1 if args.shard == "heads" else world) * w.q_tokens / (ms_step * 1e-3),
                 "how": "pairs_per_s: kept (query, key, head) triples per second of attn_fwd; "
                        "query_tokens_per_s: query tokens through the whole step (append + "
-                       "attention, all heads) per second; both summed over the replicas"},
+                       "attention, all heads) per second; both summed over the ranks (head "
+                       "shards share their query tokens)"},
             # per step: the append, the attention kernel and, with a key split, the merge
             "gpu_launches": args.steps * (2 + (1 if info["kv_splits"] > 1 else 0)),
             "clocks": clk,
@@ -677,6 +698,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas of the step (weak scaling, default) or one "
+                         "step's heads split evenly over the ranks (strong scaling)")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip timing the other attention configurations")
     args = ap.parse_args()

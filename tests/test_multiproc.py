@@ -236,3 +236,45 @@ def test_kv_push_gloo_two_ranks():
     # the receiver appended exactly what the sender appended
     assert (k0 == k1).all() and (v0 == v1).all()
     assert abs(k0).max() > 0
+
+
+# ----------------------------------------------------------------------------- head shards
+
+def _shard_worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        h0, h1 = bench.head_shard(12, world, rank)
+        # per-rank FLOPs of a dense step on this rank's heads; step time: the slowest rank
+        flops_rank = 4.0 * 128 * (h1 - h0) * 32760 * 32760
+        got = bench.max_over_ranks(4.0 + rank, world)
+        out[rank] = (h0, h1, got, bench.aggregate_tflops(world, flops_rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_shards_cover_the_heads_and_aggregate_strong_scaling(world):
+    port = _free_port()
+    with mp.Manager() as man:
+        out = man.dict()
+        mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    spans = sorted((res[r][0], res[r][1]) for r in range(world))
+    assert spans[0][0] == 0 and spans[-1][1] == 12
+    assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))  # disjoint and contiguous
+    slowest = 4.0 + world - 1
+    assert all(res[r][2] == slowest for r in range(world))
+    # the whole step (all 12 heads) over the slowest rank's time
+    assert res[0][3] == pytest.approx(6.594e12 / (slowest * 1e-3) / 1e12, rel=1e-3)
+
+
+def test_head_shard_rejects_an_uneven_split():
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    with pytest.raises(ValueError):
+        bench.head_shard(12, 8, 0)
