@@ -311,7 +311,17 @@ def time_append(vdit, g, capacity_frames, n_frames, start_frame, dev, stream, n=
         one(i)
     with _nvtx(f"kv_append {n_frames} frames x {g.heads} heads"):
         ms = _time_back_to_back(one, n, stream)
-    return ms, per_set
+    # context: torch's device-to-device copy of the same bytes (K and V into the first frames of
+    # the caches' storage), same sets, same launch pattern: what a plain copy of this size reaches
+    def copy(i):
+        k, v, kc, vc = sets[i % n_sets]
+        kc.view(-1)[:k.numel()].copy_(k.view(-1))
+        vc.view(-1)[:v.numel()].copy_(v.view(-1))
+
+    for i in range(n_sets):
+        copy(i)
+    copy_ms = _time_back_to_back(copy, n, stream)
+    return ms, per_set, copy_ms
 
 
 def time_workload(vdit, w, dev, stream, burst_peak, n=10):
@@ -525,11 +535,12 @@ def run_gpu(args, w):
     for name, heads, nf, start in (("clip", g.heads, n_last, s_last),
                                    ("chunk_1.3b_h12", 12, 3, 18), ("chunk_14b_h40", 40, 3, 396)):
         ga = vdit.Geometry(g.grid_h, g.grid_w, heads, g.head_dim, g.bands, g.theta)
-        a_ms, a_bytes = time_append(vdit, ga, w.capacity_frames if name == "clip" else 21, nf,
-                                    start, dev, stream)
+        a_ms, a_bytes, c_ms = time_append(vdit, ga, w.capacity_frames if name == "clip" else 21, nf,
+                                          start, dev, stream)
         gbs = a_bytes / (a_ms * 1e-3) / 1e9
         appends[name] = {"frames": nf, "heads": heads, "ms": a_ms, "bytes": a_bytes, "gbs": gbs,
-                         "frac_hbm": gbs / pk0["hbm_gbs"]}
+                         "frac_hbm": gbs / pk0["hbm_gbs"],
+                         "torch_copy_same_bytes_gbs": a_bytes / (c_ms * 1e-3) / 1e9}
     torch.cuda.synchronize()
 
     # the other attention configurations, timed in the same run (not part of the step)
@@ -664,7 +675,9 @@ def run_gpu(args, w):
                 "kv_append_frac_hbm": appends["clip"]["frac_hbm"],
                 "kv_append": dict(appends, how="vdit_kv_append alone, 20 launches back to back "
                                   "over distinct source and cache buffers (> 400 MB in all); "
-                                  "bytes = read K, V + write K', V"),
+                                  "bytes = read K, V + write K', V; torch_copy_same_bytes_gbs: "
+                                  "torch's device copy of K and V (two launches) over the same "
+                                  "buffers, for context"),
                 "kv_append_in_step_ms": app_ms,
                 "kv_append_in_step_gbs": append_bytes / (app_ms * 1e-3) / 1e9,
                 "rope3d_apply_ms": rope_ms, "rope3d_apply_gbs": rope_bytes / (rope_ms * 1e-3) / 1e9,

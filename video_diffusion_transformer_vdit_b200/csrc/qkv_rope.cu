@@ -9,17 +9,25 @@
 // (fp32 math, tables built in fp64) and stores bf16: Q to [tokens, heads, head_dim], K' and V
 // straight into the chunk's frame slots of the head-major ring cache (what vdit_kv_append does).
 //
-// One CTA per SM, persistent over 128 x 256 output tiles (in the order that keeps the smaller
-// operand in L2); 6 warps:
-//   warp 0      producer: TMA (SWIZZLE_128B) of the 128 x 64 X tile and the 256 x 64 W tile of
-//               each 64-wide k step into a 4-stage ring;
-//   warp 1      TMEM allocator (512 columns: two 256-column fp32 accumulators) and the single
-//               thread issuing kind::f16 MMAs, M = 128, N = 256, K = 16 (four per k step);
-//   warps 2-5   epilogue: thread r owns accumulator row r (TMEM lane r); per 64-column slab it
-//               loads the fp32 row (tcgen05.ld), rotates the pairs, rounds to bf16 into a
-//               swizzled shared-memory slab and one thread stores the slab with a TMA tensor
-//               store. The accumulator is released as soon as it has been read, so the next
-//               tile's MMAs overlap the stores.
+// Pairs of CTAs (clusters of two, one CTA per SM) run persistent over 256 x 256 output tiles (in
+// the order that keeps the smaller operand in L2) with tcgen05 cta_group::2: one M = 256, N = 256,
+// K = 16 MMA covers the tile, CTA r of the pair staging the X rows m0 + 128 r .. and the W rows
+// n0 + 128 r .. of each 64-wide k step, and receiving its 128 output rows in its own TMEM. 6 warps
+// per CTA:
+//   warp 0      producer: TMA (SWIZZLE_128B) of the CTA's 128 x 64 X and W tiles into a 5-stage
+//               ring; both CTAs' copies complete on the first CTA's stage barrier;
+//   warp 1      paired TMEM allocation (512 columns in each CTA: two 256-column fp32
+//               accumulators); in the first CTA, the single thread issuing the MMAs (four per k
+//               step), which commits them to the barriers of both CTAs;
+//   warps 2-5   epilogue of the CTA's 128 rows: thread r owns accumulator row r (TMEM lane r);
+//               per 64-column slab it loads the fp32 row (tcgen05.ld), rotates the pairs, rounds
+//               to bf16 into a swizzled shared-memory slab and one thread stores the slab with a
+//               TMA tensor store. The accumulator is released (on the first CTA's barrier, which
+//               counts both CTAs' threads) as soon as it has been read, so the next tile's MMAs
+//               overlap the stores.
+// Per SM each MMA reads 8 KiB of operands in 128 cycles and TMA writes 32 KiB per k step: 128 B of
+// shared-memory traffic per cycle at the tensor rate, where a single CTA's M = 128, N = 256 tile
+// would need 192 (its B operand, 256 W rows, read whole by each CTA).
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA raises its abort flag and the
 // status word (VDIT_ERR_TIMEOUT), drains what it issued and frees TMEM before exiting.
 #include <algorithm>
@@ -39,25 +47,11 @@
 namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kGStages = 4;
 constexpr int kGThreads = 192;
 constexpr int kGWarpTMA = 0, kGWarpMMA = 1;  // warps 2-5: epilogue
-constexpr uint32_t kABytes = kBM * kBK * 2;        // 16 KiB
-constexpr uint32_t kBBytes = kBN * kBK * 2;        // 32 KiB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kOutSlab = kBM * 64 * 2;        // 16 KiB: 128 rows x 64 columns of bf16
 constexpr uint32_t kAccCols = kBN;                 // fp32 columns per accumulator
 
-enum { G_FULL = 0, G_EMPTY = G_FULL + kGStages, G_AFULL = G_EMPTY + kGStages,
-       G_AEMPTY = G_AFULL + 2, G_DRAIN = G_AEMPTY + 2, G_COUNT };
-static_assert(G_COUNT <= 16, "barrier area");
-
-constexpr uint32_t OFF_STAGE = 0;
-constexpr uint32_t OFF_OUT = OFF_STAGE + kGStages * kStageBytes;     // two output slabs
-constexpr uint32_t OFF_BAR = OFF_OUT + 2 * kOutSlab;
-constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 16;                        // [0] tmem, [1] abort
-constexpr uint32_t kGSmemBytes = OFF_MISC + 64 + 1024;                 // + alignment slack
-static_assert(kGSmemBytes <= 227 * 1024, "shared memory budget");
 
 struct GemmArgs {
     int m;              // tokens of this launch
@@ -78,20 +72,6 @@ struct GemmArgs {
 
 __device__ int g_qkv_status = 0;
 
-// Output tile t -> (first row, first column). Consecutive tiles run at the same time on different
-// SMs, so the operand they share should be the one that does not fit in L2: with row blocks
-// outer they share X rows and stream all of W (kept when W is the smaller), with column blocks
-// outer they share W columns and stream all of X.
-__device__ __forceinline__ void tile_origin(int t, const GemmArgs& a, int& m0, int& n0) {
-    if (a.n_major) {
-        m0 = (t % a.n_tiles_m) * kBM;
-        n0 = (t / a.n_tiles_m) * kBN;
-    } else {
-        m0 = (t / a.n_tiles_n) * kBM;
-        n0 = (t % a.n_tiles_n) * kBN;
-    }
-}
-
 // (cos, sin) of RoPE pair pp of a head vector at position (t, h, w): bands t, h, w in order.
 __device__ __forceinline__ float2 pair_angle(int pp, int t, int h, int w, const GemmArgs& a) {
     const bool in_h = pp >= a.bt2, in_w = pp >= a.bt2 + a.bh2;
@@ -102,14 +82,6 @@ __device__ __forceinline__ float2 pair_angle(int pp, int t, int h, int w, const 
     return __ldg(tab + (size_t)row * width + jj);
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(map), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
                  "r"(src), "r"(c0), "r"(c1)
@@ -128,42 +100,106 @@ __device__ __forceinline__ void bulk_wait_read() {
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kGThreads, 1)
-    qkv_rope_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
-                    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                    const __grid_constant__ CUtensorMap map_v, const GemmArgs a) {
+// ------------------------------------------------------------------------------ the kernel
+constexpr int kPStages = 5;
+constexpr uint32_t kPABytes = 128 * kBK * 2;                      // 16 KiB of X rows
+constexpr uint32_t kPBBytes = 128 * kBK * 2;                      // 16 KiB of W rows
+constexpr uint32_t kPStageBytes = kPABytes + kPBBytes;
+enum { PG_FULL = 0, PG_EMPTY = PG_FULL + kPStages, PG_AFULL = PG_EMPTY + kPStages,
+       PG_AEMPTY = PG_AFULL + 2, PG_DRAIN = PG_AEMPTY + 2, PG_COUNT };
+static_assert(PG_COUNT <= 16, "barrier area");
+constexpr uint32_t OFF_PSTAGE = 0;
+constexpr uint32_t OFF_POUT = OFF_PSTAGE + kPStages * kPStageBytes;
+constexpr uint32_t OFF_PBAR = OFF_POUT + 2 * kOutSlab;
+constexpr uint32_t OFF_PMISC = OFF_PBAR + 8 * 16;
+constexpr uint32_t kPSmemBytes = OFF_PMISC + 64 + 1024;
+static_assert(kPSmemBytes <= 227 * 1024, "shared memory budget");
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory, completing on an mbarrier of either CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrives on the barrier at this offset in both CTAs of the pair once the MMAs issued so far
+// have completed.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((unsigned short)3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+    qkv_rope_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                         const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                         const __grid_constant__ CUtensorMap map_v, const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    auto BAR = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
-    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+    auto BAR = [&](int i) { return sbase + OFF_PBAR + 8u * (uint32_t)i; };
+    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + OFF_PMISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_PMISC + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_tiles = a.n_tiles_m * a.n_tiles_n;
+    const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs; 1: its peer
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int n_tiles = a.n_tiles_m * a.n_tiles_n;  // 256 x 256 tiles
     const int k_steps = (a.k + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGStages; ++s) {
-            mbar_init(BAR(G_FULL + s), 1);
-            mbar_init(BAR(G_EMPTY + s), 1);
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(BAR(PG_FULL + s), 1);
+            mbar_init(BAR(PG_EMPTY + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(G_AFULL + b), 1);
-            mbar_init(BAR(G_AEMPTY + b), 128);
+            mbar_init(BAR(PG_AFULL + b), 1);
+            mbar_init(BAR(PG_AEMPTY + b), 256);  // the epilogue threads of both CTAs
         }
-        mbar_init(BAR(G_DRAIN), 1);
+        mbar_init(BAR(PG_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kGWarpMMA) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sbase + OFF_MISC),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sbase + OFF_PMISC),
                      "r"(2 * kAccCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
     tc_fence_after();
     const uint32_t tmem = misc[0];
 
@@ -171,54 +207,67 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // ---------------------------------------------------------------------- producer
         int it = 0, issued = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+        const uint32_t full0 = mapa_shared(BAR(PG_FULL), 0);  // the first CTA's stage barriers
+        for (int tile = pair; ok && tile < n_tiles; tile += n_pairs) {
             int m0, n0;
-            tile_origin(tile, a, m0, n0);
+            if (a.n_major) {
+                m0 = (tile % a.n_tiles_m) * 256;
+                n0 = (tile / a.n_tiles_m) * 256;
+            } else {
+                m0 = (tile / a.n_tiles_n) * 256;
+                n0 = (tile % a.n_tiles_n) * 256;
+            }
             for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                const int s = it % kGStages;
-                if (it >= kGStages &&
-                    !warp_wait(BAR(G_EMPTY + s), (uint32_t)((it / kGStages) - 1) & 1u, abort_flag, a.status)) {
+                const int s = it % kPStages;
+                if (it >= kPStages &&
+                    !warp_wait(BAR(PG_EMPTY + s), (uint32_t)((it / kPStages) - 1) & 1u, abort_flag, a.status)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0) {
-                    mbar_expect_tx(BAR(G_FULL + s), kStageBytes);
-                    const uint32_t dst = sbase + OFF_STAGE + s * kStageBytes;
-                    tma_load_2d(dst, &map_x, BAR(G_FULL + s), ks * kBK, m0);
-                    tma_load_2d(dst + kABytes, &map_w, BAR(G_FULL + s), ks * kBK, n0);
+                    if (rank == 0) mbar_expect_tx(BAR(PG_FULL + s), 2 * kPStageBytes);
+                    const uint32_t dst = sbase + OFF_PSTAGE + s * kPStageBytes;
+                    tma_load_2d_pair(dst, &map_x, full0 + 8u * (uint32_t)s, ks * kBK, m0 + 128 * (int)rank);
+                    tma_load_2d_pair(dst + kPABytes, &map_w, full0 + 8u * (uint32_t)s, ks * kBK, n0 + 128 * (int)rank);
                 }
                 issued = it + 1;
                 __syncwarp();
             }
         }
         if (*abort_flag && lane == 0) {
-            // drain: the last kGStages loads this warp issued must land before the CTA exits
-            for (int i = max(0, issued - kGStages); i < issued; ++i) {
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(BAR(G_FULL + i % kGStages), (uint32_t)(i / kGStages) & 1u) &&
-                       globaltimer() - t0 < kWaitLimitNs) {
+            // drain: the loads this warp issued land before the CTA exits. The first CTA waits
+            // on its stage barriers (bounded); the second cannot wait on the first's barriers and
+            // gives its in-flight copies a fixed 200 us
+            const uint64_t t0 = globaltimer();
+            if (rank == 0) {
+                for (int i = max(0, issued - kPStages); i < issued; ++i)
+                    while (!mbar_try_wait(BAR(PG_FULL + i % kPStages), (uint32_t)(i / kPStages) & 1u) &&
+                           globaltimer() - t0 < kWaitLimitNs) {
+                    }
+            } else {
+                while (globaltimer() - t0 < 200000ull) {
                 }
             }
         }
     } else if (warp == kGWarpMMA) {
         // ---------------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = instr_desc(kBN, 0);
-            const uint64_t da = smem_desc_sw128(sbase + OFF_STAGE, 16, 1024);
-            const uint64_t db = smem_desc_sw128(sbase + OFF_STAGE + kABytes, 16, 1024);
-            constexpr uint64_t kStageDesc = kStageBytes >> 4;
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = instr_desc(256, 0, 256);
+            const uint64_t da = smem_desc_sw128(sbase + OFF_PSTAGE, 16, 1024);
+            const uint64_t db = smem_desc_sw128(sbase + OFF_PSTAGE + kPABytes, 16, 1024);
+            constexpr uint64_t kStageDesc = kPStageBytes >> 4;
             int it = 0, nt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++nt) {
+            for (int tile = pair; ok && tile < n_tiles; tile += n_pairs, ++nt) {
                 const int b = nt & 1;
-                if (nt >= 2) {  // the epilogue has read this accumulator's previous tile
-                    if (!wait_bounded(BAR(G_AEMPTY + b), (uint32_t)((nt >> 1) - 1) & 1u, abort_flag, a.status)) break;
+                if (nt >= 2) {  // both CTAs' epilogues have read this accumulator's previous tile
+                    if (!wait_bounded(BAR(PG_AEMPTY + b), (uint32_t)((nt >> 1) - 1) & 1u, abort_flag, a.status)) break;
                     tc_fence_after();
                 }
                 const uint32_t d_t = tmem + (uint32_t)b * kAccCols;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int s = it % kGStages;
-                    if (!wait_bounded(BAR(G_FULL + s), (uint32_t)(it / kGStages) & 1u, abort_flag, a.status)) {
+                    const int s = it % kPStages;
+                    if (!wait_bounded(BAR(PG_FULL + s), (uint32_t)(it / kPStages) & 1u, abort_flag, a.status)) {
                         ok = false;
                         break;
                     }
@@ -226,31 +275,38 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     const uint64_t sa = da + (uint64_t)s * kStageDesc, sb = db + (uint64_t)s * kStageDesc;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(d_t, sa + (uint64_t)(kk * 2), sb + (uint64_t)(kk * 2), idesc, (ks | kk) ? 1u : 0u);
-                    tc_commit(BAR(G_EMPTY + s));
+                        tc_mma_pair(d_t, sa + (uint64_t)(kk * 2), sb + (uint64_t)(kk * 2), idesc, (ks | kk) ? 1u : 0u);
+                    tc_commit_pair_both(BAR(PG_EMPTY + s));
                 }
                 if (!ok) break;
-                tc_commit(BAR(G_AFULL + b));
+                tc_commit_pair_both(BAR(PG_AFULL + b));
             }
-            tc_commit(BAR(G_DRAIN));
+            tc_commit_pair(BAR(PG_DRAIN));
             const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(BAR(G_DRAIN), 0) && globaltimer() - t0 < kWaitLimitNs) {
+            while (!mbar_try_wait(BAR(PG_DRAIN), 0) && globaltimer() - t0 < kWaitLimitNs) {
             }
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------------------------- epilogue
-        const int row = (warp & 3) * 32 + lane;  // TMEM lane of this warp's quarter
+        const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const bool leader = threadIdx.x == 64;   // issues the TMA stores
+        const bool leader = threadIdx.x == 64;
         const int ft = a.grid_h * a.grid_w;
+        const uint32_t aempty0 = mapa_shared(BAR(PG_AEMPTY), 0);  // the first CTA's release barriers
         int nt = 0, slab_n = 0;
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++nt) {
+        for (int tile = pair; tile < n_tiles; tile += n_pairs, ++nt) {
             const int b = nt & 1;
             int m0, n0;
-            tile_origin(tile, a, m0, n0);
-            // the four epilogue warps decide together, so none is left alone in a named barrier
-            const bool got = warp_wait(BAR(G_AFULL + b), (uint32_t)(nt >> 1) & 1u, abort_flag, a.status);
+            if (a.n_major) {
+                m0 = (tile % a.n_tiles_m) * 256;
+                n0 = (tile / a.n_tiles_m) * 256;
+            } else {
+                m0 = (tile / a.n_tiles_n) * 256;
+                n0 = (tile % a.n_tiles_n) * 256;
+            }
+            m0 += 128 * (int)rank;  // this CTA's rows of the tile
+            const bool got = warp_wait(BAR(PG_AFULL + b), (uint32_t)(nt >> 1) & 1u, abort_flag, a.status);
             uint32_t all_got;
             asm volatile(
                 "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
@@ -260,9 +316,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 : "memory");
             if (!all_got) break;
             tc_fence_after();
-            const int section = n0 / a.hd;             // 0: Q, 1: K, 2: V
-            const int col0 = n0 - section * a.hd;      // first feature of the tile in its section
-            // position of this row's token (rows past the launch's tokens are never stored)
+            const int section = n0 / a.hd;
+            const int col0 = n0 - section * a.hd;
             const int tok = a.tok0 + min(m0 + row, a.m - 1);
             const int f = tok / ft, rem = tok - f * ft;
             const int t = a.start_frame + f, hh = rem / a.grid_w, ww = rem - hh * a.grid_w;
@@ -273,13 +328,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 tmem_ld_wait(v);
                 reg_touch32(v + 32);
                 if (sl == kBN / 64 - 1) {
-                    // every column of the accumulator is in registers: release it to the MMAs
+                    // every column of this CTA's accumulator is in registers: release it
                     tc_fence_before();
-                    mbar_arrive(BAR(G_AEMPTY + b));
+                    mbar_arrive_cluster(aempty0 + 8u * (uint32_t)b);
                 }
-                const int feat0 = col0 + sl * 64;  // first feature of the slab in its section
+                const int feat0 = col0 + sl * 64;
                 if (section < 2) {
-                    const int pp0 = (feat0 % a.head_dim) >> 1;  // first pair of the slab in its head
+                    const int pp0 = (feat0 % a.head_dim) >> 1;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const float2 cs = pair_angle(pp0 + i, t, hh, ww, a);
@@ -288,11 +343,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         v[2 * i + 1] = __float_as_uint(fmaf(x0, cs.y, x1 * cs.x));
                     }
                 }
-                // the staging slab written two slabs ago must have been read by its TMA store
                 const int buf = slab_n & 1;
                 if (leader) bulk_wait_read<1>();
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                uint8_t* stage = smem + OFF_OUT + buf * kOutSlab;
+                uint8_t* stage = smem + OFF_POUT + buf * kOutSlab;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t w4[4];
@@ -307,15 +361,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
                 fence_proxy_async_smem();
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (leader) {
-                    const uint32_t src = sbase + OFF_OUT + buf * kOutSlab;
+                if (leader && m0 < a.m) {
+                    const uint32_t src = sbase + OFF_POUT + buf * kOutSlab;
                     if (section == 0)
                         tma_store_2d(&map_q, src, feat0, m0);
                     else
                         tma_store_3d(section == 1 ? &map_k : &map_v, src, feat0 % a.head_dim, m0,
                                      feat0 / a.head_dim);
-                    bulk_commit();
                 }
+                if (leader) bulk_commit();
             }
         }
         if (leader) bulk_wait_all();
@@ -323,9 +377,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // ------------------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // the first CTA's MMAs into this CTA's TMEM have completed (its drain)
     if (warp == kGWarpMMA) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kAccCols)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kAccCols)
                      : "memory");
     }
 }
@@ -373,9 +428,10 @@ int qkv_device_state(int dev, QkvDeviceState* out) {
     std::lock_guard<std::mutex> lk(g_qkv_dev_mu);
     QkvDeviceState& st = g_qkv_dev[dev];
     if (!st.ready) {
-        if (int rc = vdit::cuda_check(cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                           (int)kGSmemBytes),
-                                      "cudaFuncSetAttribute(qkv_rope)"))
+        if (int rc = vdit::cuda_check(cudaFuncSetAttribute(qkv_rope_pair_kernel,
+                                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                           (int)kPSmemBytes),
+                                      "cudaFuncSetAttribute(qkv_rope_pair)"))
             return rc;
         void* sp = nullptr;
         if (int rc = vdit::cuda_check(cudaGetSymbolAddress(&sp, g_qkv_status), "cudaGetSymbolAddress(status)"))
@@ -404,9 +460,10 @@ int launch_part(const vdit_geom* g, const vdit::RopeTables& tabs, const uint8_t*
         if (int rc = encode(&mx, x + (size_t)tok0 * d_model * 2, 2, dims, str, box)) return rc;
     }
     {
+        // each CTA of a pair stages 128 of the 256 W rows of a tile
         cuuint64_t dims[2] = {(cuuint64_t)d_model, (cuuint64_t)3 * hd};
         cuuint64_t str[1] = {(cuuint64_t)d_model * 2};
-        cuuint32_t box[2] = {64, kBN};
+        cuuint32_t box[2] = {64, 128};
         if (int rc = encode(&mw, w, 2, dims, str, box)) return rc;
     }
     {
@@ -425,7 +482,7 @@ int launch_part(const vdit_geom* g, const vdit::RopeTables& tabs, const uint8_t*
     GemmArgs a{};
     a.m = n_tok;
     a.k = d_model;
-    a.n_tiles_m = (n_tok + kBM - 1) / kBM;
+    a.n_tiles_m = (n_tok + 255) / 256;
     a.n_tiles_n = 3 * hd / kBN;
     a.n_major = (long long)3 * hd > (long long)n_tok ? 1 : 0;  // W larger than X: keep X in L2
     a.hd = hd;
@@ -442,8 +499,8 @@ int launch_part(const vdit_geom* g, const vdit::RopeTables& tabs, const uint8_t*
     a.bw2 = g->band_w / 2;
     a.status = ds.status;
     const int tiles = a.n_tiles_m * a.n_tiles_n;
-    const int grid = std::min(tiles, ds.sms);
-    qkv_rope_kernel<<<grid, kGThreads, kGSmemBytes, st>>>(mx, mw, mq, mk, mv, a);
+    const int grid = 2 * std::min(tiles, ds.sms / 2);  // clusters of two CTAs, persistent
+    qkv_rope_pair_kernel<<<grid, kGThreads, kPSmemBytes, st>>>(mx, mw, mq, mk, mv, a);
     return vdit::cuda_check(cudaGetLastError(), "qkv_rope kernel launch");
 }
 
