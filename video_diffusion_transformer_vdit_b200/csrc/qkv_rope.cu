@@ -101,17 +101,17 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------------------ the kernel
-constexpr int kPStages = 5;
+constexpr int kPStages = 5;  // 4 / 5 / 6 stages measured 1 424 / 1 424 / 1 433 TFLOP/s (1.3B clip)
 constexpr uint32_t kPABytes = 128 * kBK * 2;                      // 16 KiB of X rows
 constexpr uint32_t kPBBytes = 128 * kBK * 2;                      // 16 KiB of W rows
 constexpr uint32_t kPStageBytes = kPABytes + kPBBytes;
 enum { PG_FULL = 0, PG_EMPTY = PG_FULL + kPStages, PG_AFULL = PG_EMPTY + kPStages,
        PG_AEMPTY = PG_AFULL + 2, PG_DRAIN = PG_AEMPTY + 2, PG_COUNT };
-static_assert(PG_COUNT <= 16, "barrier area");
+static_assert(PG_COUNT <= 32, "barrier area");
 constexpr uint32_t OFF_PSTAGE = 0;
 constexpr uint32_t OFF_POUT = OFF_PSTAGE + kPStages * kPStageBytes;
 constexpr uint32_t OFF_PBAR = OFF_POUT + 2 * kOutSlab;
-constexpr uint32_t OFF_PMISC = OFF_PBAR + 8 * 16;
+constexpr uint32_t OFF_PMISC = OFF_PBAR + 8 * 32;
 constexpr uint32_t kPSmemBytes = OFF_PMISC + 64 + 1024;
 static_assert(kPSmemBytes <= 227 * 1024, "shared memory budget");
 
