@@ -121,6 +121,9 @@ typedef struct vdit_plan_info_t {
     long long mask_bytes;      /* keep masks of the partial tiles: 2 KiB per distinct block
                                   (identical blocks of several tiles are stored once; see
                                   vdit_plan_export_masks) */
+    int work_entries;          /* entries of the kernel's work list (vdit_plan_export_work) */
+    int single_patch_entries;  /* of which single-patch entries at unaligned key rows */
+    long long work_mask_bytes; /* keep-mask blocks of the work list (2 KiB per distinct block) */
 } vdit_plan_info_t;
 
 /* 3-D RoPE ([CRoPE] 2.B, [TR] Metodologia 1) of n_tokens consecutive tokens of one chunk whose
@@ -190,6 +193,19 @@ VDIT_API int vdit_plan_export(const vdit_plan* p, int* row_ptr, int* col_idx, un
  * is kept iff bit (k mod 32) of words[512 b + 4 r + k / 32] is set. Rows and keys past the token
  * counts are 0. mask_index: [tiles]; words: [mask_bytes / 4] (may be NULL when mask_bytes is 0). */
 VDIT_API int vdit_plan_export_masks(const vdit_plan* p, int* mask_index, unsigned int* words);
+
+/* Host copy of the attention kernel's work list. It covers the same kept pairs as the schedule
+ * above, each exactly once, but for radial masks on frames of at least 128 tokens the "same
+ * patch" pairs of frame offsets whose radial window is a single patch (radius 0; [DR] sec. 2:
+ * the window narrows with temporal distance) leave the aligned tiles: per query tile and such
+ * offset one entry at an unaligned key row k holds them, query row r meeting key row k + r (the
+ * same patch dt frames away), when that shortens the tile's list. For query tile qt, entries
+ * row_ptr[qt] .. row_ptr[qt + 1] - 1 give key_row (first of 128 consecutive key rows) and
+ * mask_index (a block of words, laid out as in vdit_plan_export_masks, or -1 for a complete,
+ * wholly kept tile). row_ptr: [q_tiles + 1]; key_row, mask_index: [work_entries]; words:
+ * [work_mask_bytes / 4] (may be NULL when that is 0). */
+VDIT_API int vdit_plan_export_work(const vdit_plan* p, int* row_ptr, int* key_row, int* mask_index,
+                                   unsigned int* words);
 
 VDIT_API void vdit_plan_destroy(vdit_plan* p);
 

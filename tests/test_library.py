@@ -127,6 +127,77 @@ def _check_masks(plan, grid_h, grid_w, q_start, q_frames, cap, first, last, kind
             assert np.array_equal(got, want), (qt, kt)
 
 
+def _check_work(plan, grid_h, grid_w, q_start, q_frames, cap, first, last, kind, chunk, w0, g, lam,
+                q_tiles=None):
+    """The kernel's work list covers exactly the oracle's kept pairs, each once: per query tile,
+    the entries' 128-key blocks (all ones for a full tile) placed at their key rows add up to the
+    oracle's explicit mask rows, with no pair covered twice."""
+    rp, kr, mi, words = plan.export_work()
+    n_q = q_frames * grid_h * grid_w
+    qpos = oracle.positions(n_q, grid_h, grid_w, q_start)
+    kpos, kvalid = oracle.cache_positions(cap, first, last, grid_h, grid_w)
+    m = oracle.Mask(block_causal=bool(kind & 1), radial=bool(kind & 2), chunk_frames=chunk,
+                    w0=w0, gamma_shift=g, lam=lam)
+    n_k = len(kvalid)
+    bits = np.arange(32, dtype=np.uint32)
+    for qt in (range(len(rp) - 1) if q_tiles is None else q_tiles):
+        q0, q1 = qt * 128, min(n_q, qt * 128 + 128)
+        ref = oracle.mask_rows(tuple(p[q0:q1] for p in qpos), kpos, kvalid, m).astype(bool)
+        cover = np.zeros((q1 - q0, n_k + 128), np.int32)
+        for e in range(rp[qt], rp[qt + 1]):
+            k0 = int(kr[e])
+            assert 0 <= k0 < n_k
+            if mi[e] < 0:
+                blk = np.ones((128, 128), bool)
+            else:
+                blk = ((words[mi[e]][:, :, None] >> bits) & 1).reshape(128, 128).astype(bool)
+            cover[:, k0:k0 + 128] += blk[:q1 - q0]
+        assert cover.max(initial=0) <= 1, qt          # no pair twice
+        assert not cover[:, n_k:].any(), qt             # nothing past the last key
+        assert np.array_equal(cover[:, :n_k].astype(bool), ref), qt
+
+
+@pytest.mark.parametrize("wid", sorted(WORKLOADS))
+def test_kernel_work_list_covers_the_mask_once_workloads(wid):
+    w = WORKLOADS[wid]
+    first, last = w.window()
+    plan = vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                     kv_first_frame=first, kv_last_frame=last, upload=False)
+    n_qt = plan.info["q_tiles"]
+    sample = None if n_qt <= 8 else sorted({0, 1, n_qt // 3, n_qt // 2, (2 * n_qt) // 3, n_qt - 2, n_qt - 1})
+    _check_work(plan, w.grid_h, w.grid_w, w.q_start, w.q_frames, w.capacity_frames, first, last,
+                w.mask_kind, w.chunk_frames, w.w0, w.gamma_shift, w.lam, sample)
+    info = plan.info
+    if w.mask_kind & 2:
+        # the radial workloads take their single-patch pairs off the aligned tiles
+        assert info["single_patch_entries"] > 0 and info["work_entries"] < info["tiles"]
+    else:
+        assert info["single_patch_entries"] == 0 and info["work_entries"] == info["tiles"]
+
+
+def test_kernel_work_list_covers_the_mask_once_random_geometries():
+    # frames of at least 128 tokens (where single-patch entries apply), rings that wrap, both
+    # causal and not, radial radii that reach 0 within the window
+    rng = np.random.default_rng(12)
+    n_single = 0
+    for _ in range(24):
+        gh, gw = int(rng.integers(4, 14)), int(rng.integers(32, 60))
+        cap = int(rng.integers(3, 14))
+        last = int(rng.integers(0, 40))
+        first = max(0, last - int(rng.integers(0, cap)))
+        q_frames = int(rng.integers(1, 4))
+        q_start = int(rng.integers(max(0, last - 6), last + 2))
+        kind = int(rng.choice([2, 3]))
+        chunk = int(rng.integers(1, 4))
+        w0, gs, lam = int(rng.integers(0, 20)), int(rng.integers(1, 3)), int(rng.integers(0, 7))
+        g = vdit.Geometry(gh, gw, 1, 64, (24, 20, 20))
+        plan = vdit.Plan(g, vdit.Mask(kind, chunk, w0, gs, lam), q_start, q_frames,
+                         capacity_frames=cap, kv_first_frame=first, kv_last_frame=last, upload=False)
+        _check_work(plan, gh, gw, q_start, q_frames, cap, first, last, kind, chunk, w0, gs, lam)
+        n_single += plan.info["single_patch_entries"]
+    assert n_single > 0
+
+
 @pytest.mark.parametrize("wid", sorted(WORKLOADS))
 def test_plan_masks_bit_exact_vs_oracle_workloads(wid):
     w = WORKLOADS[wid]

@@ -64,7 +64,8 @@ class _PlanInfo(ctypes.Structure):
                 ("kv_tiles", ctypes.c_int), ("tiles", ctypes.c_int), ("full_tiles", ctypes.c_int),
                 ("kept_pairs", ctypes.c_longlong), ("uploaded", ctypes.c_int),
                 ("kv_splits", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong),
-                ("mask_bytes", ctypes.c_longlong)]
+                ("mask_bytes", ctypes.c_longlong), ("work_entries", ctypes.c_int),
+                ("single_patch_entries", ctypes.c_int), ("work_mask_bytes", ctypes.c_longlong)]
 
 
 _lib = None
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_info.argtypes = [P, ctypes.POINTER(_PlanInfo)]
         L.vdit_plan_export.argtypes = [P, P, P, P]
         L.vdit_plan_export_masks.argtypes = [P, P, P]
+        L.vdit_plan_export_work.argtypes = [P, P, P, P, P]
         L.vdit_plan_split_for.argtypes = [P, I, ctypes.POINTER(I)]
         L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
         L.vdit_seq_pack.argtypes = [gp, P, P, P, P, P, P, P, I, I, I, LL, I, P]
@@ -498,6 +500,22 @@ class Plan:
         _check(lib().vdit_plan_export_masks(self._h, ctypes.c_void_p(idx.ctypes.data),
                                             ctypes.c_void_p(words.ctypes.data)))
         return idx[:inf["tiles"]], words[:inf["mask_bytes"] // 4].reshape(-1, 128, 4)
+
+    def export_work(self):
+        """The kernel's work list: (row_ptr [q_tiles + 1], key_row [entries], mask_index
+        [entries], words [blocks, 128, 4]) as numpy arrays (vdit_plan_export_work)."""
+        import numpy as np
+        inf = self.info
+        rp = np.zeros(inf["q_tiles"] + 1, np.int32)
+        kr = np.zeros(max(1, inf["work_entries"]), np.int32)
+        mi = np.zeros(max(1, inf["work_entries"]), np.int32)
+        words = np.zeros(max(4, inf["work_mask_bytes"] // 4), np.uint32)
+        _check(lib().vdit_plan_export_work(self._h, ctypes.c_void_p(rp.ctypes.data),
+                                           ctypes.c_void_p(kr.ctypes.data),
+                                           ctypes.c_void_p(mi.ctypes.data),
+                                           ctypes.c_void_p(words.ctypes.data)))
+        n = inf["work_entries"]
+        return rp, kr[:n], mi[:n], words[:inf["work_mask_bytes"] // 4].reshape(-1, 128, 4)
 
     def split_for(self, sm_count: int) -> int:
         """The key split vdit_plan_upload would choose on a device with sm_count SMs."""

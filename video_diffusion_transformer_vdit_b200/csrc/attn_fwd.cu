@@ -110,8 +110,9 @@ struct Layout {
 };
 
 struct AttnArgs {
-    const int* u_row_ptr;  // per block of two q-tiles: union key-tile list
-    const int* u_col;
+    const int* u_row_ptr;  // per block of two q-tiles: union list of key tiles
+    const int* u_col;      // first key row of each entry (a multiple of 128, or the unaligned
+                           // row of a single-patch entry)
     const unsigned char* u_flags;
     const int* unit_order; // q-blocks, longest list first
     float* ws_o;           // split > 1: normalised partial O [split][q_tokens][heads][D]
@@ -512,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dst = sbase + L::OFF_K + s * kTileBytes;
 #pragma unroll
                 for (int sl = 0; sl < L::kSlabs; ++sl)
-                    tma_load_3d(dst + sl * kSlabBytes, &tmap_k, BAR(B_KFULL + s), 64 * sl, kt * kTile, head);
+                    tma_load_3d(dst + sl * kSlabBytes, &tmap_k, BAR(B_KFULL + s), 64 * sl, kt, head);
                 k_last = it;
             }
             if (it >= kStages && !warp_wait(BAR(B_IEMPTY + s), ph, abort_flag, a.status)) break;
@@ -548,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dst = sbase + L::OFF_V + sv * kTileBytes;
 #pragma unroll
                 for (int sl = 0; sl < L::kSlabs; ++sl)
-                    tma_load_3d(dst + sl * kSlabBytes, &tmap_v, BAR(B_VFULL + sv), 64 * sl, kt * kTile, head);
+                    tma_load_3d(dst + sl * kSlabBytes, &tmap_v, BAR(B_VFULL + sv), 64 * sl, kt, head);
                 v_last = jv;
             }
             __syncwarp();

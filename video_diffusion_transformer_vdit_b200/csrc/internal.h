@@ -53,7 +53,8 @@ struct vdit_plan {
     std::vector<int> slot_frame;  // global frame held by each frame slot, -1 if empty
     std::vector<int> radius;      // per dt in [0, dt_max]: largest kept Chebyshev distance
     // Blocks of two consecutive q-tiles (2b, 2b+1), the unit one attention CTA works on: the
-    // ascending union of the two tiles' key-tile lists, with per entry
+    // union of the two tiles' work lists (aligned entries merged by key row, ascending; then the
+    // single-patch entries, each for one q-tile), with per entry
     //   bit0: listed for q-tile 2b, bit1: full for 2b, bit2: listed for 2b+1, bit3: full for 2b+1.
     int n_qb = 0;
     std::vector<int> u_row_ptr, u_col;
@@ -61,10 +62,20 @@ struct vdit_plan {
     std::vector<int> unit_order;  // q-blocks by descending union-list length (longest first)
     // keep masks of the partial tiles: mask_of[i] = block of CSR entry i (-1: full tile); block b
     // = masks[512 b ..): 128 rows x 4 words, bit k of row r = key k of the tile kept for query r.
-    // u_mask[2 e + x] = block of union entry e for q-tile 2b + x (-1: not listed or full)
+    // u_mask[2 e + x] = block in kmasks of union entry e for q-tile 2b + x (-1: not listed or full)
     std::vector<int> mask_of;
     std::vector<uint32_t> masks;
     std::vector<int> u_mask;
+    // The kernel's work list, per q-tile: entries (first key row, keep-mask block or -1 for a full
+    // tile) in kmasks. It holds the listed tiles above, except that for frames whose radial
+    // window is a single patch (radius 0) the kept "same patch" pairs of a q-tile are taken out of
+    // the aligned tiles into one entry at an unaligned key row: query row r of the q-tile meets
+    // key row w_key + r, the same patch dt frames away (when that moves work off the tensor path).
+    // The union lists u_* are built from this list (u_col holds first key rows).
+    std::vector<int> w_row_ptr, w_key, w_mask;
+    std::vector<int> w_aligned;   // per q-tile: its first w_aligned[qt] entries are aligned tiles
+    std::vector<uint32_t> kmasks;
+    int n_diag = 0;               // entries of the single-patch kind
     // key-range split of every (q-block, head) unit, chosen at upload from the SM count so the
     // number of CTAs fills whole waves; > 1 uses the fp32 partial workspace below
     int n_split = 1;

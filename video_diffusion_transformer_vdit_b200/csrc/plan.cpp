@@ -112,7 +112,7 @@ long long pairs_within(int a0, int a1, int b0, int b1, int r) {
 // query q0 + r. Per (query, key segment) the kept keys form one run of columns (the predicate's
 // frame and row terms are constant on a segment and the Chebyshev window is an interval of w).
 void tile_mask(const vdit_plan& p, int q0, int q1, const std::vector<Seg>& keys,
-               std::vector<uint32_t>& out) {
+               std::vector<uint32_t>& out, const std::vector<int>* skip_dt = nullptr) {
     const size_t base = out.size();
     out.resize(base + 512, 0u);
     uint32_t* blk = out.data() + base;
@@ -124,6 +124,7 @@ void tile_mask(const vdit_plan& p, int q0, int q1, const std::vector<Seg>& keys,
         uint32_t* row = blk + 4 * r;
         for (const Seg& b : keys) {
             if (b.t < 0) continue;
+            if (skip_dt && std::find(skip_dt->begin(), skip_dt->end(), b.t - tq) != skip_dt->end()) continue;
             if (causal && b.t / p.m.chunk_frames > tq / p.m.chunk_frames) continue;
             const long long rad = p.radius[std::abs(tq - b.t)];
             if (std::abs(hq - b.h) > rad) continue;
@@ -137,6 +138,56 @@ void tile_mask(const vdit_plan& p, int q0, int q1, const std::vector<Seg>& keys,
             }
         }
     }
+}
+
+// Kept-pair scan of one (query tile, key tile) pair from its row segments: whether any pair is
+// kept, whether the tile is complete and wholly kept, and the number of kept pairs. Key segments
+// at a frame offset (key frame - query frame) listed in skip_dt count as not kept.
+void scan_tile(const vdit_plan& p, const std::vector<Seg>& qs, const std::vector<Seg>& ks, bool complete,
+               const std::vector<int>* skip_dt, bool& any, bool& all, long long& kept) {
+    const bool causal = p.m.kind & VDIT_MASK_BLOCK_CAUSAL;
+    any = false;
+    all = complete;
+    kept = 0;
+    for (const Seg& a : qs) {
+        for (const Seg& b : ks) {
+            if (b.t < 0) { all = false; continue; }
+            if (skip_dt && std::find(skip_dt->begin(), skip_dt->end(), b.t - a.t) != skip_dt->end()) {
+                all = false;
+                continue;
+            }
+            if (causal && b.t / p.m.chunk_frames > a.t / p.m.chunk_frames) {
+                all = false;
+                continue;
+            }
+            const int r = p.radius[std::abs(a.t - b.t)];
+            if (std::abs(a.h - b.h) > r) { all = false; continue; }
+            const int dmin = std::max(0, std::max(b.wlo - a.whi, a.wlo - b.whi));
+            const int dmax = std::max(a.whi - b.wlo, b.whi - a.wlo);
+            if (dmin <= r) {
+                any = true;
+                kept += pairs_within(a.wlo, a.whi, b.wlo, b.whi, r);
+            }
+            if (dmax > r) all = false;
+        }
+    }
+}
+
+// Stores the 512-word block at the end of `pool` once: returns the number of an identical block
+// already in the pool (and drops the new copy), else the new block's number.
+int dedupe_block(std::vector<uint32_t>& pool, std::unordered_map<uint64_t, std::vector<int>>& seen) {
+    const size_t at = pool.size() - 512;
+    uint64_t hsh = 1469598103934665603ull;  // FNV-1a over the 512 words
+    for (size_t wi = at; wi < at + 512; ++wi) hsh = (hsh ^ pool[wi]) * 1099511628211ull;
+    auto& same = seen[hsh];
+    for (int b : same)
+        if (std::equal(pool.begin() + at, pool.begin() + at + 512, pool.begin() + (size_t)b * 512)) {
+            pool.resize(at);
+            return b;
+        }
+    const int block = (int)(at / 512);
+    same.push_back(block);
+    return block;
 }
 
 }  // namespace
@@ -202,84 +253,151 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
         segments(kt * VDIT_TILE, std::min(p->kv_tokens, (kt + 1) * VDIT_TILE), g->grid_h,
                  g->grid_w, [&](int slot) { return p->slot_frame[slot]; }, kseg[kt]);
     std::vector<Seg> qs;
-    std::unordered_map<uint64_t, std::vector<int>> seen;  // mask block hash -> block numbers
+    std::unordered_map<uint64_t, std::vector<int>> seen, kseen;  // mask block hash -> block numbers
     p->row_ptr.assign(p->n_qt + 1, 0);
+    p->w_row_ptr.assign(p->n_qt + 1, 0);
+    p->w_aligned.assign(p->n_qt, 0);
     p->kept_pairs = 0;
     p->n_full = 0;
+    // single-patch entries need a q-tile to span at most two frames (128 <= tokens per frame)
+    const bool single_patch = (m->kind & VDIT_MASK_RADIAL) && ft >= VDIT_TILE;
+    std::vector<int> dts;
     for (int qt = 0; qt < p->n_qt; ++qt) {
         const int q0 = qt * VDIT_TILE, q1 = std::min(p->q_tokens, q0 + VDIT_TILE);
         segments(q0, q1, g->grid_h, g->grid_w, [&](int f) { return q_start_frame + f; }, qs);
+        // schedule of the mask as it is (export, and the kernel's unless single-patch entries
+        // pay off below)
+        int n_export = 0;
         for (int kt = 0; kt < p->n_kt; ++kt) {
             const int k0 = kt * VDIT_TILE, k1 = std::min(p->kv_tokens, k0 + VDIT_TILE);
-            bool any = false;
-            bool all = (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE);
-            long long kept = 0;
-            for (const Seg& a : qs) {
-                for (const Seg& b : kseg[kt]) {
-                    if (b.t < 0) { all = false; continue; }
-                    if (causal && b.t / m->chunk_frames > a.t / m->chunk_frames) {
-                        all = false;
-                        continue;
-                    }
-                    const int r = p->radius[std::abs(a.t - b.t)];
-                    if (std::abs(a.h - b.h) > r) { all = false; continue; }
-                    const int dmin = std::max(0, std::max(b.wlo - a.whi, a.wlo - b.whi));
-                    const int dmax = std::max(a.whi - b.wlo, b.whi - a.wlo);
-                    if (dmin <= r) {
-                        any = true;
-                        kept += pairs_within(a.wlo, a.whi, b.wlo, b.whi, r);
-                    }
-                    if (dmax > r) all = false;
-                }
-            }
+            bool any, all;
+            long long kept;
+            scan_tile(*p, qs, kseg[kt], (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE), nullptr, any, all, kept);
             p->kept_pairs += kept;
-            if (any) {
-                p->col_idx.push_back(kt);
-                p->full.push_back(all ? 1 : 0);
-                p->n_full += all;
-                int block = -1;
-                if (!all) {
-                    // keep-mask block of this tile; identical blocks (tiles at the same offsets
-                    // within their frames with the same radii) are stored once, so the blocks the
-                    // kernel reads for all heads stay resident in L2
-                    const size_t at = p->masks.size();
-                    tile_mask(*p, q0, q1, kseg[kt], p->masks);
-                    uint64_t hsh = 1469598103934665603ull;  // FNV-1a over the 512 words
-                    for (size_t wi = at; wi < at + 512; ++wi) hsh = (hsh ^ p->masks[wi]) * 1099511628211ull;
-                    block = (int)(at / 512);
-                    auto& same = seen[hsh];
-                    for (int b : same)
-                        if (std::equal(p->masks.begin() + at, p->masks.begin() + at + 512,
-                                       p->masks.begin() + (size_t)b * 512)) {
-                            block = b;
-                            break;
-                        }
-                    if (block != (int)(at / 512)) p->masks.resize(at);
-                    else same.push_back(block);
-                }
-                p->mask_of.push_back(block);
+            if (!any) continue;
+            ++n_export;
+            p->col_idx.push_back(kt);
+            p->full.push_back(all ? 1 : 0);
+            p->n_full += all;
+            int block = -1;
+            if (!all) {
+                // keep-mask block of this tile; identical blocks (tiles at the same offsets within
+                // their frames with the same radii) are stored once, so the blocks the kernel
+                // reads for all heads stay resident in L2
+                tile_mask(*p, q0, q1, kseg[kt], p->masks);
+                block = dedupe_block(p->masks, seen);
             }
+            p->mask_of.push_back(block);
         }
         p->row_ptr[qt + 1] = (int)p->col_idx.size();
+
+        // frame offsets dt (key frame - query frame) whose radial window is one patch: the kept
+        // pairs at dt are (q, q + dt frames), one contiguous run of 128 key rows when the key
+        // frames of the tile's (at most two) query frames sit in consecutive ring slots
+        dts.clear();
+        const int fa = q0 / ft, fb = (q1 - 1) / ft;
+        const int ta = q_start_frame + fa, tb = q_start_frame + fb;
+        if (single_patch) {
+            for (int dt = kv_first_frame - tb; dt <= kv_last_frame - ta; ++dt) {
+                if (p->radius[std::abs(dt)] != 0 || ta + dt < 0) continue;
+                const int sa = (ta + dt) % capacity_frames;
+                if (fb != fa && sa == capacity_frames - 1) continue;  // the run wraps the ring
+                bool valid = false;
+                for (int t = ta; t <= tb && !valid; ++t) {
+                    const int kf = t + dt;
+                    valid = kf >= kv_first_frame && kf <= kv_last_frame &&
+                            !(causal && kf / m->chunk_frames > t / m->chunk_frames);
+                }
+                if (valid) dts.push_back(dt);
+            }
+        }
+        // kernel work list: the aligned tiles without the single-patch pairs, plus one entry per
+        // offset, kept only when it shortens the list
+        std::vector<int> key, blk;
+        if (!dts.empty()) {
+            for (int kt = 0; kt < p->n_kt; ++kt) {
+                const int k0 = kt * VDIT_TILE, k1 = std::min(p->kv_tokens, k0 + VDIT_TILE);
+                bool any, all;
+                long long kept;
+                scan_tile(*p, qs, kseg[kt], (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE), &dts, any, all, kept);
+                if (!any) continue;
+                key.push_back(k0);
+                int block = -1;
+                if (!all) {
+                    tile_mask(*p, q0, q1, kseg[kt], p->kmasks, &dts);
+                    block = dedupe_block(p->kmasks, kseen);
+                }
+                blk.push_back(block);
+            }
+            if ((int)(key.size() + dts.size()) >= n_export) dts.clear();  // no gain: plain tiles
+        }
+        if (dts.empty()) {
+            p->w_aligned[qt] = p->row_ptr[qt + 1] - p->row_ptr[qt];
+            for (int i = p->row_ptr[qt]; i < p->row_ptr[qt + 1]; ++i) {
+                p->w_key.push_back(p->col_idx[i] * VDIT_TILE);
+                int block = -1;
+                if (!p->full[i]) {
+                    p->kmasks.insert(p->kmasks.end(), p->masks.begin() + (size_t)p->mask_of[i] * 512,
+                                     p->masks.begin() + (size_t)p->mask_of[i] * 512 + 512);
+                    block = dedupe_block(p->kmasks, kseen);
+                }
+                p->w_mask.push_back(block);
+            }
+        } else {
+            p->w_aligned[qt] = (int)key.size();
+            p->w_key.insert(p->w_key.end(), key.begin(), key.end());
+            p->w_mask.insert(p->w_mask.end(), blk.begin(), blk.end());
+            for (int dt : dts) {
+                // row r (query q0 + r at frame t) keeps key row k_start + r, its own patch at
+                // frame t + dt, if that frame is held and the chunk order allows it
+                const int k_start = ((ta + dt) % capacity_frames) * ft + (q0 - fa * ft);
+                const size_t at = p->kmasks.size();
+                p->kmasks.resize(at + 512, 0u);
+                for (int r = 0; r < q1 - q0; ++r) {
+                    const int t = q_start_frame + (q0 + r) / ft, kf = t + dt;
+                    const bool keep = kf >= kv_first_frame && kf <= kv_last_frame &&
+                                      !(causal && kf / m->chunk_frames > t / m->chunk_frames) &&
+                                      k_start + r < p->kv_tokens;
+                    if (keep) p->kmasks[at + 4 * r + (r >> 5)] |= 1u << (r & 31);
+                }
+                p->w_key.push_back(k_start);
+                p->w_mask.push_back(dedupe_block(p->kmasks, kseen));
+                ++p->n_diag;
+            }
+        }
+        p->w_row_ptr[qt + 1] = (int)p->w_key.size();
     }
-    // union lists of q-tile pairs
+    // union lists of q-tile pairs, from the kernel's work list: entries at the same (aligned) key
+    // row merge; an unaligned single-patch entry stays on its own (one q-tile)
     p->n_qb = (p->n_qt + 1) / 2;
     p->u_row_ptr.assign(p->n_qb + 1, 0);
     for (int b = 0; b < p->n_qb; ++b) {
         const int t0 = 2 * b, t1 = 2 * b + 1;
-        int i = p->row_ptr[t0], ie = p->row_ptr[t0 + 1];
-        int k = t1 < p->n_qt ? p->row_ptr[t1] : 0, ke = t1 < p->n_qt ? p->row_ptr[t1 + 1] : 0;
+        // aligned entries of the two q-tiles, merged by key row (both ascending)
+        int i = p->w_row_ptr[t0], ie = i + p->w_aligned[t0];
+        int k = t1 < p->n_qt ? p->w_row_ptr[t1] : 0, ke = t1 < p->n_qt ? k + p->w_aligned[t1] : 0;
         while (i < ie || k < ke) {
-            const int ci = i < ie ? p->col_idx[i] : INT_MAX, ck = k < ke ? p->col_idx[k] : INT_MAX;
+            const int ci = i < ie ? p->w_key[i] : INT_MAX, ck = k < ke ? p->w_key[k] : INT_MAX;
             const int c = std::min(ci, ck);
             unsigned char f = 0;
             int m0 = -1, m1 = -1;
-            if (ci == c) { f |= 1 | (p->full[i] ? 2 : 0); m0 = p->mask_of[i]; ++i; }
-            if (ck == c) { f |= 4 | (p->full[k] ? 8 : 0); m1 = p->mask_of[k]; ++k; }
+            if (ci == c) { f |= 1 | (p->w_mask[i] < 0 ? 2 : 0); m0 = p->w_mask[i]; ++i; }
+            if (ck == c) { f |= 4 | (p->w_mask[k] < 0 ? 8 : 0); m1 = p->w_mask[k]; ++k; }
             p->u_col.push_back(c);
             p->u_flags.push_back(f);
             p->u_mask.push_back(m0);
             p->u_mask.push_back(m1);
+        }
+        // single-patch entries, each for one q-tile
+        for (int x = 0; x < 2; ++x) {
+            const int qt = t0 + x;
+            if (qt >= p->n_qt) break;
+            for (int e = p->w_row_ptr[qt] + p->w_aligned[qt]; e < p->w_row_ptr[qt + 1]; ++e) {
+                p->u_col.push_back(p->w_key[e]);
+                p->u_flags.push_back((unsigned char)(x ? 4 : 1));
+                p->u_mask.push_back(x ? -1 : p->w_mask[e]);
+                p->u_mask.push_back(x ? p->w_mask[e] : -1);
+            }
         }
         p->u_row_ptr[b + 1] = (int)p->u_col.size();
     }
@@ -357,6 +475,22 @@ extern "C" int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info) {
     info->kv_splits = p->n_split;
     info->workspace_bytes = (long long)p->ws_bytes;
     info->mask_bytes = (long long)(sizeof(uint32_t) * p->masks.size());
+    info->work_entries = (int)p->w_key.size();
+    info->single_patch_entries = p->n_diag;
+    info->work_mask_bytes = (long long)(sizeof(uint32_t) * p->kmasks.size());
+    return VDIT_OK;
+}
+
+extern "C" int vdit_plan_export_work(const vdit_plan* p, int* row_ptr, int* key_row, int* mask_index,
+                                     unsigned int* words) {
+    if (!p || !row_ptr || (!p->w_key.empty() && (!key_row || !mask_index)) || (!p->kmasks.empty() && !words))
+        return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or output");
+    std::memcpy(row_ptr, p->w_row_ptr.data(), sizeof(int) * p->w_row_ptr.size());
+    if (!p->w_key.empty()) {
+        std::memcpy(key_row, p->w_key.data(), sizeof(int) * p->w_key.size());
+        std::memcpy(mask_index, p->w_mask.data(), sizeof(int) * p->w_mask.size());
+    }
+    if (!p->kmasks.empty()) std::memcpy(words, p->kmasks.data(), sizeof(uint32_t) * p->kmasks.size());
     return VDIT_OK;
 }
 
@@ -404,7 +538,7 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t n_uf = std::max<size_t>(1, p->u_flags.size());
     const size_t n_uo = sizeof(int) * std::max<size_t>(1, p->unit_order.size());
     const size_t n_um = sizeof(int) * std::max<size_t>(1, p->u_mask.size());
-    const size_t n_mk = sizeof(uint32_t) * std::max<size_t>(4, p->masks.size());
+    const size_t n_mk = sizeof(uint32_t) * std::max<size_t>(4, p->kmasks.size());
     const size_t n_wo = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
                                              p->g.heads * p->g.head_dim : 0;
     const size_t n_wl = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads * p->q_tokens : 0;
@@ -423,7 +557,7 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t o_uf = put(p->u_flags.data(), p->u_flags.size(), n_uf);
     const size_t o_uo = put(p->unit_order.data(), sizeof(int) * p->unit_order.size(), n_uo);
     const size_t o_um = put(p->u_mask.data(), sizeof(int) * p->u_mask.size(), n_um);
-    const size_t o_mk = put(p->masks.data(), sizeof(uint32_t) * p->masks.size(), n_mk);
+    const size_t o_mk = put(p->kmasks.data(), sizeof(uint32_t) * p->kmasks.size(), n_mk);
     if (off != meta) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
     host.resize(meta);  // the workspace is not initialised: every entry is written before use
     void* d = nullptr;
