@@ -200,3 +200,28 @@ def test_seq_pack_rejects_bad_arguments():
     with pytest.raises(vdit.VditError):  # two outputs overlapping
         vdit.seq_pack(x, x, x, G13, 0, 0, 2, send,
                       (full[0], full[1], send.view(-1)[:32 * 6 * 128].view(32, 6, 128)))
+
+
+@pytest.mark.parametrize("wid", [3, 5])
+def test_rotated_forward_equals_forward_on_rotated_queries(wid):
+    # vdit_attn_forward_rotated on RoPE(q) (vdit_rope3d_apply at the plan's query positions) runs
+    # the same kernel as vdit_attn_forward on q with the rotation in the Q load: bit-identical
+    w = WORKLOADS[wid]
+    qb, kb, vb = inputs(w)
+    g = geom(w)
+    cache = vdit.KVCache(g, w.capacity_frames)
+    kd, vd = dev(kb), dev(vb)
+    ft = w.frame_tokens
+    for s, n in w.appends:
+        off = (s - w.kv_stream_first_frame) * ft
+        cache.append(kd[off:off + n * ft], vd[off:off + n * ft], s)
+    plan = vdit.Plan(g, mask(w), w.q_start, w.q_frames, cache=cache)
+    q = dev(qb)
+    la = torch.empty(w.heads, w.q_tokens, device="cuda")
+    lb = torch.empty_like(la)
+    a = vdit.attn_forward(plan, q, cache, lse=la, scale=w.scale)
+    b = vdit.attn_forward(plan, vdit.rope3d_apply(q, g, w.q_start), cache, lse=lb, scale=w.scale,
+                          q_rotated=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+    assert vdit.get_status() == vdit.OK
