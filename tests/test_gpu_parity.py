@@ -141,6 +141,41 @@ def test_attention_medium_full(name):
     _full_check(MEDIUM[name])
 
 
+def _single_patch(kind, q_start, q_frames, cap, appends, tau=0.0):
+    # 8 x 20 = 160 tokens per frame (tiles straddle frames), radius 4 >> dt: 0 from 3 frames
+    # apart (lambda 0: no long-range frames), so the plan moves those frames' same-patch pairs
+    # into single-patch entries at unaligned key rows
+    return Workload(96, "single-patch", grid_h=8, grid_w=20, heads=2, head_dim=128,
+                    bands=(44, 42, 42), mask_kind=kind, q_start=q_start, q_frames=q_frames,
+                    capacity_frames=cap, appends=appends, kv_stream_first_frame=0, chunk_frames=3,
+                    w0=4, gamma_shift=1, lam=0, tau=tau)
+
+
+SINGLE_PATCH = {
+    "radial": _single_patch(2, 0, 9, 9, ((0, 9),)),
+    # a ring of 10 holding frames 2..11 (slots 2..9, 0, 1): the queries' single-patch key frames
+    # 3..8 sit in consecutive slots
+    "causal_radial_ring": _single_patch(3, 9, 3, 10, tuple((s, 3) for s in range(0, 12, 3))),
+    "radial_odd_start": _single_patch(2, 2, 5, 8, ((0, 8),)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SINGLE_PATCH))
+def test_attention_single_patch_entries_full(name):
+    w = SINGLE_PATCH[name]
+    first, last = w.window()
+    plan = vdit.Plan(geom(w), mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                     kv_first_frame=first, kv_last_frame=last, upload=False)
+    assert plan.info["single_patch_entries"] > 0
+    _full_check(w)
+
+
+def test_attention_single_patch_entries_dynamic_threshold():
+    import dataclasses
+    w = dataclasses.replace(SINGLE_PATCH["radial"], mask_kind=6, tau=1.5)
+    _dynamic_check(w)
+
+
 @pytest.mark.parametrize("name", ["causal_radial", "dense"])
 def test_attention_sharp_softmax(name):
     # Q scaled by 4: logits of standard deviation ~4 and a peaked softmax (|o| ~ 1), where the

@@ -175,6 +175,18 @@ def test_kernel_work_list_covers_the_mask_once_workloads(wid):
         assert info["single_patch_entries"] == 0 and info["work_entries"] == info["tiles"]
 
 
+@pytest.mark.parametrize("kind,q_start,q_frames,cap,last", [(2, 0, 9, 9, 8), (3, 9, 3, 10, 11),
+                                                            (2, 2, 5, 8, 7)])
+def test_kernel_work_list_medium_single_patch_cases(kind, q_start, q_frames, cap, last):
+    # the medium geometries the GPU parity tests run in full (8 x 20 patches, radius 4 >> dt)
+    first = max(0, last - cap + 1)
+    g = vdit.Geometry(8, 20, 2, 128, (44, 42, 42))
+    plan = vdit.Plan(g, vdit.Mask(kind, 3, 4, 1, 0), q_start, q_frames, capacity_frames=cap,
+                     kv_first_frame=first, kv_last_frame=last, upload=False)
+    assert plan.info["single_patch_entries"] > 0
+    _check_work(plan, 8, 20, q_start, q_frames, cap, first, last, kind, 3, 4, 1, 0)
+
+
 def test_kernel_work_list_covers_the_mask_once_random_geometries():
     # frames of at least 128 tokens (where single-patch entries apply), rings that wrap, both
     # causal and not, radial radii that reach 0 within the window

@@ -52,11 +52,10 @@ constexpr int kGWarpTMA = 0, kGWarpMMA = 1;  // warps 2-5: epilogue
 constexpr uint32_t kOutSlab = kBM * 64 * 2;        // 16 KiB: 128 rows x 64 columns of bf16
 constexpr uint32_t kAccCols = kBN;                 // fp32 columns per accumulator
 
-
 struct GemmArgs {
     int m;              // tokens of this launch
     int k;              // d_model
-    int n_tiles_m, n_tiles_n;
+    int n_tiles_m, n_tiles_n;  // 256 x 256 output tiles (a CTA pair each)
     int n_major;        // tile order: 0 = row blocks outer (W stays in L2), 1 = column blocks outer
     int hd;             // heads * head_dim (one of the Q, K, V sections)
     int head_dim;
