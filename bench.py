@@ -357,12 +357,13 @@ def time_workload(vdit, w, dev, stream, burst_peak, n=10):
             "attn_fwd_ms": ms, "tflops": tf, "frac_of_burst_peak": tf / burst_peak,
             "kept_fraction": info["kept_pairs"] / (w.q_tokens * w.kv_tokens),
             "tiles": info["tiles"], "full_tiles": info["full_tiles"],
+            "ctas": info["ctas"], "cut_units": info["cut_units"],
             "kv_splits": info["kv_splits"],
-            "launches": 1 + (1 if info["kv_splits"] > 1 else 0),
+            "launches": 1 + (1 if info["cut_units"] > 0 else 0),
             "plan_host_ms": 1e3 * t_plan, "status": status,
             "how": "%d back-to-back launches after 3 warm-up, CUDA events; ms includes the "
-                   "split merge kernel when kv_splits > 1; TFLOP/s counts 4*d per kept pair"
-                   % n}
+                   "merge kernel of the cut units' key pieces when cut_units > 0; TFLOP/s counts "
+                   "4*d per kept pair" % n}
 
 
 def run_gpu(args, w):
@@ -645,8 +646,13 @@ def run_gpu(args, w):
                 "step": "kv_append(newest chunk) + attn_forward (RoPE of Q fused); plan built "
                         "once per geometry outside the timed region (%.1f ms host)" % (1e3 * t_plan),
                 "tiles": info["tiles"], "full_tiles": info["full_tiles"],
+                "ctas": info["ctas"], "cut_units": info["cut_units"],
                 "kept_fraction": info["kept_pairs"] / (w.q_tokens * w.kv_tokens)}),
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved,
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd",
+                         "timed": "one vdit_attn_forward call: attn_fwd_kernel, plus split_combine_kernel "
+                                  "when the CTA schedule cuts units into key pieces (%d cut units here)"
+                                  % plan.info["cut_units"],
+                         "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_kind": peak_kind,
                          "frac_of_burst_peak": achieved / pk["bf16_tflops"],
@@ -666,8 +672,8 @@ def run_gpu(args, w):
                        "query_tokens_per_s: query tokens through the whole step (append + "
                        "attention, all heads) per second; both summed over the ranks (head "
                        "shards share their query tokens)"},
-            # per step: the append, the attention kernel and, with a key split, the merge
-            "gpu_launches": args.steps * (2 + (1 if info["kv_splits"] > 1 else 0)),
+            # per step: the append, the attention kernel and, when units are cut, the merge
+            "gpu_launches": args.steps * (2 + (1 if info["cut_units"] > 0 else 0)),
             "clocks": clk,
             "kernels": {
                 "attn_fwd_ms": attn_ms, "attn_fwd_tflops": achieved,

@@ -116,14 +116,18 @@ typedef struct vdit_plan_info_t {
     int full_tiles;      /* listed tiles that are complete and wholly kept */
     long long kept_pairs;/* kept (query, key) pairs per head */
     int uploaded;        /* 1 after vdit_plan_upload */
-    int kv_splits;       /* key-range pieces per (query block, head), set by vdit_plan_upload */
-    long long workspace_bytes; /* device scratch the plan holds for kv_splits > 1 */
+    int kv_splits;       /* most key-range pieces of one (query block, head) unit in the CTA
+                            schedule (1: no unit is cut), set by vdit_plan_upload */
+    long long workspace_bytes; /* device scratch the plan holds for the pieces' partial results */
     long long mask_bytes;      /* keep masks of the partial tiles: 2 KiB per distinct block
                                   (identical blocks of several tiles are stored once; see
                                   vdit_plan_export_masks) */
     int work_entries;          /* entries of the kernel's work list (vdit_plan_export_work) */
     int single_patch_entries;  /* of which single-patch entries at unaligned key rows */
     long long work_mask_bytes; /* keep-mask blocks of the work list (2 KiB per distinct block) */
+    int ctas;                  /* CTAs of the attention launch (set by vdit_plan_upload) */
+    int cut_units;             /* (query block, head) units cut into key pieces (merged by a
+                                  second kernel; set by vdit_plan_upload) */
 } vdit_plan_info_t;
 
 /* 3-D RoPE ([CRoPE] 2.B, [TR] Metodologia 1) of n_tokens consecutive tokens of one chunk whose
@@ -166,19 +170,29 @@ VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask
                    int capacity_frames, int kv_first_frame, int kv_last_frame);
 
 /* Copies the plan's schedule and tables to the current device (allocates; the copy is ordered on
- * stream). Idempotent. Required before vdit_attn_forward. It also fixes the key-range split of
- * the forward pass from the device's SM count: when cutting each (query block, head) unit's key
- * tiles into kv_splits pieces shortens the estimated time (the CTAs' makespan over the SMs plus
- * the cost of the partial results), the pieces' normalised fp32 partial outputs and
- * log-sum-exps go to a scratch workspace held by the plan and are merged by a second kernel
- * (never in the dynamic-threshold mode, whose threshold needs each row's maximum over all its
- * candidates). Forward calls that share one plan must therefore
- * not run concurrently on different streams. */
+ * stream). Idempotent. Required before vdit_attn_forward. It also fixes the CTA schedule of the
+ * forward pass from the device's SM count (one CTA per SM at a time, launched in order, each
+ * running one query block of two 128-query tiles of one head, a "unit", over its key list):
+ * units run whole in head-major order, longest list first, except where the SMs would otherwise
+ * idle at the end of the launch; there units are cut into key pieces that fill the SMs up to one
+ * common level, found by bisection on a list-scheduling model of the launch. Each piece writes
+ * its normalised fp32 partial output and log-sum-exp into a workspace slot held by the plan, and
+ * a second kernel merges the pieces of every cut unit. The cut schedule is kept only when its
+ * estimated time (makespan plus the partial results and the extra launch) is shorter; it never
+ * uses more than 32768 / (head_dim + 1) slots (the no-allocation buffer's capacity), and the
+ * dynamic-threshold mode, whose threshold needs each row's maximum over all its candidates, is
+ * never cut. Forward calls that share one plan must therefore not run concurrently on different
+ * streams. */
 VDIT_API int vdit_plan_upload(vdit_plan* p, void* stream);
 
-/* Host only: the key split vdit_plan_upload would choose for this plan on a device with
- * sm_count SMs (the rule above), without touching any device. */
-VDIT_API int vdit_plan_split_for(const vdit_plan* p, int sm_count, int* kv_splits);
+/* Host only: the CTA schedule vdit_plan_upload would fix for this plan on a device with
+ * sm_count SMs (the rule above), without touching any device. *n_ctas and *n_cut_units receive
+ * the counts; when cta (or merge) is not NULL it receives, per CTA in launch order, 5 ints
+ * (query block, head, first entry of the piece within the unit's key list, entries, partial slot
+ * or -1 for a unit that runs whole), and per cut unit 4 ints (query block, head, first slot,
+ * pieces). Call once with NULL arrays for the sizes. */
+VDIT_API int vdit_plan_export_schedule(const vdit_plan* p, int sm_count, int* n_ctas, int* n_cut_units,
+                                       int* cta, int* merge);
 
 VDIT_API int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info);
 
@@ -233,12 +247,11 @@ VDIT_API int vdit_attn_forward_rotated(const vdit_plan* p, const void* q_rotated
  * for instance code running while another framework owns the GPU's memory through its own
  * pool (a cudaMalloc would fail or fragment it), or latency-critical loops that must not enter
  * the allocator or synchronise the device. Same arguments, results and error codes as
- * vdit_attn_forward; the difference is where the key-split scratch lives: instead of the
+ * vdit_attn_forward; the difference is where the key-piece scratch lives: instead of the
  * workspace that vdit_plan_upload gives the plan, the partial results go to one fixed 32 MiB
  * device buffer that is part of the library (every GPU that loads the library holds it until
- * the process exits). A plan whose split needs more than 32 MiB
- * (kv_splits x q_tokens x heads x (head_dim + 1) x 4 bytes) is rejected with
- * VDIT_ERR_UNSUPPORTED and a message giving both sizes; plans with kv_splits == 1 need none.
+ * the process exits). The CTA schedule never uses more partial slots than the buffer holds
+ * (256 x (head_dim + 1) x 4 bytes each), so every uploaded plan runs here.
  * The call itself makes no cudaMalloc / cudaFree or other allocating call: the plan must already
  * be uploaded, and the RoPE tables for its bands must already exist on the device (any earlier
  * vdit_kv_append, vdit_rope3d_apply or vdit_attn_forward builds them; otherwise

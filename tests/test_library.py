@@ -243,23 +243,96 @@ def test_plan_masks_bit_exact_vs_oracle_random_geometries():
         _check_masks(plan, gh, gw, q_start, q_frames, cap, first, last, kind, chunk, w0, gs, lam)
 
 
-def test_key_split_rule_picks_the_measured_best_counts():
-    """vdit_plan_upload's key split (host-only twin vdit_plan_split_for) on a 148-SM B200: on the
-    causal chunk forced splits 2 / 3 / 4 / 5 / 6 measured 1 018 / 1 133 / 1 068 / 1 088 / 1 038
-    TFLOP/s and on the 14B rollout chunk 1 / 2 / 4 measured 556 / 518 / 456, so the rule must
-    pick 3 and 1; the dense and radial shapes fill 10 waves unsplit; the dynamic threshold
-    never splits; one head of the causal chunk (19 CTAs unsplit) splits, within the 32 MiB the
-    no-allocation forward holds."""
-    def plan(w):
-        first, last = w.window()
-        return vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
-                         kv_first_frame=first, kv_last_frame=last, upload=False)
-    assert {k: plan(w).split_for(148) for k, w in WORKLOADS.items()} == {1: 1, 2: 1, 3: 3, 4: 1, 5: 1, 6: 1}
+def _plan_of(w):
+    first, last = w.window()
+    return vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                     kv_first_frame=first, kv_last_frame=last, upload=False)
+
+
+def _list_schedule_span(lengths, sms, fixed=12.0):
+    """Makespan of CTAs of the given entry counts dispatched in order, each to the SM that frees
+    first, a CTA costing its entries plus `fixed`."""
+    import heapq
+    free = [0.0] * sms
+    for n in lengths:
+        heapq.heapreplace(free, free[0] + n + fixed)
+    return max(free)
+
+
+def _check_schedule(plan, heads, sms, dynamic=False):
+    """The CTA schedule (vdit_plan_export_schedule) runs every (q-block, head) unit's union list
+    exactly once: whole (slot -1), or cut into consecutive pieces of at least 8 entries, each with
+    its own partial slot, listed once in the merge table; head-major launch order; slots within
+    the no-allocation buffer. Returns (cta, merge, unit lengths)."""
+    whole, none = plan.schedule_for(1)  # one SM: nothing to balance, every unit whole
+    assert len(none) == 0 and (whole[:, 2] == 0).all() and (whole[:, 4] == -1).all()
+    length = {(int(r[0]), int(r[1])): int(r[3]) for r in whole}
+    assert len(length) == len(whole) == plan.info["q_tiles"] // 2 * heads + (plan.info["q_tiles"] % 2) * heads
+    cta, merge = plan.schedule_for(sms)
+    assert (np.diff(cta[:, 1]) >= 0).all()                      # head-major
+    pieces = {}
+    for qb, hd, e0, n, slot in cta.tolist():
+        pieces.setdefault((qb, hd), []).append((e0, n, slot))
+    assert set(pieces) == set(length)
+    slots = sorted(int(x) for x in cta[:, 4] if x >= 0)
+    assert slots == list(range(len(slots)))                     # each slot used once
+    assert len(slots) <= 32768 // (plan.g.head_dim + 1)
+    cut = {(int(r[0]), int(r[1])): (int(r[2]), int(r[3])) for r in merge}
+    assert len(cut) == len(merge)
+    for u, ps in pieces.items():
+        if len(ps) == 1 and u not in cut:
+            assert ps[0] == (0, length[u], -1), u
+            continue
+        first, k = cut[u]
+        assert k == len(ps) >= 2, u
+        assert [p[2] for p in ps] == list(range(first, first + k)), u
+        at = 0
+        for e0, n, _ in ps:
+            assert e0 == at and n >= 8, u
+            at += n
+        assert at == length[u], u
+    if dynamic:
+        assert len(merge) == 0
+    return cta, merge, length
+
+
+@pytest.mark.parametrize("wid", sorted(WORKLOADS))
+def test_cta_schedule_covers_every_unit_once(wid):
+    w = WORKLOADS[wid]
+    plan = _plan_of(w)
+    for sms in (148, 7, 1000):
+        _check_schedule(plan, w.heads, sms, dynamic=bool(w.mask_kind & 4))
+
+
+def test_cta_schedule_shortens_the_modelled_launch():
+    """On a 148-SM B200 the cut schedule fills the last wave: the modelled makespan of the
+    exported CTA table (list scheduling in launch order) is well below the whole-unit one on the
+    dense, causal-chunk and 14B-rollout shapes (1 536, 228 and 760 units: 10.4, 1.5 and 5.1
+    waves) and never above it; the dynamic threshold never cuts; one head of the causal chunk
+    (19 units) is cut over the SMs."""
+    for wid, gain in ((2, 0.04), (3, 0.10), (4, 0.0), (5, 0.05), (6, 0.0)):
+        w = WORKLOADS[wid]
+        plan = _plan_of(w)
+        cta, merge, length = _check_schedule(plan, w.heads, 148, dynamic=bool(w.mask_kind & 4))
+        whole, _ = plan.schedule_for(1)
+        t_whole = _list_schedule_span(whole[:, 3], 148)
+        t_cut = _list_schedule_span(cta[:, 3], 148)
+        assert t_cut <= t_whole * (1 - gain), (wid, t_cut, t_whole)
+        if w.mask_kind & 4:
+            assert len(merge) == 0 and len(cta) == len(whole)
+    # query blocks with empty lists (chunk 0 against a cache holding only frame 3) run whole
+    for q_start, q_frames in ((0, 1), (2, 2)):
+        empty = Workload(93, "no-keys", grid_h=6, grid_w=10, heads=2, head_dim=128, bands=(44, 42, 42),
+                         mask_kind=1, q_start=q_start, q_frames=q_frames, capacity_frames=4,
+                         appends=((3, 1),), kv_stream_first_frame=3, chunk_frames=3)
+        for sms in (1, 2, 148):
+            cta, merge, length = _check_schedule(_plan_of(empty), 2, sms)
+            assert len(cta) == len(length) and len(merge) == 0
     one = Workload(**{**WORKLOADS[3].__dict__, "id": 95, "heads": 1})
-    sp = plan(one).split_for(148)
-    assert sp > 1 and sp * one.q_tokens * (one.head_dim + 1) * 4 <= 32 << 20
+    cta, merge, _ = _check_schedule(_plan_of(one), 1, 148)
+    assert len(merge) == len(_plan_of(one).schedule_for(1)[0]) and len(cta) > 100
     with pytest.raises(vdit.VditError):
-        plan(one).split_for(0)
+        _plan_of(one).schedule_for(0)
 
 
 def test_plan_rejects_bad_arguments():

@@ -4,8 +4,8 @@ kernels run on the same plan) and against the fp64 oracle.
 
 It exists for callers that cannot allocate device memory when they run attention (another
 framework owns the GPU's memory through its own pool, or a latency-critical loop must not enter
-the allocator): its key-split partial results go to a fixed device buffer inside the library
-instead of the workspace the plan allocates. This file is collected last so that a run that
+the allocator): the partial results of the key pieces of its cut units go to a fixed device buffer
+inside the library instead of the workspace the plan allocates. This file is collected last so that a run that
 stops at the first failure has already run every other test; it also passes on its own in a
 fresh process (it builds everything it needs, including the RoPE tables, before the call).
 """
@@ -50,14 +50,13 @@ def _call(fn, plan, q, cache, w):
 
 def test_noalloc_forward_matches_forward_twice_in_a_row():
     # one head of the causal-chunk shape: 19 query blocks x 1 head leave most SMs idle, so the
-    # plan splits every unit's key tiles and the scratch path is the one exercised
+    # schedule cuts every unit into key pieces and the scratch path is the one exercised
     base = WORKLOADS[3]
     w = Workload(**{**base.__dict__, "id": 95, "heads": 1})
     q, cache, plan = _setup(w)
     info = plan.info
-    assert info["kv_splits"] > 1
-    needed = info["kv_splits"] * w.q_tokens * w.heads * (w.head_dim + 1) * 4
-    assert needed <= 32 << 20
+    assert info["kv_splits"] > 1 and info["cut_units"] == 19
+    assert 0 < info["workspace_bytes"] <= 32 << 20
     L = vdit.lib()
     rc, o_ref, lse_ref = _call(L.vdit_attn_forward, plan, q, cache, w)
     assert rc == vdit.OK
@@ -83,13 +82,17 @@ def test_noalloc_forward_matches_forward_twice_in_a_row():
     assert np.max(np.abs(lse[0][rows].cpu().numpy() - rl[0])) < 2e-2
 
 
-def test_noalloc_forward_rejects_a_split_larger_than_its_buffer():
-    w = WORKLOADS[3]  # 12 heads: the split workspace is tens of MB
+def test_noalloc_forward_runs_the_full_causal_chunk():
+    # all 12 heads of the causal-chunk shape: the schedule cuts units into key pieces, and their
+    # partial slots stay within the fixed buffer, so the call runs and matches vdit_attn_forward
+    w = WORKLOADS[3]
     q, cache, plan = _setup(w)
-    if plan.info["kv_splits"] == 1:
-        pytest.skip("this device needs no key split for this shape")
+    info = plan.info
+    assert 0 < info["workspace_bytes"] <= 32 << 20
     L = vdit.lib()
-    rc, _, _ = _call(L.vdit_attn_forward_noalloc, plan, q, cache, w)
-    assert rc == vdit.ERR_UNSUPPORTED
-    msg = L.vdit_last_error().decode()
-    assert "scratch" in msg and str(32 << 20) in msg
+    rc, o_ref, lse_ref = _call(L.vdit_attn_forward, plan, q, cache, w)
+    assert rc == vdit.OK
+    rc, o, lse = _call(L.vdit_attn_forward_noalloc, plan, q, cache, w)
+    assert rc == vdit.OK, L.vdit_last_error()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    assert vdit.get_status() == vdit.OK

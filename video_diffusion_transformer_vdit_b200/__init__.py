@@ -65,7 +65,8 @@ class _PlanInfo(ctypes.Structure):
                 ("kept_pairs", ctypes.c_longlong), ("uploaded", ctypes.c_int),
                 ("kv_splits", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong),
                 ("mask_bytes", ctypes.c_longlong), ("work_entries", ctypes.c_int),
-                ("single_patch_entries", ctypes.c_int), ("work_mask_bytes", ctypes.c_longlong)]
+                ("single_patch_entries", ctypes.c_int), ("work_mask_bytes", ctypes.c_longlong),
+                ("ctas", ctypes.c_int), ("cut_units", ctypes.c_int)]
 
 
 _lib = None
@@ -89,7 +90,7 @@ def lib() -> ctypes.CDLL:
         L.vdit_plan_export.argtypes = [P, P, P, P]
         L.vdit_plan_export_masks.argtypes = [P, P, P]
         L.vdit_plan_export_work.argtypes = [P, P, P, P, P]
-        L.vdit_plan_split_for.argtypes = [P, I, ctypes.POINTER(I)]
+        L.vdit_plan_export_schedule.argtypes = [P, I, ctypes.POINTER(I), ctypes.POINTER(I), P, P]
         L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
         L.vdit_seq_pack.argtypes = [gp, P, P, P, P, P, P, P, I, I, I, LL, I, P]
         L.vdit_seq_unpack.argtypes = [gp, P, P, P, I, I, LL, P]
@@ -517,11 +518,20 @@ class Plan:
         n = inf["work_entries"]
         return rp, kr[:n], mi[:n], words[:inf["work_mask_bytes"] // 4].reshape(-1, 128, 4)
 
-    def split_for(self, sm_count: int) -> int:
-        """The key split vdit_plan_upload would choose on a device with sm_count SMs."""
-        out = ctypes.c_int()
-        _check(lib().vdit_plan_split_for(self._h, int(sm_count), ctypes.byref(out)))
-        return out.value
+    def schedule_for(self, sm_count: int):
+        """The CTA schedule vdit_plan_upload would fix on a device with sm_count SMs
+        (vdit_plan_export_schedule): (cta [ctas, 5]: q-block, head, first entry, entries, slot or
+        -1; merge [cut units, 4]: q-block, head, first slot, pieces) as numpy int32 arrays."""
+        import numpy as np
+        n_cta, n_cut = ctypes.c_int(), ctypes.c_int()
+        _check(lib().vdit_plan_export_schedule(self._h, int(sm_count), ctypes.byref(n_cta),
+                                               ctypes.byref(n_cut), None, None))
+        cta = np.zeros((max(1, n_cta.value), 5), np.int32)
+        merge = np.zeros((max(1, n_cut.value), 4), np.int32)
+        _check(lib().vdit_plan_export_schedule(self._h, int(sm_count), ctypes.byref(n_cta),
+                                               ctypes.byref(n_cut), ctypes.c_void_p(cta.ctypes.data),
+                                               ctypes.c_void_p(merge.ctypes.data)))
+        return cta[:n_cta.value], merge[:n_cut.value]
 
     def flops(self) -> float:
         """Unmasked-entry FLOPs of one forward: 4 * head_dim per kept (query, key, head)."""

@@ -114,10 +114,10 @@ struct AttnArgs {
     const int* u_col;      // first key row of each entry (a multiple of 128, or the unaligned
                            // row of a single-patch entry)
     const unsigned char* u_flags;
-    const int* unit_order; // q-blocks, longest list first
-    float* ws_o;           // split > 1: normalised partial O [split][q_tokens][heads][D]
-    float* ws_lse;         // split > 1: partial log2-sum-exp [split][heads][q_tokens]
-    int n_qb, n_split;
+    const int* cta;        // per CTA, 4 ints: q-block, head, first union entry of its piece, entries
+    const int* cta_slot;   // per CTA: partial slot of a piece of a cut unit, or -1
+    float* ws_o;           // normalised partial O of the pieces [slot][256 query rows][D]
+    float* ws_lse;         // their log2-sum-exp [slot][256 query rows]
     const uint32_t* masks; // keep-mask blocks of the partial tiles (2 KiB each)
     const int* u_mask;     // per union entry and query tile: mask block, or -1
     const uint4* q;
@@ -189,15 +189,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // work unit: q-block (longest lists first), head, and the piece `sp` of its key tiles
-    const int unit = blockIdx.x, head = blockIdx.y;
-    const int sp = unit / a.n_qb;
-    const int qb = __ldg(a.unit_order + (unit - sp * a.n_qb));
-    const int u_first = __ldg(a.u_row_ptr + qb);
-    const int n_all = __ldg(a.u_row_ptr + qb + 1) - u_first;
-    const int e0 = (int)((long long)n_all * sp / a.n_split);
-    const int u_begin = u_first + e0;
-    const int n_ent = (int)((long long)n_all * (sp + 1) / a.n_split) - e0;
+    // work of this CTA (the plan's schedule): q-block, head and a piece of the union list, whole
+    // or cut; a piece of a cut unit writes partial results into its slot
+    // (scalar loads: a 16-byte vector load here costs the kernel register spills)
+    const int* work = a.cta + 4 * blockIdx.x;
+    const int qb = __ldg(work), head = __ldg(work + 1);
+    const int u_begin = __ldg(a.u_row_ptr + qb) + __ldg(work + 2);
+    const int n_ent = __ldg(work + 3);
+    const int unit = blockIdx.x;
     // Every CTA walks its key tiles starting at a different position (the online softmax does
     // not depend on the order): CTAs of one head run concurrently, and starting them all at the
     // same tile makes them request the same 32 KiB of K / V from the same L2 slices at once.
@@ -264,7 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_p = tmem + kTmemP + 64u * h + lane_base;
         const uint32_t t_o = tmem + kTmemO + 128u * h + lane_base;
         const uint32_t f_in = h ? 4u : 1u, f_full = h ? 8u : 2u;
-        const int qi = (qb * kQTiles + h) * kTile + row;
         const float c = a.scale_log2;
         float m = -INFINITY, l = 0.f;  // running max (raw score units) and sum
         int cnt = 0;                   // score tiles read
@@ -408,12 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             : "=r"(any_fail)
             : "r"((uint32_t)ok), "r"(1 + h)
             : "memory");
-        if (!any_fail && a.n_split > 1) {
+        // the CTA's slot, q-block and head, read again here rather than kept live through the
+        // loop (the softmax warps are short of registers)
+        const int slot = __ldg(a.cta_slot + blockIdx.x);
+        const int qb_e = __ldg(a.cta + 4 * blockIdx.x), head_e = __ldg(a.cta + 4 * blockIdx.x + 1);
+        const int qi = (qb_e * kQTiles + h) * kTile + row;
+        if (!any_fail && slot >= 0) {
             // partial result of this key piece: O / l in fp32 and log2(sum) for the merge
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            float4* dst = reinterpret_cast<float4*>(
-                a.ws_o + (((size_t)sp * a.q_tokens + (qi < a.q_tokens ? qi : 0)) * a.heads + head) * D);
+            const size_t prow = (size_t)slot * (kQTiles * kTile) + h * kTile + row;
+            float4* dst = reinterpret_cast<float4*>(a.ws_o + prow * D);
 #pragma unroll 1
             for (int q4 = 0; q4 < D / 32; ++q4) {
                 uint32_t orow[32];
@@ -433,9 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                       __uint_as_float(orow[4 * g + 3]) * inv_l);
                 }
             }
-            if (qi < a.q_tokens)
-                a.ws_lse[((size_t)sp * a.heads + head) * a.q_tokens + qi] =
-                    l > 0.f ? m * c + log2f(l) : -INFINITY;
+            if (qi < a.q_tokens) a.ws_lse[prow] = l > 0.f ? m * c + log2f(l) : -INFINITY;
         } else if (!any_fail) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -466,17 +467,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (a.lse && qi < a.q_tokens)
-                a.lse[(size_t)head * a.q_tokens + qi] =
+                a.lse[(size_t)head_e * a.q_tokens + qi] =
                     l > 0.f ? (m * c + log2f(l)) * 0.6931471805599453f : -INFINITY;
             asm volatile("bar.sync %0, 128;" ::"r"(3 + h) : "memory");
-            const int q0 = (qb * kQTiles + h) * kTile;
+            const int q0 = (qb_e * kQTiles + h) * kTile;
 #pragma unroll 4
             for (int i = 0; i < kC16; ++i) {
                 const int r = i * (128 / kC16) + row / kC16, chunk = row % kC16;
                 if (q0 + r < a.q_tokens) {
                     const uint4 v = *reinterpret_cast<const uint4*>(stage + r * (D * 2) +
                                                                     ((chunk ^ (r & 7)) << 4));
-                    __stcs(a.o + ((size_t)(q0 + r) * a.heads + head) * kC16 + chunk, v);
+                    __stcs(a.o + ((size_t)(q0 + r) * a.heads + head_e) * kC16 + chunk, v);
                 }
             }
         }
@@ -697,36 +698,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Merge of the key pieces of every (query, head) row: with piece i holding O_i = (sum over its
-// keys of p v) / l_i and L_i = log2 l_i (in the shared log2 units of the scaled scores),
+// Merge of the key pieces of every cut unit's (query, head) rows: with piece i holding
+// O_i = (sum over its keys of p v) / l_i and L_i = log2 l_i (in the shared log2 units of the
+// scaled scores),
 //   L = log2 sum_i 2^L_i,   o = sum_i 2^(L_i - L) O_i,   lse = L ln 2.
-// One warp per row; each lane owns D / 32 consecutive channels.
+// merge[4 j ..] = q-block, head, first slot, pieces of cut unit j; its 256 query rows are rows
+// 256 j .. 256 j + 255 of the grid-stride loop. One warp per row; each lane owns D / 32
+// consecutive channels.
 template <int D>
 __global__ void __launch_bounds__(256) split_combine_kernel(const float* __restrict__ ws_o,
                                                             const float* __restrict__ ws_lse,
-                                                            int n_split, int q_tokens, int heads,
+                                                            const int4* __restrict__ merge, int n_cut,
+                                                            int q_tokens, int heads,
                                                             __nv_bfloat16* __restrict__ o,
                                                             float* __restrict__ lse) {
-    constexpr int kPer = D / 32;
-    const long long rows = (long long)q_tokens * heads;
+    constexpr int kPer = D / 32, kRows = kQTiles * kTile;
+    const long long rows = (long long)n_cut * kRows;
     const long long n_warps = (long long)gridDim.x * (blockDim.x / 32);
     const int lane = threadIdx.x & 31;
     for (long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; row < rows;
          row += n_warps) {
-        const int qi = (int)(row / heads), hd = (int)(row - (long long)qi * heads);
+        const int j = (int)(row / kRows), r = (int)(row - (long long)j * kRows);
+        const int4 mu = __ldg(merge + j);
+        const int qi = mu.x * kRows + r, hd = mu.y;
+        if (qi >= q_tokens) continue;
+        const size_t first = (size_t)mu.z * kRows + r;  // partial row of piece 0
         float lmax = -INFINITY;
-        for (int i = 0; i < n_split; ++i)
-            lmax = fmaxf(lmax, __ldg(ws_lse + ((size_t)i * heads + hd) * q_tokens + qi));
+        for (int i = 0; i < mu.w; ++i) lmax = fmaxf(lmax, __ldg(ws_lse + first + (size_t)i * kRows));
         float acc[kPer];
 #pragma unroll
         for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
         float wsum = 0.f;
         if (lmax != -INFINITY) {
-            for (int i = 0; i < n_split; ++i) {
-                const float li = __ldg(ws_lse + ((size_t)i * heads + hd) * q_tokens + qi);
-                const float w = exp2f(li - lmax);
+            for (int i = 0; i < mu.w; ++i) {
+                const size_t prow = first + (size_t)i * kRows;
+                const float w = exp2f(__ldg(ws_lse + prow) - lmax);
                 wsum += w;
-                const float* src = ws_o + (((size_t)i * q_tokens + qi) * heads + hd) * D + lane * kPer;
+                const float* src = ws_o + prow * D + lane * kPer;
 #pragma unroll
                 for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, __ldg(src + e), acc[e]);
             }
@@ -793,8 +801,7 @@ DeviceState g_dev[kMaxDevices];
 
 }  // namespace
 // the no-allocation scratch buffer (its declaration and rules are with the entry point below)
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[vdit::kNoAllocScratchBytes];
 namespace {
 
 int device_state(int dev, const DeviceState** out) {
@@ -829,8 +836,8 @@ int device_state(int dev, const DeviceState** out) {
 }
 
 // Tensor maps, arguments and launches of one forward pass (the attention kernel for the plan's
-// head_dim and mode, then the split merge when the plan splits key ranges). ws_o / ws_lse: the
-// split scratch (unused without a split).
+// head_dim and mode over the plan's CTA table, then the merge when the schedule cuts units into
+// key pieces). ws_o / ws_lse: the pieces' scratch (unused when no unit is cut).
 int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, const void* v_cache,
                      void* o, float* lse, float scale, float* ws_o, float* ws_lse,
                      const vdit::RopeTables& tabs, cudaStream_t st, int dev, bool q_rotated = false) {
@@ -846,11 +853,10 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     a.u_row_ptr = p->d_u_row_ptr;
     a.u_col = p->d_u_col;
     a.u_flags = p->d_u_flags;
-    a.unit_order = p->d_unit_order;
+    a.cta = p->d_cta;
+    a.cta_slot = p->d_cta_slot;
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
-    a.n_qb = p->n_qb;
-    a.n_split = p->n_split;
     a.masks = p->d_masks;
     a.u_mask = p->d_u_mask;
     a.q = static_cast<const uint4*>(q);
@@ -874,7 +880,9 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
     a.tau_log2 = (float)(p->m.tau * 1.4426950408889634);
     const bool dyn = p->m.kind & VDIT_MASK_DYNAMIC;
-    const dim3 grid((unsigned)(p->n_qb * p->n_split), (unsigned)p->g.heads);
+    const int n_cta = (int)(p->cta.size() / 5), n_cut = (int)(p->merge.size() / 4);
+    if (n_cta == 0) return VDIT_OK;
+    const dim3 grid((unsigned)n_cta);
     if (d == 128 && !dyn)
         attn_fwd_kernel<128, false><<<grid, kThreads, Layout<128>::kSmemBytes, st>>>(mk, mv, a);
     else if (d == 64 && !dyn)
@@ -884,15 +892,16 @@ int launch_attention(const vdit_plan* p, const void* q, const void* k_cache, con
     else
         attn_fwd_kernel<64, true><<<grid, kThreads, Layout<64>::kSmemBytes, st>>>(mk, mv, a);
     if (int rc = vdit::cuda_check(cudaGetLastError(), "attention kernel launch")) return rc;
-    if (p->n_split > 1) {
-        const long long rows = (long long)p->q_tokens * p->g.heads;
+    if (n_cut > 0) {
+        const long long rows = (long long)n_cut * kQTiles * kTile;
         const int blocks = (int)std::min<long long>((rows + 7) / 8, (long long)ds->sms * 8);
         auto* ob = static_cast<__nv_bfloat16*>(o);
+        const int4* mg = reinterpret_cast<const int4*>(p->d_merge);
         if (d == 128)
-            split_combine_kernel<128><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
+            split_combine_kernel<128><<<blocks, 256, 0, st>>>(ws_o, ws_lse, mg, n_cut, p->q_tokens,
                                                               p->g.heads, ob, lse);
         else
-            split_combine_kernel<64><<<blocks, 256, 0, st>>>(ws_o, ws_lse, p->n_split, p->q_tokens,
+            split_combine_kernel<64><<<blocks, 256, 0, st>>>(ws_o, ws_lse, mg, n_cut, p->q_tokens,
                                                              p->g.heads, ob, lse);
         return vdit::cuda_check(cudaGetLastError(), "split merge launch");
     }
@@ -991,28 +1000,24 @@ extern "C" int vdit_attn_forward_noalloc(const vdit_plan* p, const void* q, cons
     int dev = 0;
     if (int rc = vdit::cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
     if (dev != p->device) return fail(VDIT_ERR_INVALID_ARG, "plan was uploaded to another device");
-    // scratch this plan's key split needs: partial O [split][q][heads][d] fp32, then partial
-    // log2-sum-exp [split][heads][q] fp32 at the next 256-byte boundary
+    // scratch this plan's key pieces need: partial O [slot][256][d] fp32, then partial
+    // log2-sum-exp [slot][256] fp32 (the schedule keeps the slots within the buffer)
     const int d = p->g.head_dim;
-    const size_t o_bytes = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
-                                                p->g.heads * d : 0;
-    const size_t o_bytes_al = (o_bytes + 255) / 256 * 256;
-    const size_t l_bytes = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads *
-                                                p->q_tokens : 0;
-    if (o_bytes_al + l_bytes > kNoAllocScratchBytes)
+    const size_t o_bytes = sizeof(float) * (size_t)p->n_slots * kQTiles * kTile * d;
+    const size_t l_bytes = sizeof(float) * (size_t)p->n_slots * kQTiles * kTile;
+    if (o_bytes + l_bytes > vdit::kNoAllocScratchBytes)
         return fail(VDIT_ERR_UNSUPPORTED,
-                    "this plan's key split needs " + std::to_string(o_bytes_al + l_bytes) +
-                        " bytes of scratch; the no-allocation variant's static buffer holds " +
-                        std::to_string(kNoAllocScratchBytes) + " (use vdit_attn_forward)");
+                    "internal: this plan's key pieces need " + std::to_string(o_bytes + l_bytes) +
+                        " bytes of scratch; the no-allocation buffer holds " +
+                        std::to_string(vdit::kNoAllocScratchBytes));
     const DeviceState* ds = nullptr;
     if (int rc = device_state(dev, &ds)) return rc;
     void* scratch = ds->noalloc;
     vdit::RopeTables tabs;
     if (int rc = vdit::find_rope_tables(&p->g, &tabs)) return rc;
-    float* ws_o = p->n_split > 1 ? static_cast<float*>(scratch) : nullptr;
-    float* ws_lse = p->n_split > 1
-                        ? reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + o_bytes_al)
-                        : nullptr;
+    float* ws_o = p->n_slots ? static_cast<float*>(scratch) : nullptr;
+    float* ws_lse = p->n_slots ? reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + o_bytes)
+                               : nullptr;
     return launch_attention(p, q, k_cache, v_cache, o, lse, scale, ws_o, ws_lse, tabs,
                             static_cast<cudaStream_t>(stream), dev);
 }

@@ -33,6 +33,14 @@ int find_rope_tables(const vdit_geom* g, RopeTables* out);
 // Reads and clears the device status word of the fused QKV projection kernel.
 int qkv_status_take(int* out);
 
+// Size of the attention module's fixed no-allocation scratch buffer, and the number of key-piece
+// partial results (256 query rows x (head_dim + 1) fp32 each: normalised O and log2-sum-exp) that
+// it holds. The schedule never uses more slots than this, so every plan fits the buffer.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr int max_partial_slots(int head_dim) {
+    return (int)(kNoAllocScratchBytes / (256u * 4u * (size_t)(head_dim + 1)));
+}
+
 // One-time set-up of the attention kernels on device dev (current): shared-memory opt-in of every
 // kernel instance, device addresses of the status word and of the no-allocation scratch buffer.
 int attn_prepare_device(int dev);
@@ -76,19 +84,26 @@ struct vdit_plan {
     std::vector<int> w_aligned;   // per q-tile: its first w_aligned[qt] entries are aligned tiles
     std::vector<uint32_t> kmasks;
     int n_diag = 0;               // entries of the single-patch kind
-    // key-range split of every (q-block, head) unit, chosen at upload from the SM count so the
-    // number of CTAs fills whole waves; > 1 uses the fp32 partial workspace below
-    int n_split = 1;
+    // CTA schedule of the attention kernel, fixed at upload from the device's SM count:
+    //   cta[5 i ..]: q-block, head, first union entry of the piece (within the unit), entries,
+    //                partial slot (-1: the unit runs whole and writes O itself);
+    //   merge[4 j ..]: a unit cut into pieces: q-block, head, first slot, pieces (slots
+    //                  first .. first + pieces - 1, merged by the second kernel).
+    std::vector<int> cta, merge;
+    int n_slots = 0;
+    int n_split = 1;  // most pieces of one unit
     // device copy
     int device = -1;
     void* d_buf = nullptr;
     const int* d_u_row_ptr = nullptr;
     const int* d_u_col = nullptr;
     const unsigned char* d_u_flags = nullptr;
-    const int* d_unit_order = nullptr;
+    const int* d_cta = nullptr;        // int4 per CTA: q-block, head, first entry, entries
+    const int* d_cta_slot = nullptr;   // per CTA: partial slot or -1
+    const int* d_merge = nullptr;      // int4 per cut unit: q-block, head, first slot, pieces
     const uint32_t* d_masks = nullptr;
     const int* d_u_mask = nullptr;
-    float* d_ws_o = nullptr;    // [n_split][q_tokens][heads][head_dim] normalised partial O
-    float* d_ws_lse = nullptr;  // [n_split][heads][q_tokens] partial log2-sum-exp
+    float* d_ws_o = nullptr;    // [slots][256 query rows][head_dim] normalised partial O
+    float* d_ws_lse = nullptr;  // [slots][256 query rows] partial log2-sum-exp
     size_t ws_bytes = 0;
 };

@@ -412,53 +412,139 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
 
 namespace {
 
-// Key-range split of every (q-block, head) unit for a device with `sms` SMs: the count (1 .. 8,
-// at least 8 key tiles a piece) with the least estimated time. The attention kernel's time is
-// the makespan of its CTAs, dispatched in launch order (per head, piece-major, units longest
-// first) each to the SM that frees first, a CTA costing its key tiles plus kPieceTiles for its
-// prologue, pipeline fill and epilogue; a split adds its fp32 partial results, written and read
-// back by the merge. Constants measured on a B200 (one CTA per SM runs a union-list entry of two
-// 128-query tiles in ~1.44 us); they reproduce the measured order of split counts on the causal
-// chunk (3 best, then 5, 4, 6, 2) and on the 14B rollout chunk (1, then 2, then 4).
-int choose_split(const vdit_plan& p, int sms) {
-    constexpr double kPieceTiles = 12.0, kTileSeconds = 1.44e-6, kBytesPerSecond = 6.5e12;
-    int max_len = 0;
-    for (int b = 0; b < p.n_qb; ++b) max_len = std::max(max_len, p.u_row_ptr[b + 1] - p.u_row_ptr[b]);
-    int best = 1;
-    double best_t = 0.0;
-    // the dynamic threshold needs each row's maximum over all its candidates: no key split
-    const int max_split = (p.m.kind & VDIT_MASK_DYNAMIC) ? 1 : 8;
-    std::vector<double> sm_free;
-    for (int sp = 1; sp <= max_split; ++sp) {
-        if (sp > 1 && max_len / sp < 8) break;
-        sm_free.assign(std::max(1, sms), 0.0);
-        std::make_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
-        double span = 0.0;
-        for (int h = 0; h < p.g.heads; ++h)
-            for (int piece = 0; piece < sp; ++piece)
-                for (int i = 0; i < p.n_qb; ++i) {
-                    const int u = p.unit_order[i];
-                    const long long n = p.u_row_ptr[u + 1] - p.u_row_ptr[u];
-                    const double cost = (double)(n * (piece + 1) / sp - n * piece / sp) + kPieceTiles;
-                    std::pop_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
-                    sm_free.back() += cost;
-                    span = std::max(span, sm_free.back());
-                    std::push_heap(sm_free.begin(), sm_free.end(), std::greater<double>());
-                }
-        double t = span * kTileSeconds;
-        if (sp > 1)
-            t += 2.0 * sp * (double)p.q_tokens * p.g.heads * (p.g.head_dim + 1) * 4.0 / kBytesPerSecond;
-        if (sp == 1 || t < best_t) { best_t = t; best = sp; }
+// CTA schedule of the attention kernel on a device with `sms` SMs, one CTA per SM at a time.
+// A unit is one q-block (two 128-query tiles) of one head with its union list of n entries; the
+// CTAs go out in launch order, each to the SM that frees first, so the kernel's time is the
+// makespan of that list schedule. A CTA costs its entries plus kPieceTiles (prologue: Q load and
+// RoPE, TMEM allocation, pipeline fill; epilogue: O write). Units go in head-major order (the
+// CTAs in flight then share few heads' K / V in L2), longest list first within a head.
+//
+// Whole units alone leave the SMs idle at the end (1 536 equal units over 148 SMs: 10.4 waves,
+// the last 38% full). So the schedule picks a level T and walks the units in order: a unit that
+// ends by T on the first free SM runs whole; one that does not is cut into pieces (each at least
+// kMinPiece entries), each piece filling the SM that frees next up to T. A piece writes its
+// normalised partial O and log2-sum-exp in fp32 into a slot of the workspace, and a second
+// kernel merges the pieces of every cut unit. The level is the smallest T (binary search) at
+// which every unit fits within kMaxSlots partial slots; the split schedule is kept when its
+// estimated time (makespan plus the partial results written and read back, plus one launch) is
+// below the whole-unit schedule's. The dynamic-threshold mode never cuts: its threshold needs
+// each row's maximum over all its candidates. Constants measured on a B200 (one CTA runs a union
+// entry of two 128-query tiles in ~1.44 us, ~12 entries' worth of fixed cost per CTA).
+struct Schedule {
+    std::vector<int> cta;    // per CTA: q-block, head, first entry (within the unit), entries, slot
+    std::vector<int> merge;  // per cut unit: q-block, head, first slot, pieces
+    int slots = 0, max_pieces = 1;
+    double span = 0.0;       // makespan, in entry times
+};
+
+constexpr double kPieceTiles = 12.0, kTileSeconds = 1.44e-6, kBytesPerSecond = 6.5e12,
+                 kLaunchSeconds = 4e-6;
+constexpr int kMinPiece = 8;
+
+// List schedule at level T (T <= 0: whole units only). false if some unit cannot be placed by
+// the rule (a cut unit needs more than max_slots slots, or the first free SM has no room left
+// for a piece).
+bool schedule_at(const vdit_plan& p, int sms, double T, int max_slots, Schedule* out) {
+    std::vector<double> f(std::max(1, sms), 0.0);  // min-heap of the SMs' free times
+    auto less = std::greater<double>();
+    Schedule s;
+    s.cta.reserve(5 * (size_t)p.n_qb * p.g.heads);
+    for (int h = 0; h < p.g.heads; ++h)
+        for (int i = 0; i < p.n_qb; ++i) {
+            const int u = p.unit_order[i];
+            const int n = p.u_row_ptr[u + 1] - p.u_row_ptr[u];
+            std::pop_heap(f.begin(), f.end(), less);
+            double& t = f.back();
+            // whole: when it ends by T, or is too short to cut (an empty list included; its CTA
+            // still writes o = 0 and lse = -inf)
+            if (T <= 0.0 || t + n + kPieceTiles <= T || n < 2 * kMinPiece) {
+                t += n + kPieceTiles;
+                s.span = std::max(s.span, t);
+                std::push_heap(f.begin(), f.end(), less);
+                s.cta.insert(s.cta.end(), {u, h, 0, n, -1});
+                continue;
+            }
+            std::push_heap(f.begin(), f.end(), less);
+            const int first_slot = s.slots;
+            int done = 0, pieces = 0;
+            while (done < n) {
+                std::pop_heap(f.begin(), f.end(), less);
+                double& tf = f.back();
+                const int rem = n - done;
+                const double room = T - tf - kPieceTiles;
+                int take;
+                if (room >= rem) take = rem;                                   // the rest fits
+                else if (room >= kMinPiece && rem >= 2 * kMinPiece)
+                    take = std::min((int)room, rem - kMinPiece);               // leave >= kMinPiece
+                else return false;
+                if (s.slots >= max_slots) return false;
+                tf += take + kPieceTiles;
+                s.span = std::max(s.span, tf);
+                std::push_heap(f.begin(), f.end(), less);
+                s.cta.insert(s.cta.end(), {u, h, done, take, s.slots++});
+                done += take;
+                ++pieces;
+            }
+            if (pieces == 1) {  // the whole unit fitted after all: no partial result needed
+                --s.slots;
+                s.cta.back() = -1;
+            } else {
+                s.merge.insert(s.merge.end(), {u, h, first_slot, pieces});
+                s.max_pieces = std::max(s.max_pieces, pieces);
+            }
+        }
+    *out = std::move(s);
+    return true;
+}
+
+double schedule_seconds(const vdit_plan& p, const Schedule& s) {
+    double t = s.span * kTileSeconds;
+    if (s.slots > 0)
+        t += 2.0 * s.slots * 256.0 * (p.g.head_dim + 1) * 4.0 / kBytesPerSecond + kLaunchSeconds;
+    return t;
+}
+
+Schedule build_schedule(const vdit_plan& p, int sms) {
+    Schedule whole;
+    schedule_at(p, sms, 0.0, 0, &whole);
+    if (p.m.kind & VDIT_MASK_DYNAMIC) return whole;
+    double work = 0.0;
+    for (int b = 0; b < p.n_qb; ++b) work += p.u_row_ptr[b + 1] - p.u_row_ptr[b] + kPieceTiles;
+    double lo = work * p.g.heads / std::max(1, sms), hi = whole.span;
+    const int max_slots = vdit::max_partial_slots(p.g.head_dim);
+    Schedule best = whole, s;
+    double best_t = schedule_seconds(p, whole);
+    for (int it = 0; it < 40 && hi - lo > 0.5; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (schedule_at(p, sms, mid, max_slots, &s)) {
+            hi = mid;
+            const double t = schedule_seconds(p, s);
+            if (t < best_t) { best_t = t; best = std::move(s); }
+        } else {
+            lo = mid;
+        }
     }
     return best;
 }
 
+void apply_schedule(vdit_plan* p, Schedule&& s) {
+    p->cta = std::move(s.cta);
+    p->merge = std::move(s.merge);
+    p->n_slots = s.slots;
+    p->n_split = s.max_pieces;
+}
+
 }  // namespace
 
-extern "C" int vdit_plan_split_for(const vdit_plan* p, int sm_count, int* kv_splits) {
-    if (!p || !kv_splits || sm_count < 1)
-        return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or output, or sm_count < 1");
-    *kv_splits = choose_split(*p, sm_count);
+extern "C" int vdit_plan_export_schedule(const vdit_plan* p, int sm_count, int* n_ctas, int* n_cut_units,
+                                         int* cta, int* merge) {
+    if (!p || !n_ctas || !n_cut_units || sm_count < 1)
+        return vdit::fail(VDIT_ERR_INVALID_ARG, "NULL plan or count, or sm_count < 1");
+    const Schedule s = build_schedule(*p, sm_count);
+    *n_ctas = (int)(s.cta.size() / 5);
+    *n_cut_units = (int)(s.merge.size() / 4);
+    if (cta) std::memcpy(cta, s.cta.data(), sizeof(int) * s.cta.size());
+    if (merge && !s.merge.empty()) std::memcpy(merge, s.merge.data(), sizeof(int) * s.merge.size());
     return VDIT_OK;
 }
 
@@ -474,6 +560,8 @@ extern "C" int vdit_plan_info(const vdit_plan* p, vdit_plan_info_t* info) {
     info->uploaded = p->d_buf != nullptr;
     info->kv_splits = p->n_split;
     info->workspace_bytes = (long long)p->ws_bytes;
+    info->ctas = (int)(p->cta.size() / 5);
+    info->cut_units = (int)(p->merge.size() / 4);
     info->mask_bytes = (long long)(sizeof(uint32_t) * p->masks.size());
     info->work_entries = (int)p->w_key.size();
     info->single_patch_entries = p->n_diag;
@@ -528,23 +616,31 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     // the attention kernels' per-device set-up happens here, in a call that allocates anyway, so
     // that the forward calls on this plan (the no-allocation one included) only launch
     if (int rc = vdit::attn_prepare_device(dev)) return rc;
-    p->n_split = choose_split(*p, sms);
-    // one allocation of what the kernels read: u_row_ptr | u_col | u_flags | unit_order | u_mask |
-    // masks | (split workspace: partial O | partial lse); the per-q-tile lists, the slot frames
-    // and the radius table stay on the host (exports, mask construction)
+    apply_schedule(p, build_schedule(*p, sms));
+    // one allocation of what the kernels read: u_row_ptr | u_col | u_flags | CTA table (int4) |
+    // CTA slots | merge table (int4) | u_mask | masks | (workspace: partial O | partial lse); the
+    // per-q-tile lists, the slot frames and the radius table stay on the host (exports, mask
+    // construction)
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+    const int n_cta = (int)(p->cta.size() / 5), n_cut = (int)(p->merge.size() / 4);
+    std::vector<int> cta4(4 * (size_t)n_cta), slot(n_cta);
+    for (int c = 0; c < n_cta; ++c) {
+        for (int k = 0; k < 4; ++k) cta4[4 * (size_t)c + k] = p->cta[5 * (size_t)c + k];
+        slot[c] = p->cta[5 * (size_t)c + 4];
+    }
     const size_t n_urp = sizeof(int) * p->u_row_ptr.size();
     const size_t n_uc = sizeof(int) * std::max<size_t>(1, p->u_col.size());
     const size_t n_uf = std::max<size_t>(1, p->u_flags.size());
-    const size_t n_uo = sizeof(int) * std::max<size_t>(1, p->unit_order.size());
+    const size_t n_ct = sizeof(int) * std::max<size_t>(4, cta4.size());
+    const size_t n_cs = sizeof(int) * std::max<size_t>(1, slot.size());
+    const size_t n_mg = sizeof(int) * std::max<size_t>(4, p->merge.size());
     const size_t n_um = sizeof(int) * std::max<size_t>(1, p->u_mask.size());
     const size_t n_mk = sizeof(uint32_t) * std::max<size_t>(4, p->kmasks.size());
-    const size_t n_wo = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->q_tokens *
-                                             p->g.heads * p->g.head_dim : 0;
-    const size_t n_wl = p->n_split > 1 ? sizeof(float) * (size_t)p->n_split * p->g.heads * p->q_tokens : 0;
-    const size_t meta = up(n_urp) + up(n_uc) + up(n_uf) + up(n_uo) + up(n_um) + up(n_mk);
+    const size_t n_wo = sizeof(float) * (size_t)p->n_slots * 256 * p->g.head_dim;
+    const size_t n_wl = sizeof(float) * (size_t)p->n_slots * 256;
+    const size_t meta = up(n_urp) + up(n_uc) + up(n_uf) + up(n_ct) + up(n_cs) + up(n_mg) + up(n_um) + up(n_mk);
     const size_t total = meta + up(n_wo) + up(n_wl);
-    std::vector<unsigned char> host(total, 0);
+    std::vector<unsigned char> host(meta, 0);
     size_t off = 0;
     auto put = [&](const void* src, size_t n, size_t reserved) {
         size_t at = off;
@@ -555,11 +651,13 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     const size_t o_urp = put(p->u_row_ptr.data(), n_urp, n_urp);
     const size_t o_uc = put(p->u_col.data(), sizeof(int) * p->u_col.size(), n_uc);
     const size_t o_uf = put(p->u_flags.data(), p->u_flags.size(), n_uf);
-    const size_t o_uo = put(p->unit_order.data(), sizeof(int) * p->unit_order.size(), n_uo);
+    const size_t o_ct = put(cta4.data(), sizeof(int) * cta4.size(), n_ct);
+    const size_t o_cs = put(slot.data(), sizeof(int) * slot.size(), n_cs);
+    const size_t o_mg = put(p->merge.data(), sizeof(int) * p->merge.size(), n_mg);
     const size_t o_um = put(p->u_mask.data(), sizeof(int) * p->u_mask.size(), n_um);
     const size_t o_mk = put(p->kmasks.data(), sizeof(uint32_t) * p->kmasks.size(), n_mk);
     if (off != meta) return vdit::fail(VDIT_ERR_INVALID_ARG, "internal: plan layout mismatch");
-    host.resize(meta);  // the workspace is not initialised: every entry is written before use
+    // the workspace is not initialised: a piece writes every partial row it owns before the merge
     void* d = nullptr;
     if (int rc = cuda_check(cudaMalloc(&d, total), "cudaMalloc(plan)")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -575,11 +673,13 @@ extern "C" int vdit_plan_upload(vdit_plan* p, void* stream) {
     p->d_u_row_ptr = reinterpret_cast<const int*>(b + o_urp);
     p->d_u_col = reinterpret_cast<const int*>(b + o_uc);
     p->d_u_flags = b + o_uf;
-    p->d_unit_order = reinterpret_cast<const int*>(b + o_uo);
+    p->d_cta = reinterpret_cast<const int*>(b + o_ct);
+    p->d_cta_slot = reinterpret_cast<const int*>(b + o_cs);
+    p->d_merge = reinterpret_cast<const int*>(b + o_mg);
     p->d_u_mask = reinterpret_cast<const int*>(b + o_um);
     p->d_masks = reinterpret_cast<const uint32_t*>(b + o_mk);
-    p->ws_bytes = n_wo + n_wl;
-    if (p->n_split > 1) {
+    p->ws_bytes = p->n_slots ? up(n_wo) + n_wl : 0;
+    if (p->n_slots) {
         p->d_ws_o = reinterpret_cast<float*>(b + meta);
         p->d_ws_lse = reinterpret_cast<float*>(b + meta + up(n_wo));
     }
