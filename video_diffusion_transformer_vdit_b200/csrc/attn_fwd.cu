@@ -46,6 +46,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -268,22 +269,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         int cnt = 0;                   // score tiles read
         int npv_dyn = 0;               // dynamic-threshold mode: P tiles stored (else == cnt)
         bool ok = true;
-        for (int j = 0; j < n_v; ++j) {
+        // One score tile of the union list (entry j): P = 0 the attention tile of the static mask,
+        // P = 1 the logit pass and P = 2 the attention pass of the dynamic-threshold mode. The
+        // dynamic mode runs the two passes as two loops, so each loop body is compiled for its
+        // pass alone (one body for both spilled registers in the loop). false: a wait ran out.
+        auto score_tile = [&](const int j, auto pass) -> bool {
             // dynamic-threshold mode: pass 0 (j < n_ent) only takes the row maxima of the
             // candidates' logits; pass 1 keeps a candidate iff its logit is within tau of it
-            const bool pass0 = DYN && j < n_ent, pass1 = DYN && j >= n_ent;
+            constexpr bool pass0 = decltype(pass)::value == 1, pass1 = decltype(pass)::value == 2;
             const int npv = DYN ? npv_dyn : cnt;
             const int s = j % kStages;
-            if (!warp_wait(BAR(B_IFULL + s), (j / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+            if (!warp_wait(BAR(B_IFULL + s), (j / kStages) & 1, abort_flag, a.status)) { ok = false; return false; }
             const uint8_t* info = smem + L::OFF_KINFO + s * kKinfoBytes;
             const uint32_t flags = (uint32_t)reinterpret_cast<const int*>(info)[1];
             // dynamic-threshold logit pass: each query tile's score tiles have a buffer of their own
             const uint32_t sbuf = pass0 ? (uint32_t)h : 0u;
             if (!(flags & f_in)) {
                 mbar_arrive(BAR(B_IEMPTY + s));
-                continue;
+                return true;
             }
-            if (!warp_wait(BAR(B_SFULL + h), cnt & 1, abort_flag, a.status)) { ok = false; break; }
+            if (!warp_wait(BAR(B_SFULL + h), cnt & 1, abort_flag, a.status)) { ok = false; return false; }
             tc_fence_after();
             uint32_t sr[128];
 #pragma unroll
@@ -306,11 +311,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mbar_arrive(BAR(B_IEMPTY + s));
             float m_tile = -INFINITY;
-            if (pass1) {
-                // the row maximum m is final: drop candidates more than tau below it
-                const float thr = m * c - a.tau_log2;
+            if constexpr (pass1) {
+                // the row maximum m is final: drop candidates more than tau below it, compared in
+                // raw score units (s >= m - tau / scale: a compare and a select per element; one
+                // select for both the keep bit and the threshold measured 12% slower)
+                const float thr = m - a.tau_log2 / c;
 #pragma unroll
-                for (int jj = 0; jj < 128; ++jj) sv[jj] = sv[jj] * c >= thr ? sv[jj] : -INFINITY;
+                for (int jj = 0; jj < 128; ++jj) sv[jj] = sv[jj] >= thr ? sv[jj] : -INFINITY;
             } else {
                 // row max: 8 independent chains of 3-input max
                 float mx[8];
@@ -323,10 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             }
-            if (pass0) {
+            if constexpr (pass0) {
                 m = fmaxf(m, m_tile);
                 ++cnt;
-                continue;
+                return true;
             }
             const float m_new = fmaxf(m, m_tile);
             const bool resc = (m_new - m) * c > kRescaleTau;
@@ -339,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // PV_h of the previous tile must have completed: it reads P_h (overwritten below)
             // and accumulates into O_h (rescaled below)
             if (npv > 0) {
-                if (!warp_wait(BAR(B_PVDONE + h), (npv - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (!warp_wait(BAR(B_PVDONE + h), (npv - 1) & 1, abort_flag, a.status)) { ok = false; return false; }
                 tc_fence_after();
             }
             if (npv > 0 && __any_sync(0xffffffffu, resc)) {
@@ -390,6 +397,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(BAR(B_PFULL + h));
             ++cnt;
             if (DYN) ++npv_dyn;
+            return true;
+        };
+        if constexpr (DYN) {
+            for (int j = 0; j < n_ent; ++j)
+                if (!score_tile(j, std::integral_constant<int, 1>{})) break;
+            if (ok)
+                for (int j = n_ent; j < n_v; ++j)
+                    if (!score_tile(j, std::integral_constant<int, 2>{})) break;
+        } else {
+            for (int j = 0; j < n_ent; ++j)
+                if (!score_tile(j, std::integral_constant<int, 0>{})) break;
         }
         const int n_pv = DYN ? npv_dyn : cnt;
         if (ok && n_pv > 0) {
