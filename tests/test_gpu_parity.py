@@ -203,6 +203,11 @@ def test_attention_full_size_sampled(wid):
     last_tile = np.arange((w.q_tokens - 1) // 128 * 128, w.q_tokens)
     rows = np.unique(np.r_[np.arange(0, 64), rng.integers(0, w.q_tokens, 96), last_tile])
     hs = [0, w.heads // 2, w.heads - 1]
+    # the sample includes rows of units that the CTA schedule cut into key pieces, where it cuts
+    cta, merge = plan.schedule_for(torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan.info["ctas"] == len(cta) and plan.info["cut_units"] == len(merge)
+    cut = {(hd, r) for qb, hd, _, _ in merge.tolist() for r in range(qb * 256, min(qb * 256 + 256, w.q_tokens))}
+    assert not cut or any((hd, int(r)) in cut for hd in hs for r in rows)
     ro, rl = run_oracle(w, q, k, v, rows, hs)
     assert_close(f64(o[rows][:, hs]), ro)
     assert np.max(np.abs(lse[hs][:, rows].cpu().numpy() - rl)) < 2e-2
