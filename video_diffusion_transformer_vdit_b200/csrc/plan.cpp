@@ -7,14 +7,18 @@
 // range splits into row segments (constant frame and patch row h, a contiguous run of columns w),
 // and for two segments every predicate term is either constant (validity, causal chunk order,
 // |dt|, |dh|) or a function of |w_q - w_k| over two integer intervals, whose minimum and maximum
-// are closed forms. Cost is O(tiles x segment pairs) instead of O(tokens^2).
+// are closed forms. Cost is O(tiles x segment pairs) instead of O(tokens^2). The query tiles are
+// computed independently by a few host threads and merged in tile order, so the plan (the
+// numbering of its shared keep-mask blocks included) does not depend on the thread count.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstdio>
 #include <cstring>
 #include <functional>
 #include <new>
 #include <unordered_map>
+#include <thread>
 #include <vector>
 
 #include <cuda_runtime.h>
@@ -107,34 +111,40 @@ long long pairs_within(int a0, int a1, int b0, int b1, int r) {
     return n;
 }
 
-// Appends the keep mask of one partial tile: rows q0 .. q1-1 (query tokens) against the key tile
-// whose row segments are `keys`; 128 rows x 4 words, bit k of row r set iff key k is kept for
-// query q0 + r. Per (query, key segment) the kept keys form one run of columns (the predicate's
-// frame and row terms are constant on a segment and the Chebyshev window is an interval of w).
-void tile_mask(const vdit_plan& p, int q0, int q1, const std::vector<Seg>& keys,
+// Appends the keep mask of one partial tile: its query row segments `qs` (rows q0 .. of the tile,
+// segment offsets relative to q0) against the key tile whose row segments are `keys`; 128 rows x
+// 4 words, bit k of row r set iff key k is kept for query q0 + r. The predicate's frame and row
+// terms are constant on a (query segment, key segment) pair, so they are evaluated once per pair;
+// per query row the kept keys of a key segment are then one run of columns (the Chebyshev window
+// is an interval of w). Key segments at a frame offset (key frame - query frame) listed in
+// skip_dt are left out.
+void tile_mask(const vdit_plan& p, const std::vector<Seg>& qs, const std::vector<Seg>& keys,
                std::vector<uint32_t>& out, const std::vector<int>* skip_dt = nullptr) {
     const size_t base = out.size();
     out.resize(base + 512, 0u);
     uint32_t* blk = out.data() + base;
-    const int ft = p.g.grid_h * p.g.grid_w;
     const bool causal = p.m.kind & VDIT_MASK_BLOCK_CAUSAL;
-    for (int r = 0; r < q1 - q0; ++r) {
-        const int qi = q0 + r, f = qi / ft, rem = qi % ft;
-        const int tq = p.q_start + f, hq = rem / p.g.grid_w, wq = rem % p.g.grid_w;
-        uint32_t* row = blk + 4 * r;
+    for (const Seg& a : qs) {
         for (const Seg& b : keys) {
             if (b.t < 0) continue;
-            if (skip_dt && std::find(skip_dt->begin(), skip_dt->end(), b.t - tq) != skip_dt->end()) continue;
-            if (causal && b.t / p.m.chunk_frames > tq / p.m.chunk_frames) continue;
-            const long long rad = p.radius[std::abs(tq - b.t)];
-            if (std::abs(hq - b.h) > rad) continue;
-            const long long lo = std::max<long long>(b.wlo, wq - rad);
-            const long long hi = std::min<long long>(b.whi, wq + rad);
-            if (lo > hi) continue;
-            const int k0 = b.off + (int)(lo - b.wlo), k1 = b.off + (int)(hi - b.wlo);
-            for (int wd = k0 >> 5; wd <= k1 >> 5; ++wd) {
-                const int a0 = std::max(k0 - 32 * wd, 0), a1 = std::min(k1 - 32 * wd, 31);
-                row[wd] |= (0xffffffffu >> (31 - a1)) & (0xffffffffu << a0);
+            if (skip_dt && std::find(skip_dt->begin(), skip_dt->end(), b.t - a.t) != skip_dt->end()) continue;
+            if (causal && b.t / p.m.chunk_frames > a.t / p.m.chunk_frames) continue;
+            const long long rad = p.radius[std::abs(a.t - b.t)];
+            if (std::abs(a.h - b.h) > rad) continue;
+            for (int wq = a.wlo; wq <= a.whi; ++wq) {
+                const long long lo = std::max<long long>(b.wlo, wq - rad);
+                const long long hi = std::min<long long>(b.whi, wq + rad);
+                if (lo > hi) continue;
+                // keys k0 .. k1 of the tile as a 128-bit run, OR-ed into the row's four words
+                const int k0 = b.off + (int)(lo - b.wlo), k1 = b.off + (int)(hi - b.wlo);
+                const unsigned __int128 one = 1;
+                const unsigned __int128 run = (k1 == 127 ? ~(unsigned __int128)0 : (one << (k1 + 1)) - 1) &
+                                              ~((one << k0) - 1);
+                uint32_t* row = blk + 4 * (a.off + (wq - a.wlo));
+                row[0] |= (uint32_t)run;
+                row[1] |= (uint32_t)(run >> 32);
+                row[2] |= (uint32_t)(run >> 64);
+                row[3] |= (uint32_t)(run >> 96);
             }
         }
     }
@@ -173,21 +183,137 @@ void scan_tile(const vdit_plan& p, const std::vector<Seg>& qs, const std::vector
     }
 }
 
-// Stores the 512-word block at the end of `pool` once: returns the number of an identical block
-// already in the pool (and drops the new copy), else the new block's number.
-int dedupe_block(std::vector<uint32_t>& pool, std::unordered_map<uint64_t, std::vector<int>>& seen) {
-    const size_t at = pool.size() - 512;
-    uint64_t hsh = 1469598103934665603ull;  // FNV-1a over the 512 words
-    for (size_t wi = at; wi < at + 512; ++wi) hsh = (hsh ^ pool[wi]) * 1099511628211ull;
-    auto& same = seen[hsh];
+// Hash of one 512-word keep-mask block: FNV-1a-style over 64-bit words in four interleaved lanes
+// (independent multiply chains), folded into one value. Equal blocks are confirmed word by word.
+uint64_t block_hash(const uint32_t* blk) {
+    uint64_t lane[4] = {1469598103934665603ull, 1469598103934665603ull ^ 1, 1469598103934665603ull ^ 2,
+                        1469598103934665603ull ^ 3};
+    for (int wi = 0; wi < 512; wi += 8)
+        for (int l = 0; l < 4; ++l)
+            lane[l] = (lane[l] ^ ((uint64_t)blk[wi + 2 * l] | (uint64_t)blk[wi + 2 * l + 1] << 32)) *
+                      1099511628211ull;
+    return ((lane[0] * 31 + lane[1]) * 31 + lane[2]) * 31 + lane[3];
+}
+
+// Stores block `blk` (hash h) in `pool` once: returns the number of an identical block already in
+// the pool, else appends it and returns its new number.
+int dedupe_block(std::vector<uint32_t>& pool, std::unordered_map<uint64_t, std::vector<int>>& seen,
+                 const uint32_t* blk, uint64_t h) {
+    auto& same = seen[h];
     for (int b : same)
-        if (std::equal(pool.begin() + at, pool.begin() + at + 512, pool.begin() + (size_t)b * 512)) {
-            pool.resize(at);
-            return b;
-        }
-    const int block = (int)(at / 512);
+        if (std::equal(blk, blk + 512, pool.begin() + (size_t)b * 512)) return b;
+    const int block = (int)(pool.size() / 512);
+    pool.insert(pool.end(), blk, blk + 512);
     same.push_back(block);
     return block;
+}
+
+// What one query tile contributes to the plan, computed independently of the other tiles (so the
+// tiles are computed in parallel) and merged into the plan in tile order (so the result, block
+// numbering included, does not depend on the threads).
+struct QtOut {
+    // schedule of the mask as it is: listed key tiles, full flags, kept pairs; the keep-mask
+    // blocks of the partial ones (512 words each, in list order) and their hashes
+    std::vector<int> kt;
+    std::vector<unsigned char> full;
+    long long kept = 0;
+    std::vector<uint32_t> blocks;
+    std::vector<uint64_t> hashes;
+    // kernel work list when single-patch entries pay off (dts not empty): aligned entries (key
+    // row, partial or not) without the single-patch pairs, then one entry per offset in dts with
+    // first key row diag_key; wblocks / whashes: the partial aligned entries' blocks, then one
+    // block per offset
+    std::vector<int> dts, wkey, diag_key;
+    std::vector<unsigned char> wpartial;
+    std::vector<uint32_t> wblocks;
+    std::vector<uint64_t> whashes;
+};
+
+void plan_qtile(const vdit_plan& p, int qt, const std::vector<std::vector<Seg>>& kseg, bool single_patch,
+                std::vector<Seg>& qs, QtOut& o) {
+    const vdit_mask* m = &p.m;
+    const int ft = p.g.grid_h * p.g.grid_w;
+    const bool causal = m->kind & VDIT_MASK_BLOCK_CAUSAL;
+    const int q0 = qt * VDIT_TILE, q1 = std::min(p.q_tokens, q0 + VDIT_TILE);
+    segments(q0, q1, p.g.grid_h, p.g.grid_w, [&](int f) { return p.q_start + f; }, qs);
+    o = QtOut();
+    for (int kt = 0; kt < p.n_kt; ++kt) {
+        const int k0 = kt * VDIT_TILE, k1 = std::min(p.kv_tokens, k0 + VDIT_TILE);
+        bool any, all;
+        long long kept;
+        scan_tile(p, qs, kseg[kt], (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE), nullptr, any, all, kept);
+        o.kept += kept;
+        if (!any) continue;
+        o.kt.push_back(kt);
+        o.full.push_back(all ? 1 : 0);
+        if (!all) {
+            // keep-mask block of this tile; identical blocks (tiles at the same offsets within
+            // their frames with the same radii) are stored once at the merge, so the blocks the
+            // kernel reads for all heads stay resident in L2
+            tile_mask(p, qs, kseg[kt], o.blocks);
+            o.hashes.push_back(block_hash(o.blocks.data() + o.blocks.size() - 512));
+        }
+    }
+    const int n_export = (int)o.kt.size();
+    // frame offsets dt (key frame - query frame) whose radial window is one patch: the kept
+    // pairs at dt are (q, q + dt frames), one contiguous run of 128 key rows when the key
+    // frames of the tile's (at most two) query frames sit in consecutive ring slots
+    const int fa = q0 / ft, fb = (q1 - 1) / ft;
+    const int ta = p.q_start + fa, tb = p.q_start + fb;
+    if (single_patch) {
+        for (int dt = p.kv_first - tb; dt <= p.kv_last - ta; ++dt) {
+            if (p.radius[std::abs(dt)] != 0 || ta + dt < 0) continue;
+            const int sa = (ta + dt) % p.cap_frames;
+            if (fb != fa && sa == p.cap_frames - 1) continue;  // the run wraps the ring
+            bool valid = false;
+            for (int t = ta; t <= tb && !valid; ++t) {
+                const int kf = t + dt;
+                valid = kf >= p.kv_first && kf <= p.kv_last &&
+                        !(causal && kf / m->chunk_frames > t / m->chunk_frames);
+            }
+            if (valid) o.dts.push_back(dt);
+        }
+    }
+    // kernel work list: the aligned tiles without the single-patch pairs, plus one entry per
+    // offset, kept only when it shortens the list
+    if (o.dts.empty()) return;
+    for (int kt = 0; kt < p.n_kt; ++kt) {
+        const int k0 = kt * VDIT_TILE, k1 = std::min(p.kv_tokens, k0 + VDIT_TILE);
+        bool any, all;
+        long long kept;
+        scan_tile(p, qs, kseg[kt], (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE), &o.dts, any, all, kept);
+        if (!any) continue;
+        o.wkey.push_back(k0);
+        o.wpartial.push_back(all ? 0 : 1);
+        if (!all) {
+            tile_mask(p, qs, kseg[kt], o.wblocks, &o.dts);
+            o.whashes.push_back(block_hash(o.wblocks.data() + o.wblocks.size() - 512));
+        }
+    }
+    if ((int)(o.wkey.size() + o.dts.size()) >= n_export) {  // no gain: plain tiles
+        o.dts.clear();
+        o.wkey.clear();
+        o.wpartial.clear();
+        o.wblocks.clear();
+        o.whashes.clear();
+        return;
+    }
+    for (int dt : o.dts) {
+        // row r (query q0 + r at frame t) keeps key row k_start + r, its own patch at frame
+        // t + dt, if that frame is held and the chunk order allows it
+        const int k_start = ((ta + dt) % p.cap_frames) * ft + (q0 - fa * ft);
+        const size_t at = o.wblocks.size();
+        o.wblocks.resize(at + 512, 0u);
+        for (int r = 0; r < q1 - q0; ++r) {
+            const int t = p.q_start + (q0 + r) / ft, kf = t + dt;
+            const bool keep = kf >= p.kv_first && kf <= p.kv_last &&
+                              !(causal && kf / m->chunk_frames > t / m->chunk_frames) &&
+                              k_start + r < p.kv_tokens;
+            if (keep) o.wblocks[at + 4 * r + (r >> 5)] |= 1u << (r & 31);
+        }
+        o.diag_key.push_back(k_start);
+        o.whashes.push_back(block_hash(o.wblocks.data() + at));
+    }
 }
 
 }  // namespace
@@ -217,197 +343,171 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
 
     vdit_plan* p = new (std::nothrow) vdit_plan();
     if (!p) return fail(VDIT_ERR_INVALID_ARG, "out of host memory");
-    p->g = *g;
-    p->m = *m;
-    p->q_start = q_start_frame;
-    p->q_frames = q_frames;
-    p->cap_frames = capacity_frames;
-    p->kv_first = kv_first_frame;
-    p->kv_last = kv_last_frame;
-    const int ft = g->grid_h * g->grid_w;
-    const long long qtok = (long long)q_frames * ft, ktok = (long long)capacity_frames * ft;
-    if (qtok > INT_MAX / 2 || ktok > INT_MAX / 2) {
+    // host allocations below may fail (bad_alloc); the C ABI reports that instead of throwing
+    try {
+        p->g = *g;
+        p->m = *m;
+        p->q_start = q_start_frame;
+        p->q_frames = q_frames;
+        p->cap_frames = capacity_frames;
+        p->kv_first = kv_first_frame;
+        p->kv_last = kv_last_frame;
+        const int ft = g->grid_h * g->grid_w;
+        const long long qtok = (long long)q_frames * ft, ktok = (long long)capacity_frames * ft;
+        if (qtok > INT_MAX / 2 || ktok > INT_MAX / 2) {
+            delete p;
+            return fail(VDIT_ERR_UNSUPPORTED, "too many tokens");
+        }
+        p->q_tokens = (int)qtok;
+        p->kv_tokens = (int)ktok;
+        p->n_qt = (p->q_tokens + VDIT_TILE - 1) / VDIT_TILE;
+        p->n_kt = (p->kv_tokens + VDIT_TILE - 1) / VDIT_TILE;
+
+        p->slot_frame.assign(capacity_frames, -1);
+        for (int f = kv_first_frame; f <= kv_last_frame; ++f) p->slot_frame[f % capacity_frames] = f;
+
+        const int q_last = q_start_frame + q_frames - 1;
+        p->dt_max = std::max(std::abs(q_last - kv_first_frame), std::abs(kv_last_frame - q_start_frame));
+        if (p->dt_max > VDIT_MAX_DT) {
+            delete p;
+            return fail(VDIT_ERR_UNSUPPORTED, "query and key frames further apart than VDIT_MAX_DT");
+        }
+        p->radius.resize(p->dt_max + 1);
+        for (int dt = 0; dt <= p->dt_max; ++dt) p->radius[dt] = radius_at(*m, dt);
+
+        std::vector<std::vector<Seg>> kseg(p->n_kt);
+        for (int kt = 0; kt < p->n_kt; ++kt)
+            segments(kt * VDIT_TILE, std::min(p->kv_tokens, (kt + 1) * VDIT_TILE), g->grid_h,
+                     g->grid_w, [&](int slot) { return p->slot_frame[slot]; }, kseg[kt]);
+        std::unordered_map<uint64_t, std::vector<int>> seen, kseen;  // mask block hash -> block numbers
+        p->row_ptr.assign(p->n_qt + 1, 0);
+        p->w_row_ptr.assign(p->n_qt + 1, 0);
+        p->w_aligned.assign(p->n_qt, 0);
+        p->kept_pairs = 0;
+        p->n_full = 0;
+        // single-patch entries need a q-tile to span at most two frames (128 <= tokens per frame)
+        const bool single_patch = (m->kind & VDIT_MASK_RADIAL) && ft >= VDIT_TILE;
+        // q-tiles are computed in batches by a few host threads, then merged in order
+        const int n_threads = (int)std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+        const int batch = std::max(1, std::min(p->n_qt, 8 * n_threads));
+        std::vector<QtOut> outs(batch);
+        std::vector<std::vector<Seg>> qsegs(n_threads);
+        for (int b0 = 0; b0 < p->n_qt; b0 += batch) {
+            const int nb = std::min(batch, p->n_qt - b0);
+            std::atomic<int> next{0};
+            std::atomic<bool> failed{false};
+            auto work = [&](int tid) {
+                try {
+                    for (int i = next++; i < nb; i = next++) plan_qtile(*p, b0 + i, kseg, single_patch, qsegs[tid], outs[i]);
+                } catch (...) {
+                    failed = true;
+                }
+            };
+            const int nt = std::min(n_threads, nb);
+            std::vector<std::thread> pool;
+            try {
+                for (int t = 1; t < nt; ++t) pool.emplace_back(work, t);
+            } catch (...) {
+                failed = true;  // no further thread: the calling thread does the rest
+            }
+            work(0);
+            for (auto& th : pool) th.join();
+            if (failed) throw std::bad_alloc();
+            // merge in q-tile order
+            for (int i = 0; i < nb; ++i) {
+                const int qt = b0 + i;
+                const QtOut& o = outs[i];
+                p->kept_pairs += o.kept;
+                const size_t first = p->col_idx.size();
+                for (size_t e = 0, pb = 0; e < o.kt.size(); ++e) {
+                    p->col_idx.push_back(o.kt[e]);
+                    p->full.push_back(o.full[e]);
+                    p->n_full += o.full[e];
+                    int block = -1;
+                    if (!o.full[e]) {
+                        block = dedupe_block(p->masks, seen, o.blocks.data() + 512 * pb, o.hashes[pb]);
+                        ++pb;
+                    }
+                    p->mask_of.push_back(block);
+                }
+                p->row_ptr[qt + 1] = (int)p->col_idx.size();
+                if (o.dts.empty()) {
+                    p->w_aligned[qt] = (int)o.kt.size();
+                    for (size_t e = first, pb = 0; e < p->col_idx.size(); ++e) {
+                        p->w_key.push_back(p->col_idx[e] * VDIT_TILE);
+                        int block = -1;
+                        if (!p->full[e]) {
+                            block = dedupe_block(p->kmasks, kseen, o.blocks.data() + 512 * pb, o.hashes[pb]);
+                            ++pb;
+                        }
+                        p->w_mask.push_back(block);
+                    }
+                } else {
+                    p->w_aligned[qt] = (int)o.wkey.size();
+                    size_t pb = 0;
+                    for (size_t e = 0; e < o.wkey.size(); ++e) {
+                        p->w_key.push_back(o.wkey[e]);
+                        int block = -1;
+                        if (o.wpartial[e]) {
+                            block = dedupe_block(p->kmasks, kseen, o.wblocks.data() + 512 * pb, o.whashes[pb]);
+                            ++pb;
+                        }
+                        p->w_mask.push_back(block);
+                    }
+                    for (size_t d = 0; d < o.dts.size(); ++d, ++pb) {
+                        p->w_key.push_back(o.diag_key[d]);
+                        p->w_mask.push_back(dedupe_block(p->kmasks, kseen, o.wblocks.data() + 512 * pb, o.whashes[pb]));
+                        ++p->n_diag;
+                    }
+                }
+                p->w_row_ptr[qt + 1] = (int)p->w_key.size();
+            }
+        }
+        // union lists of q-tile pairs, from the kernel's work list: entries at the same (aligned) key
+        // row merge; an unaligned single-patch entry stays on its own (one q-tile)
+        p->n_qb = (p->n_qt + 1) / 2;
+        p->u_row_ptr.assign(p->n_qb + 1, 0);
+        for (int b = 0; b < p->n_qb; ++b) {
+            const int t0 = 2 * b, t1 = 2 * b + 1;
+            // aligned entries of the two q-tiles, merged by key row (both ascending)
+            int i = p->w_row_ptr[t0], ie = i + p->w_aligned[t0];
+            int k = t1 < p->n_qt ? p->w_row_ptr[t1] : 0, ke = t1 < p->n_qt ? k + p->w_aligned[t1] : 0;
+            while (i < ie || k < ke) {
+                const int ci = i < ie ? p->w_key[i] : INT_MAX, ck = k < ke ? p->w_key[k] : INT_MAX;
+                const int c = std::min(ci, ck);
+                unsigned char f = 0;
+                int m0 = -1, m1 = -1;
+                if (ci == c) { f |= 1 | (p->w_mask[i] < 0 ? 2 : 0); m0 = p->w_mask[i]; ++i; }
+                if (ck == c) { f |= 4 | (p->w_mask[k] < 0 ? 8 : 0); m1 = p->w_mask[k]; ++k; }
+                p->u_col.push_back(c);
+                p->u_flags.push_back(f);
+                p->u_mask.push_back(m0);
+                p->u_mask.push_back(m1);
+            }
+            // single-patch entries, each for one q-tile
+            for (int x = 0; x < 2; ++x) {
+                const int qt = t0 + x;
+                if (qt >= p->n_qt) break;
+                for (int e = p->w_row_ptr[qt] + p->w_aligned[qt]; e < p->w_row_ptr[qt + 1]; ++e) {
+                    p->u_col.push_back(p->w_key[e]);
+                    p->u_flags.push_back((unsigned char)(x ? 4 : 1));
+                    p->u_mask.push_back(x ? -1 : p->w_mask[e]);
+                    p->u_mask.push_back(x ? p->w_mask[e] : -1);
+                }
+            }
+            p->u_row_ptr[b + 1] = (int)p->u_col.size();
+        }
+        p->unit_order.resize(p->n_qb);
+        for (int i = 0; i < p->n_qb; ++i) p->unit_order[i] = i;
+        std::stable_sort(p->unit_order.begin(), p->unit_order.end(), [&](int a, int b) {
+            return p->u_row_ptr[a + 1] - p->u_row_ptr[a] > p->u_row_ptr[b + 1] - p->u_row_ptr[b];
+        });
+        *out = p;
+        return VDIT_OK;
+    } catch (const std::bad_alloc&) {
         delete p;
-        return fail(VDIT_ERR_UNSUPPORTED, "too many tokens");
+        return fail(VDIT_ERR_UNSUPPORTED, "out of host memory while building the plan");
     }
-    p->q_tokens = (int)qtok;
-    p->kv_tokens = (int)ktok;
-    p->n_qt = (p->q_tokens + VDIT_TILE - 1) / VDIT_TILE;
-    p->n_kt = (p->kv_tokens + VDIT_TILE - 1) / VDIT_TILE;
-
-    p->slot_frame.assign(capacity_frames, -1);
-    for (int f = kv_first_frame; f <= kv_last_frame; ++f) p->slot_frame[f % capacity_frames] = f;
-
-    const int q_last = q_start_frame + q_frames - 1;
-    p->dt_max = std::max(std::abs(q_last - kv_first_frame), std::abs(kv_last_frame - q_start_frame));
-    if (p->dt_max > VDIT_MAX_DT) {
-        delete p;
-        return fail(VDIT_ERR_UNSUPPORTED, "query and key frames further apart than VDIT_MAX_DT");
-    }
-    p->radius.resize(p->dt_max + 1);
-    for (int dt = 0; dt <= p->dt_max; ++dt) p->radius[dt] = radius_at(*m, dt);
-
-    const bool causal = m->kind & VDIT_MASK_BLOCK_CAUSAL;
-    std::vector<std::vector<Seg>> kseg(p->n_kt);
-    for (int kt = 0; kt < p->n_kt; ++kt)
-        segments(kt * VDIT_TILE, std::min(p->kv_tokens, (kt + 1) * VDIT_TILE), g->grid_h,
-                 g->grid_w, [&](int slot) { return p->slot_frame[slot]; }, kseg[kt]);
-    std::vector<Seg> qs;
-    std::unordered_map<uint64_t, std::vector<int>> seen, kseen;  // mask block hash -> block numbers
-    p->row_ptr.assign(p->n_qt + 1, 0);
-    p->w_row_ptr.assign(p->n_qt + 1, 0);
-    p->w_aligned.assign(p->n_qt, 0);
-    p->kept_pairs = 0;
-    p->n_full = 0;
-    // single-patch entries need a q-tile to span at most two frames (128 <= tokens per frame)
-    const bool single_patch = (m->kind & VDIT_MASK_RADIAL) && ft >= VDIT_TILE;
-    std::vector<int> dts;
-    for (int qt = 0; qt < p->n_qt; ++qt) {
-        const int q0 = qt * VDIT_TILE, q1 = std::min(p->q_tokens, q0 + VDIT_TILE);
-        segments(q0, q1, g->grid_h, g->grid_w, [&](int f) { return q_start_frame + f; }, qs);
-        // schedule of the mask as it is (export, and the kernel's unless single-patch entries
-        // pay off below)
-        int n_export = 0;
-        for (int kt = 0; kt < p->n_kt; ++kt) {
-            const int k0 = kt * VDIT_TILE, k1 = std::min(p->kv_tokens, k0 + VDIT_TILE);
-            bool any, all;
-            long long kept;
-            scan_tile(*p, qs, kseg[kt], (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE), nullptr, any, all, kept);
-            p->kept_pairs += kept;
-            if (!any) continue;
-            ++n_export;
-            p->col_idx.push_back(kt);
-            p->full.push_back(all ? 1 : 0);
-            p->n_full += all;
-            int block = -1;
-            if (!all) {
-                // keep-mask block of this tile; identical blocks (tiles at the same offsets within
-                // their frames with the same radii) are stored once, so the blocks the kernel
-                // reads for all heads stay resident in L2
-                tile_mask(*p, q0, q1, kseg[kt], p->masks);
-                block = dedupe_block(p->masks, seen);
-            }
-            p->mask_of.push_back(block);
-        }
-        p->row_ptr[qt + 1] = (int)p->col_idx.size();
-
-        // frame offsets dt (key frame - query frame) whose radial window is one patch: the kept
-        // pairs at dt are (q, q + dt frames), one contiguous run of 128 key rows when the key
-        // frames of the tile's (at most two) query frames sit in consecutive ring slots
-        dts.clear();
-        const int fa = q0 / ft, fb = (q1 - 1) / ft;
-        const int ta = q_start_frame + fa, tb = q_start_frame + fb;
-        if (single_patch) {
-            for (int dt = kv_first_frame - tb; dt <= kv_last_frame - ta; ++dt) {
-                if (p->radius[std::abs(dt)] != 0 || ta + dt < 0) continue;
-                const int sa = (ta + dt) % capacity_frames;
-                if (fb != fa && sa == capacity_frames - 1) continue;  // the run wraps the ring
-                bool valid = false;
-                for (int t = ta; t <= tb && !valid; ++t) {
-                    const int kf = t + dt;
-                    valid = kf >= kv_first_frame && kf <= kv_last_frame &&
-                            !(causal && kf / m->chunk_frames > t / m->chunk_frames);
-                }
-                if (valid) dts.push_back(dt);
-            }
-        }
-        // kernel work list: the aligned tiles without the single-patch pairs, plus one entry per
-        // offset, kept only when it shortens the list
-        std::vector<int> key, blk;
-        if (!dts.empty()) {
-            for (int kt = 0; kt < p->n_kt; ++kt) {
-                const int k0 = kt * VDIT_TILE, k1 = std::min(p->kv_tokens, k0 + VDIT_TILE);
-                bool any, all;
-                long long kept;
-                scan_tile(*p, qs, kseg[kt], (q1 - q0 == VDIT_TILE) && (k1 - k0 == VDIT_TILE), &dts, any, all, kept);
-                if (!any) continue;
-                key.push_back(k0);
-                int block = -1;
-                if (!all) {
-                    tile_mask(*p, q0, q1, kseg[kt], p->kmasks, &dts);
-                    block = dedupe_block(p->kmasks, kseen);
-                }
-                blk.push_back(block);
-            }
-            if ((int)(key.size() + dts.size()) >= n_export) dts.clear();  // no gain: plain tiles
-        }
-        if (dts.empty()) {
-            p->w_aligned[qt] = p->row_ptr[qt + 1] - p->row_ptr[qt];
-            for (int i = p->row_ptr[qt]; i < p->row_ptr[qt + 1]; ++i) {
-                p->w_key.push_back(p->col_idx[i] * VDIT_TILE);
-                int block = -1;
-                if (!p->full[i]) {
-                    p->kmasks.insert(p->kmasks.end(), p->masks.begin() + (size_t)p->mask_of[i] * 512,
-                                     p->masks.begin() + (size_t)p->mask_of[i] * 512 + 512);
-                    block = dedupe_block(p->kmasks, kseen);
-                }
-                p->w_mask.push_back(block);
-            }
-        } else {
-            p->w_aligned[qt] = (int)key.size();
-            p->w_key.insert(p->w_key.end(), key.begin(), key.end());
-            p->w_mask.insert(p->w_mask.end(), blk.begin(), blk.end());
-            for (int dt : dts) {
-                // row r (query q0 + r at frame t) keeps key row k_start + r, its own patch at
-                // frame t + dt, if that frame is held and the chunk order allows it
-                const int k_start = ((ta + dt) % capacity_frames) * ft + (q0 - fa * ft);
-                const size_t at = p->kmasks.size();
-                p->kmasks.resize(at + 512, 0u);
-                for (int r = 0; r < q1 - q0; ++r) {
-                    const int t = q_start_frame + (q0 + r) / ft, kf = t + dt;
-                    const bool keep = kf >= kv_first_frame && kf <= kv_last_frame &&
-                                      !(causal && kf / m->chunk_frames > t / m->chunk_frames) &&
-                                      k_start + r < p->kv_tokens;
-                    if (keep) p->kmasks[at + 4 * r + (r >> 5)] |= 1u << (r & 31);
-                }
-                p->w_key.push_back(k_start);
-                p->w_mask.push_back(dedupe_block(p->kmasks, kseen));
-                ++p->n_diag;
-            }
-        }
-        p->w_row_ptr[qt + 1] = (int)p->w_key.size();
-    }
-    // union lists of q-tile pairs, from the kernel's work list: entries at the same (aligned) key
-    // row merge; an unaligned single-patch entry stays on its own (one q-tile)
-    p->n_qb = (p->n_qt + 1) / 2;
-    p->u_row_ptr.assign(p->n_qb + 1, 0);
-    for (int b = 0; b < p->n_qb; ++b) {
-        const int t0 = 2 * b, t1 = 2 * b + 1;
-        // aligned entries of the two q-tiles, merged by key row (both ascending)
-        int i = p->w_row_ptr[t0], ie = i + p->w_aligned[t0];
-        int k = t1 < p->n_qt ? p->w_row_ptr[t1] : 0, ke = t1 < p->n_qt ? k + p->w_aligned[t1] : 0;
-        while (i < ie || k < ke) {
-            const int ci = i < ie ? p->w_key[i] : INT_MAX, ck = k < ke ? p->w_key[k] : INT_MAX;
-            const int c = std::min(ci, ck);
-            unsigned char f = 0;
-            int m0 = -1, m1 = -1;
-            if (ci == c) { f |= 1 | (p->w_mask[i] < 0 ? 2 : 0); m0 = p->w_mask[i]; ++i; }
-            if (ck == c) { f |= 4 | (p->w_mask[k] < 0 ? 8 : 0); m1 = p->w_mask[k]; ++k; }
-            p->u_col.push_back(c);
-            p->u_flags.push_back(f);
-            p->u_mask.push_back(m0);
-            p->u_mask.push_back(m1);
-        }
-        // single-patch entries, each for one q-tile
-        for (int x = 0; x < 2; ++x) {
-            const int qt = t0 + x;
-            if (qt >= p->n_qt) break;
-            for (int e = p->w_row_ptr[qt] + p->w_aligned[qt]; e < p->w_row_ptr[qt + 1]; ++e) {
-                p->u_col.push_back(p->w_key[e]);
-                p->u_flags.push_back((unsigned char)(x ? 4 : 1));
-                p->u_mask.push_back(x ? -1 : p->w_mask[e]);
-                p->u_mask.push_back(x ? p->w_mask[e] : -1);
-            }
-        }
-        p->u_row_ptr[b + 1] = (int)p->u_col.size();
-    }
-    p->unit_order.resize(p->n_qb);
-    for (int i = 0; i < p->n_qb; ++i) p->unit_order[i] = i;
-    std::stable_sort(p->unit_order.begin(), p->unit_order.end(), [&](int a, int b) {
-        return p->u_row_ptr[a + 1] - p->u_row_ptr[a] > p->u_row_ptr[b + 1] - p->u_row_ptr[b];
-    });
-    *out = p;
-    return VDIT_OK;
 }
 
 namespace {
