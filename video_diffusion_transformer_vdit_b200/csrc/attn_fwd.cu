@@ -7,8 +7,10 @@
 // Wave Forcing / WaveRT block-causal chunks). Only the tiles the plan lists are visited; a tile
 // flagged full needs no mask; a partial one applies the per-row keep bits the plan computed.
 //
-// One CTA = two 128-row query tiles (Q0, Q1) of one head, sharing every K/V tile it loads;
-// 12 warps (3 warpgroups):
+// One CTA = two 128-row query tiles (Q0, Q1) of one head, sharing every K/V tile it loads, over
+// the union list of the two tiles' entries or, where the plan's CTA schedule cut the unit, one
+// key piece of it (its normalised fp32 partial result then goes to a workspace slot and
+// split_combine_kernel merges the pieces); 12 warps (3 warpgroups):
 //   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query row r (TMEM lane r);
 //               tcgen05.ld of its S row (after which the S columns are released), mask, online
 //               softmax in fp32 (log2 domain; O is rescaled in TMEM only when the running max
