@@ -164,7 +164,9 @@ VDIT_API int vdit_kv_write(const vdit_geom* g, void* k_cache, void* v_cache, int
  * Lists, per 128-query tile in ascending order, the 128-key tiles (ascending) that contain a kept
  * pair, each flagged full iff it is complete and wholly kept. Built exactly from the rectangle
  * geometry of the tiles (integer arithmetic only), so it is identical to the tile list of the
- * explicit per-pair mask. *out receives a new plan owned by the caller (vdit_plan_destroy). */
+ * explicit per-pair mask. *out receives a new plan owned by the caller (vdit_plan_destroy).
+ * The query tiles are computed on up to 16 host threads (environment variable VDIT_PLAN_THREADS
+ * overrides the count, 1 .. 64) and merged in tile order: the plan does not depend on it. */
 VDIT_API int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_mask* m,
                    int q_start_frame, int q_frames,
                    int capacity_frames, int kv_first_frame, int kv_last_frame);

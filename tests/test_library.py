@@ -243,6 +243,25 @@ def test_plan_masks_bit_exact_vs_oracle_random_geometries():
         _check_masks(plan, gh, gw, q_start, q_frames, cap, first, last, kind, chunk, w0, gs, lam)
 
 
+def test_plan_does_not_depend_on_the_host_thread_count(monkeypatch):
+    """vdit_attn_plan computes query tiles on host threads and merges them in tile order: one,
+    three and seven threads give the same tile lists, keep-mask blocks (numbering included) and
+    work list."""
+    def snapshot(w):
+        first, last = w.window()
+        plan = vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,
+                         kv_first_frame=first, kv_last_frame=last, upload=False)
+        return [np.ascontiguousarray(a) for a in (*plan.export(), *plan.export_masks(), *plan.export_work())]
+    for wid in (4, 5):
+        w = WORKLOADS[wid]
+        got = []
+        for n in ("1", "3", "7"):
+            monkeypatch.setenv("VDIT_PLAN_THREADS", n)
+            got.append(snapshot(w))
+        for other in got[1:]:
+            assert all(np.array_equal(a, b) for a, b in zip(got[0], other))
+
+
 def _plan_of(w):
     first, last = w.window()
     return vdit.Plan(_geom(w), _mask(w), w.q_start, w.q_frames, capacity_frames=w.capacity_frames,

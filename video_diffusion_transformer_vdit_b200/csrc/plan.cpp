@@ -14,6 +14,7 @@
 #include <atomic>
 #include <climits>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <functional>
 #include <new>
@@ -388,7 +389,11 @@ extern "C" int vdit_attn_plan(vdit_plan** out, const vdit_geom* g, const vdit_ma
         // single-patch entries need a q-tile to span at most two frames (128 <= tokens per frame)
         const bool single_patch = (m->kind & VDIT_MASK_RADIAL) && ft >= VDIT_TILE;
         // q-tiles are computed in batches by a few host threads, then merged in order
-        const int n_threads = (int)std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+        int n_threads = (int)std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+        if (const char* env = std::getenv("VDIT_PLAN_THREADS")) {
+            const int want = std::atoi(env);
+            if (want >= 1) n_threads = std::min(want, 64);
+        }
         const int batch = std::max(1, std::min(p->n_qt, 8 * n_threads));
         std::vector<QtOut> outs(batch);
         std::vector<std::vector<Seg>> qsegs(n_threads);
