@@ -501,7 +501,27 @@ def run_gpu(args, w):
         pack_bytes = 3 * 2 * n_half * g.heads * g.head_dim * 2
         pack = {"ms": pack_ms, "bytes": pack_bytes, "gbs": pack_bytes / (pack_ms * 1e-3) / 1e9,
                 "frac_hbm": pack_bytes / (pack_ms * 1e-3) / 1e9 / peaks()[0]["hbm_gbs"]}
-        del sets
+        # the peer-memory form (vdit_seq_pack_peers) with both ranks' destination buffers on this
+        # device: the same reads and writes, the writes as the kernel's own stores into the
+        # head-sharded buffers of every rank (over NVLink when they are another GPU's)
+        peer_sets = []
+        for ins, _, full in sets:
+            other = tuple(torch.empty_like(t) for t in full)
+            peer_sets.append((ins, [[full[x].data_ptr(), other[x].data_ptr()] for x in range(3)], other))
+
+        def one_peer_pack(i):
+            ins, addrs, _ = peer_sets[i % 2]
+            vdit.seq_pack_peers(ins[0], ins[1], ins[2], g, w.q_start, 0, 2, *addrs)
+
+        for i in range(2):
+            one_peer_pack(i)
+        with _nvtx("seq_pack_peers"):
+            peer_ms = _time_back_to_back(one_peer_pack, 20, stream)
+        pack["peers"] = {"ms": peer_ms, "gbs": pack_bytes / (peer_ms * 1e-3) / 1e9,
+                         "frac_hbm": pack_bytes / (peer_ms * 1e-3) / 1e9 / peaks()[0]["hbm_gbs"],
+                         "how": "vdit_seq_pack_peers as rank 0 of 2, both ranks' buffers on this "
+                                "device; same bytes"}
+        del sets, peer_sets
 
     # fused QKV projection + RoPE + cache append (vdit_qkv_rope) of the step's newest frames,
     # d_model = heads * head_dim (as in Wan2.1), random bf16 weights, its own cache

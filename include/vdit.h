@@ -73,6 +73,7 @@ enum {
 #define VDIT_MAX_FRAME 16383  /* largest global frame index the RoPE tables cover           */
 #define VDIT_MAX_GRID 1024    /* largest grid_h and grid_w                                  */
 #define VDIT_MAX_DT 1023      /* largest |t_q - t_k| a plan may contain                     */
+#define VDIT_MAX_PEERS 16     /* most ranks of the peer-memory exchange (vdit_seq_*_peers)  */
 
 /* Token grid, head layout and RoPE bands. heads >= 1; head_dim 64 or 128; bands even, > 0,
  * band_t + band_h + band_w == head_dim; theta > 1. */
@@ -316,6 +317,32 @@ VDIT_API int vdit_seq_pack(const vdit_geom* g, const void* q, const void* k, con
  * block r row n head j. A copy (bit-exact); out must not overlap recv or own. */
 VDIT_API int vdit_seq_unpack(const vdit_geom* g, const void* recv, const void* own, void* out, int rank,
                              int n_ranks, long long n_tokens, void* stream);
+
+/* The sequence-to-head exchange with the transfer fused into the pack ([CRoPE] 2.C "Comunicacao
+ * Fundida": the causal RoPE and the all-to-all of Q, K and V in one operation): instead of filling
+ * a send buffer for a library all-to-all, this rank's kernel writes the rows of its tokens
+ * straight into every rank's head-sharded buffers. q_dst, k_dst, v_dst: HOST arrays of n_ranks
+ * device addresses, valid in this process (rank r's q_full / k_full / v_full
+ * [n_ranks * n_tokens][heads / n_ranks][head_dim]: this rank's own buffers for r == rank, peer
+ * memory mapped over NVLink otherwise); this rank writes their rows rank * n_tokens ..
+ * (rank + 1) * n_tokens - 1, rotating Q and K at their global positions when `rotate` (as
+ * vdit_seq_pack). Every CTA ends with a system-scope memory fence, so once the kernels of all
+ * ranks have completed (the caller's barrier between the ranks, ordered after this call on
+ * `stream`), every rank's buffers hold the whole exchange. 1 <= n_ranks <= VDIT_MAX_PEERS,
+ * n_ranks divides heads; this rank's own destinations must not overlap the inputs or each other
+ * (peer ranges are not checked). */
+VDIT_API int vdit_seq_pack_peers(const vdit_geom* g, const void* q, const void* k, const void* v,
+                                 void* const* q_dst, void* const* k_dst, void* const* v_dst, int rank,
+                                 int n_ranks, int start_frame, long long n_tokens, int rotate,
+                                 void* stream);
+
+/* The return exchange after attention in push form: o_full [n_ranks * n_tokens][heads / n_ranks]
+ * [head_dim] holds this rank's heads' attention output for every rank's tokens; the rows of rank
+ * s's tokens go to out_dst[s] (rank s's out [n_tokens][heads][head_dim], a HOST array of n_ranks
+ * device addresses valid in this process) at this rank's head columns. A bit-exact copy; the same
+ * fence and barrier rule as vdit_seq_pack_peers. */
+VDIT_API int vdit_seq_push_peers(const vdit_geom* g, const void* o_full, void* const* out_dst, int rank,
+                                 int n_ranks, long long n_tokens, void* stream);
 
 /* Reads and clears the current device's kernel status word: *status = VDIT_OK, or
  * VDIT_ERR_TIMEOUT when a bounded wait in a kernel gave up since the last read. Synchronises the

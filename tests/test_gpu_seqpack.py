@@ -225,3 +225,44 @@ def test_rotated_forward_equals_forward_on_rotated_queries(wid):
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(la, lb)
     assert vdit.get_status() == vdit.OK
+
+
+# ---------------------------------------------------------------- peer-memory form of the exchange
+
+@pytest.mark.parametrize("ranks", [1, 2, 3, 4])
+def test_seq_pack_peers_equals_pack_and_exchange(ranks):
+    # vdit_seq_pack_peers writes each rank's rows straight into every rank's head-sharded
+    # buffers (here all on the one device, one rank after the other): the result equals, bit for
+    # bit, the pack into send blocks plus the exchange, for Q, K (rotated) and V
+    n_all, start = 3 * 1560 + 12 * 7, 396
+    qb, kb, vb = (synth.qkv_bf16(83, n_all, 12, 128, w) for w in ("q", "k", "v"))
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    n = n_all // ranks
+    packs = _pack_all(q, k, v, G13, start, ranks)
+    _exchange_on_one_device(packs, n)
+    hg = 12 // ranks
+    full = [tuple(torch.full((ranks * n, hg, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+                  for _ in range(3)) for _ in range(ranks)]
+    addrs = [[full[r][x].data_ptr() for r in range(ranks)] for x in range(3)]
+    for r in range(ranks):
+        sl = slice(r * n, (r + 1) * n)
+        vdit.seq_pack_peers(q[sl], k[sl], v[sl], G13, start, r, ranks, *addrs)
+    torch.cuda.synchronize()
+    for r in range(ranks):
+        for x in range(3):
+            assert torch.equal(full[r][x], packs[r][1][x])
+
+
+@pytest.mark.parametrize("ranks", [1, 2, 3])
+def test_seq_push_peers_is_the_inverse_layout(ranks):
+    n = 1000
+    hg = 12 // ranks
+    o_bits = [synth.qkv_bf16(95 + r, ranks * n, hg, 128, "v") for r in range(ranks)]
+    o_full = [dev(b) for b in o_bits]
+    outs = [torch.full((n, 12, 128), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(ranks)]
+    for r in range(ranks):
+        vdit.seq_push_peers(o_full[r], G13, r, ranks, [o.data_ptr() for o in outs])
+    torch.cuda.synchronize()
+    for s in range(ranks):
+        ref = np.concatenate([synth.bf16_bits_to_f64(o_bits[r][s * n:(s + 1) * n]) for r in range(ranks)], axis=1)
+        assert np.array_equal(f64(outs[s]), ref)

@@ -384,6 +384,23 @@ def test_calls_reject_null_and_misaligned_pointers_before_device_work():
     assert L.vdit_attn_forward(h, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
                                ctypes.c_void_p(16), None, ctypes.c_float(0.1), None) == vdit.ERR_NOT_UPLOADED
     L.vdit_plan_destroy(h)
+    # the peer-memory exchange: destination arrays checked entry by entry, ranks bounded
+    ok = (ctypes.c_void_p * 2)(16, 32)
+    null = (ctypes.c_void_p * 2)(16, 0)
+    odd = (ctypes.c_void_p * 2)(16, 40)
+    args = (ctypes.byref(g), ctypes.c_void_p(1 << 20), ctypes.c_void_p(2 << 20), ctypes.c_void_p(3 << 20))
+    assert L.vdit_seq_pack_peers(*args, ok, ok, ok, 0, 2, 0, 0, 1, None) == vdit.OK  # empty: no-op
+    assert L.vdit_seq_pack_peers(*args, null, ok, ok, 0, 2, 0, 5, 1, None) == vdit.ERR_INVALID_ARG
+    assert L.vdit_seq_pack_peers(*args, ok, odd, ok, 0, 2, 0, 5, 1, None) == vdit.ERR_MISALIGNED
+    assert L.vdit_seq_pack_peers(*args, ok, ok, ok, 0, 5, 0, 5, 1, None) == vdit.ERR_INVALID_ARG  # 5 !| 12
+    assert L.vdit_seq_pack_peers(*args, ok, ok, ok, 2, 2, 0, 5, 1, None) == vdit.ERR_INVALID_ARG  # rank
+    many = (ctypes.c_void_p * 24)(*[16] * 24)
+    g24 = vdit.Geometry(30, 52, 24, 128, (44, 42, 42)).c()
+    assert L.vdit_seq_pack_peers(ctypes.byref(g24), *args[1:], many, many, many, 0, 24, 0, 5, 1,
+                                 None) == vdit.ERR_INVALID_ARG  # more ranks than VDIT_MAX_PEERS
+    assert L.vdit_seq_push_peers(ctypes.byref(g), ctypes.c_void_p(16), null, 0, 2, 5, None) == vdit.ERR_INVALID_ARG
+    assert L.vdit_seq_push_peers(ctypes.byref(g), ctypes.c_void_p(16), odd, 0, 2, 5, None) == vdit.ERR_MISALIGNED
+    assert L.vdit_seq_push_peers(ctypes.byref(g), ctypes.c_void_p(16), ok, 0, 2, 0, None) == vdit.OK
 
 
 def test_plan_and_masks_bit_exact_on_the_gpu_edge_workloads():

@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.vdit_qkv_rope.argtypes = [P, P, P, I, I, I, P, P, P, I, P]
         L.vdit_seq_pack.argtypes = [gp, P, P, P, P, P, P, P, I, I, I, LL, I, P]
         L.vdit_seq_unpack.argtypes = [gp, P, P, P, I, I, LL, P]
+        L.vdit_seq_pack_peers.argtypes = [gp, P, P, P, P, P, P, I, I, I, LL, I, P]
+        L.vdit_seq_push_peers.argtypes = [gp, P, P, I, I, LL, P]
         L.vdit_kv_write.argtypes = [gp, P, P, I, P, P, I, I, P]
         L.vdit_attn_forward_rotated.argtypes = [P, P, P, P, P, P, F, P]
         L.vdit_plan_destroy.argtypes = [P]
@@ -369,6 +371,120 @@ def heads_to_seq(o_full: torch.Tensor, g: Geometry, group=None, out: Optional[to
         exchange({r: [o_full[r * n:(r + 1) * n]] for r in range(world) if r != rank},
                  {r: [recv[r]] for r in range(world) if r != rank}, group)
     return seq_unpack(recv, o_full[rank * n:(rank + 1) * n], out, g, rank, world, stream)
+
+
+def _addr_array(addrs, n_ranks: int, name: str):
+    addrs = [int(a) for a in addrs]
+    if len(addrs) != n_ranks or any(a == 0 for a in addrs):
+        raise ValueError(f"{name} must hold n_ranks device addresses")
+    return (ctypes.c_void_p * n_ranks)(*addrs)
+
+
+def seq_pack_peers(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, start_frame: int,
+                   rank: int, n_ranks: int, q_dst, k_dst, v_dst, rotate: bool = True, stream=None) -> None:
+    """vdit_seq_pack_peers: this rank's q, k, v [n, heads, head_dim] (chunk-local tokens rank * n
+    ..) written straight into every rank's head-sharded buffers; q_dst, k_dst, v_dst: n_ranks
+    device addresses valid in this process (rank r's q_full / k_full / v_full [n_ranks * n,
+    heads / n_ranks, head_dim]), Q and K rotated at their global positions when rotate."""
+    n = q.shape[0]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.dim() != 3 or tuple(t.shape) != (n, g.heads, g.head_dim):
+            raise ValueError(f"{name} must be bf16 [n_tokens, heads, head_dim]")
+    gc = g.c()
+    _check(lib().vdit_seq_pack_peers(ctypes.byref(gc), _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                     _addr_array(q_dst, n_ranks, "q_dst"), _addr_array(k_dst, n_ranks, "k_dst"),
+                                     _addr_array(v_dst, n_ranks, "v_dst"), int(rank), int(n_ranks),
+                                     int(start_frame), n, int(bool(rotate)), _stream(stream)))
+
+
+def seq_push_peers(o_full: torch.Tensor, g: Geometry, rank: int, n_ranks: int, out_dst, stream=None) -> None:
+    """vdit_seq_push_peers: o_full [n_ranks * n, heads / n_ranks, head_dim] (this rank's heads,
+    every rank's tokens) into every rank's out [n, heads, head_dim] at this rank's head columns;
+    out_dst: n_ranks device addresses valid in this process."""
+    hg = g.heads // n_ranks if n_ranks >= 1 else 0
+    if (o_full.dtype != torch.bfloat16 or o_full.dim() != 3 or n_ranks < 1 or g.heads % n_ranks
+            or o_full.shape[0] % n_ranks or tuple(o_full.shape[1:]) != (hg, g.head_dim)):
+        raise ValueError("o_full must be bf16 [n_ranks * n_tokens, heads / n_ranks, head_dim]")
+    gc = g.c()
+    _check(lib().vdit_seq_push_peers(ctypes.byref(gc), _dev_ptr(o_full, "o_full"),
+                                     _addr_array(out_dst, n_ranks, "out_dst"), int(rank), int(n_ranks),
+                                     o_full.shape[0] // n_ranks, _stream(stream)))
+
+
+class PeerExchange:
+    """The sequence-parallel exchange over peer memory ("Accelerating Video Generation Inference
+    with Sequential-Parallel 3D Positional Encoding Using a Global Time Index", section 2.C: the
+    RoPE and the all-to-all of Q, K and V in one operation). Each rank allocates its head-sharded
+    buffers q_full, k_full, v_full [world * n, heads / world, head_dim] and its output out [n,
+    heads, head_dim] once; their CUDA IPC handles (torch's CUDA storage sharing) are exchanged with
+    all_gather_object, so every rank holds the device addresses of every rank's buffers, and
+    vdit_seq_pack_peers / vdit_seq_push_peers do the transfer with their own stores (over NVLink
+    between GPUs). A barrier between the ranks precedes each kernel (no rank may still read the
+    buffers it is about to overwrite) and follows it (every rank's rows have landed): a
+    one-element all-reduce on the current stream with NCCL; with other backends (ranks sharing a
+    GPU, tests) a device synchronisation and a host barrier. Calls run on the current stream."""
+
+    def __init__(self, g: Geometry, n_tokens: int, group=None, device=None):
+        import torch.distributed as dist
+        self.g, self.n, self.group = g, int(n_tokens), group
+        self.world, self.rank = _group_info(group)
+        if g.heads % self.world:
+            raise ValueError("the group size must divide heads")
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        hg = g.heads // self.world
+        self.full = tuple(torch.empty(self.world * self.n, hg, g.head_dim, dtype=torch.bfloat16, device=dev)
+                          for _ in range(3))
+        self.out = torch.empty(self.n, g.heads, g.head_dim, dtype=torch.bfloat16, device=dev)
+        bufs = (*self.full, self.out)
+        self._mapped = []  # peer storages kept open for the lifetime of this object
+        if self.world == 1:
+            self.addrs = [[t.data_ptr()] for t in bufs]
+            self._nccl = False
+            return
+        self._nccl = dist.get_backend(group) == "nccl"
+        mine = []
+        for t in bufs:
+            st = t.untyped_storage()
+            mine.append((st._share_cuda_(), t.data_ptr() - st.data_ptr()))
+        everyone = [None] * self.world
+        dist.all_gather_object(everyone, mine, group=group)
+        self.addrs = [[0] * self.world for _ in bufs]
+        for r in range(self.world):
+            for i, (handle, offset) in enumerate(everyone[r]):
+                if r == self.rank:
+                    self.addrs[i][r] = bufs[i].data_ptr()
+                    continue
+                st = torch.UntypedStorage._new_shared_cuda(*handle)
+                self._mapped.append(st)
+                self.addrs[i][r] = st.data_ptr() + offset
+        self._flag = torch.zeros(1, device=dev)
+
+    def _barrier(self):
+        if self.world == 1:
+            return
+        import torch.distributed as dist
+        if self._nccl:
+            dist.all_reduce(self._flag, group=self.group)
+        else:
+            torch.cuda.synchronize()
+            dist.barrier(group=self.group)
+
+    def seq_to_heads(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, start_frame: int,
+                     rotate: bool = True):
+        """This rank's q, k, v [n, heads, head_dim] (tokens rank * n ..) -> (q_full, k_full,
+        v_full), each [world * n, heads / world, head_dim] (every token of this rank's heads)."""
+        self._barrier()
+        seq_pack_peers(q, k, v, self.g, start_frame, self.rank, self.world, *self.addrs[:3], rotate=rotate)
+        self._barrier()
+        return self.full
+
+    def heads_to_seq(self, o_full: torch.Tensor) -> torch.Tensor:
+        """o_full [world * n, heads / world, head_dim] -> out [n, heads, head_dim] (this rank's
+        tokens, every head)."""
+        self._barrier()
+        seq_push_peers(o_full, self.g, self.rank, self.world, self.addrs[3])
+        self._barrier()
+        return self.out
 
 
 class KVCache:

@@ -380,6 +380,101 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) seq_unpack_kernel(Unpa
     }
 }
 
+// The same exchange with the transfer fused into the pack: rank `rank` writes the rows of its
+// tokens straight into every rank's head-sharded buffers, dst[x][r] (rank r's q_full / k_full /
+// v_full, mapped into this process: peer memory over NVLink for r != rank), so the all-to-all is
+// the kernel's own stores and needs no send buffer or library transfer. Each CTA ends with a
+// system-scope fence: its stores are visible to the peers before the kernel completes, so a
+// barrier between the ranks after the launch is all the consumers need.
+struct PeerPackArgs {
+    StreamArgs s;  // tables, geometry, n_tokens (= n_tok), cpt, cpr_log2, start_frame
+    const uint4* src[3];
+    uint4* dst[3][VDIT_MAX_PEERS];
+    int rank;
+    int tok0;
+    int heads_per_rank;
+    FastDiv by_hpr;
+};
+
+template <bool ROTATE>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) rope_pack_peers_kernel(PeerPackArgs pa) {
+    const StreamArgs& a = pa.s;
+    const int lane = threadIdx.x & 31;
+    const int n_warps = gridDim.x * kWarpsPerBlock;
+    const int c8 = lane & ((1 << a.cpr_log2) - 1);
+    const int ft = a.grid_h * a.grid_w;
+    const int items = 3 * a.n_tokens;
+    for (int it = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); it < items; it += n_warps) {
+        const int x = it / a.n_tokens, n = it - x * a.n_tokens;
+        const bool rot = ROTATE && x < 2;
+        float2 cs[4];
+        if (rot) {
+            const int tok = pa.tok0 + n;
+            const uint32_t f = fdiv((uint32_t)tok, a.by_ft);
+            const int rem = tok - (int)f * ft;
+            const int h = (int)fdiv((uint32_t)rem, a.by_w);
+            chunk_angles(cs, c8 * 4, a.start_frame + (int)f, h, rem - h * a.grid_w, a);
+        }
+        const uint4* src = pa.src[x] + (size_t)n * a.cpt;
+        const size_t row = ((size_t)pa.rank * a.n_tokens + n) * pa.heads_per_rank;
+        for (int j0 = 0; j0 < a.cpt; j0 += 32 * kBatch) {
+            uint4 xin[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) xin[u] = __ldcs(src + j);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.cpt) {
+                    const int head = j >> a.cpr_log2;
+                    const int r = (int)fdiv((uint32_t)head, pa.by_hpr), hh = head - r * pa.heads_per_rank;
+                    uint4* dst = pa.dst[x][r] + ((row + hh) << a.cpr_log2);
+                    __stcs(dst + c8, rot ? rotate_chunk(xin[u], cs) : xin[u]);
+                }
+            }
+        }
+    }
+    __threadfence_system();
+}
+
+// Push form of the return exchange: this rank holds o_full [ranks * n_tok][heads / ranks][D], its
+// heads' attention output for every rank's tokens, and writes the rows of rank s's tokens into
+// rank s's output out_dst[s] [n_tok][heads][D] at this rank's head columns (peer memory for
+// s != rank). A copy: bit-exact. System-scope fence at the end, as above.
+struct PeerPushArgs {
+    const uint4* o_full;
+    uint4* dst[VDIT_MAX_PEERS];
+    int n_tokens, n_ranks, rank, row_chunks, cpt;  // row_chunks: (heads / ranks) * D / 8
+    FastDiv by_ntok;
+};
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4) seq_push_peers_kernel(PeerPushArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int n_warps = gridDim.x * kWarpsPerBlock;
+    const int rows = a.n_ranks * a.n_tokens;
+    for (int it = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); it < rows; it += n_warps) {
+        const int s = (int)fdiv((uint32_t)it, a.by_ntok), n = it - s * a.n_tokens;
+        const uint4* src = a.o_full + (size_t)it * a.row_chunks;
+        uint4* dst = a.dst[s] + (size_t)n * a.cpt + (size_t)a.rank * a.row_chunks;
+        for (int j0 = 0; j0 < a.row_chunks; j0 += 32 * kBatch) {
+            uint4 xin[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.row_chunks) xin[u] = __ldcs(src + j);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.row_chunks) __stcs(dst + j, xin[u]);
+            }
+        }
+    }
+    __threadfence_system();
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int fill_common(const vdit_geom* g, StreamArgs& a) {
@@ -587,4 +682,109 @@ extern "C" int vdit_seq_unpack(const vdit_geom* g, const void* recv, const void*
     const int blocks = (int)std::min<long long>(want, (long long)sm_count() * 4);
     seq_unpack_kernel<<<blocks, kWarpsPerBlock * 32, 0, static_cast<cudaStream_t>(stream)>>>(a);
     return vdit::cuda_check(cudaGetLastError(), "unpack kernel launch");
+}
+
+extern "C" int vdit_seq_pack_peers(const vdit_geom* g, const void* q, const void* k, const void* v,
+                                   void* const* q_dst, void* const* k_dst, void* const* v_dst, int rank,
+                                   int n_ranks, int start_frame, long long n_tokens, int rotate, void* stream) {
+    using vdit::fail;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (n_tokens < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens must be >= 0");
+    if (n_ranks < 1 || n_ranks > VDIT_MAX_PEERS || g->heads % n_ranks != 0)
+        return fail(VDIT_ERR_INVALID_ARG, "n_ranks must divide heads and be at most VDIT_MAX_PEERS");
+    if (rank < 0 || rank >= n_ranks) return fail(VDIT_ERR_INVALID_ARG, "rank outside [0, n_ranks)");
+    if (n_tokens == 0) return VDIT_OK;
+    if (!q || !k || !v || !q_dst || !k_dst || !v_dst) return fail(VDIT_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return fail(VDIT_ERR_MISALIGNED, "input not 16-byte aligned");
+    for (int r = 0; r < n_ranks; ++r) {
+        if (!q_dst[r] || !k_dst[r] || !v_dst[r]) return fail(VDIT_ERR_INVALID_ARG, "NULL destination");
+        if (!aligned16(q_dst[r]) || !aligned16(k_dst[r]) || !aligned16(v_dst[r]))
+            return fail(VDIT_ERR_MISALIGNED, "destination not 16-byte aligned");
+    }
+    const long long ft = (long long)g->grid_h * g->grid_w;
+    const long long tok0 = (long long)rank * n_tokens, last = tok0 + n_tokens - 1;
+    if (start_frame < 0 || start_frame + last / ft > VDIT_MAX_FRAME)
+        return fail(VDIT_ERR_INVALID_ARG, "frames outside [0, VDIT_MAX_FRAME]");
+    if ((unsigned long long)n_tokens * n_ranks * g->heads * (g->head_dim / 8) >= (1ull << 31) ||
+        (long long)n_tokens * n_ranks >= (1ll << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "exchange larger than 2^31 16-byte chunks");
+    // this rank's own head-sharded buffers (the only destinations in this address space that the
+    // call can tell apart from peer mappings) must not overlap the inputs or one another
+    const long long in_bytes = n_tokens * g->heads * g->head_dim * 2;
+    const long long full_bytes = in_bytes;  // n_ranks * n_tokens * (heads / n_ranks) * D * 2
+    const void* ins[3] = {q, k, v};
+    const void* own[3] = {q_dst[rank], k_dst[rank], v_dst[rank]};
+    auto overlap = [](const void* a, long long na, const void* b, long long nb) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        return x < y + nb && y < x + na;
+    };
+    for (int i = 0; i < 3; ++i) {
+        for (int j = 0; j < 3; ++j)
+            if (overlap(own[i], full_bytes, ins[j], in_bytes))
+                return fail(VDIT_ERR_INVALID_ARG, "an output overlaps an input");
+        for (int j = i + 1; j < 3; ++j)
+            if (overlap(own[i], full_bytes, own[j], full_bytes))
+                return fail(VDIT_ERR_INVALID_ARG, "outputs overlap each other");
+    }
+    PeerPackArgs pa{};
+    if (int rc = fill_common(g, pa.s)) return rc;
+    pa.s.n_tokens = (int)n_tokens;
+    pa.s.start_frame = start_frame;
+    pa.src[0] = static_cast<const uint4*>(q);
+    pa.src[1] = static_cast<const uint4*>(k);
+    pa.src[2] = static_cast<const uint4*>(v);
+    void* const* dsts[3] = {q_dst, k_dst, v_dst};
+    for (int x = 0; x < 3; ++x)
+        for (int r = 0; r < n_ranks; ++r) pa.dst[x][r] = static_cast<uint4*>(dsts[x][r]);
+    pa.rank = rank;
+    pa.tok0 = (int)tok0;
+    pa.heads_per_rank = g->heads / n_ranks;
+    pa.by_hpr = make_fastdiv((uint32_t)pa.heads_per_rank);
+    const long long want = (3 * n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int blocks = (int)std::min<long long>(want, (long long)sm_count() * 4);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rotate)
+        rope_pack_peers_kernel<true><<<blocks, kWarpsPerBlock * 32, 0, st>>>(pa);
+    else
+        rope_pack_peers_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, st>>>(pa);
+    return vdit::cuda_check(cudaGetLastError(), "peer pack kernel launch");
+}
+
+extern "C" int vdit_seq_push_peers(const vdit_geom* g, const void* o_full, void* const* out_dst, int rank,
+                                   int n_ranks, long long n_tokens, void* stream) {
+    using vdit::fail;
+    if (int rc = vdit::check_geom(g)) return rc;
+    if (n_tokens < 0) return fail(VDIT_ERR_INVALID_ARG, "n_tokens must be >= 0");
+    if (n_ranks < 1 || n_ranks > VDIT_MAX_PEERS || g->heads % n_ranks != 0)
+        return fail(VDIT_ERR_INVALID_ARG, "n_ranks must divide heads and be at most VDIT_MAX_PEERS");
+    if (rank < 0 || rank >= n_ranks) return fail(VDIT_ERR_INVALID_ARG, "rank outside [0, n_ranks)");
+    if (n_tokens == 0) return VDIT_OK;
+    if (!o_full || !out_dst) return fail(VDIT_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(o_full)) return fail(VDIT_ERR_MISALIGNED, "o_full not 16-byte aligned");
+    for (int r = 0; r < n_ranks; ++r) {
+        if (!out_dst[r]) return fail(VDIT_ERR_INVALID_ARG, "NULL destination");
+        if (!aligned16(out_dst[r])) return fail(VDIT_ERR_MISALIGNED, "destination not 16-byte aligned");
+    }
+    const long long out_bytes = n_tokens * g->heads * g->head_dim * 2;
+    const long long in_bytes = out_bytes;  // n_ranks * n_tokens * (heads / n_ranks) * D * 2
+    const char* x = static_cast<const char*>(o_full);
+    const char* y = static_cast<const char*>(out_dst[rank]);
+    if (x < y + out_bytes && y < x + in_bytes) return fail(VDIT_ERR_INVALID_ARG, "output overlaps o_full");
+    if ((unsigned long long)n_tokens * n_ranks * g->heads * (g->head_dim / 8) >= (1ull << 31) ||
+        (long long)n_tokens * n_ranks >= (1ll << 31))
+        return fail(VDIT_ERR_UNSUPPORTED, "exchange larger than 2^31 16-byte chunks");
+    PeerPushArgs a{};
+    a.o_full = static_cast<const uint4*>(o_full);
+    for (int r = 0; r < n_ranks; ++r) a.dst[r] = static_cast<uint4*>(out_dst[r]);
+    a.n_tokens = (int)n_tokens;
+    a.n_ranks = n_ranks;
+    a.rank = rank;
+    a.row_chunks = (g->heads / n_ranks) * (g->head_dim / 8);
+    a.cpt = g->heads * (g->head_dim / 8);
+    a.by_ntok = make_fastdiv((uint32_t)n_tokens);
+    const long long want = ((long long)n_ranks * n_tokens + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int blocks = (int)std::min<long long>(want, (long long)sm_count() * 4);
+    seq_push_peers_kernel<<<blocks, kWarpsPerBlock * 32, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return vdit::cuda_check(cudaGetLastError(), "peer push kernel launch");
 }
