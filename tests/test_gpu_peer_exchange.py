@@ -52,7 +52,7 @@ def _worker(rank, world, port, out):
         torch.cuda.synchronize()
         assert vdit.get_status() == vdit.OK
         out[rank] = (got_full, o.view(torch.int16).cpu().numpy().copy())
-        dist.barrier()  # no rank unmaps while another may still write
+        ex.close()  # collective: no rank unmaps while another may still write
         del ex
     finally:
         dist.destroy_process_group()

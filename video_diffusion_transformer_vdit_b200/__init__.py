@@ -422,7 +422,10 @@ class PeerExchange:
     between GPUs). A barrier between the ranks precedes each kernel (no rank may still read the
     buffers it is about to overwrite) and follows it (every rank's rows have landed): a
     one-element all-reduce on the current stream with NCCL; with other backends (ranks sharing a
-    GPU, tests) a device synchronisation and a host barrier. Calls run on the current stream."""
+    GPU, tests) a device synchronisation and a host barrier. Calls run on the current stream.
+    Every rank's buffers are mapped by the others, so the ranks keep their exchanges alive
+    together and release them together: close() (a barrier, then the mappings are dropped) on
+    every rank before any rank frees its exchange."""
 
     def __init__(self, g: Geometry, n_tokens: int, group=None, device=None):
         import torch.distributed as dist
@@ -468,6 +471,13 @@ class PeerExchange:
         else:
             torch.cuda.synchronize()
             dist.barrier(group=self.group)
+
+    def close(self) -> None:
+        """Collective: waits until no rank can still write into this rank's buffers, then drops
+        the mappings of the other ranks' buffers."""
+        self._barrier()
+        self._mapped.clear()
+        self.addrs = None
 
     def seq_to_heads(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, start_frame: int,
                      rotate: bool = True):
