@@ -229,24 +229,28 @@ def test_rotated_forward_equals_forward_on_rotated_queries(wid):
 
 # ---------------------------------------------------------------- peer-memory form of the exchange
 
-@pytest.mark.parametrize("ranks", [1, 2, 3, 4])
-def test_seq_pack_peers_equals_pack_and_exchange(ranks):
+G64 = vdit.Geometry(6, 10, 4, 64, (24, 20, 20))
+
+
+@pytest.mark.parametrize("ranks,d", [(1, 128), (2, 128), (3, 128), (4, 128), (2, 64), (4, 64)])
+def test_seq_pack_peers_equals_pack_and_exchange(ranks, d):
     # vdit_seq_pack_peers writes each rank's rows straight into every rank's head-sharded
     # buffers (here all on the one device, one rank after the other): the result equals, bit for
     # bit, the pack into send blocks plus the exchange, for Q, K (rotated) and V
-    n_all, start = 3 * 1560 + 12 * 7, 396
-    qb, kb, vb = (synth.qkv_bf16(83, n_all, 12, 128, w) for w in ("q", "k", "v"))
+    g = G13 if d == 128 else G64
+    n_all, start = (3 * 1560 + 12 * 7, 396) if d == 128 else (7 * 60 + 4 * 3, 11)
+    qb, kb, vb = (synth.qkv_bf16(83, n_all, g.heads, d, w) for w in ("q", "k", "v"))
     q, k, v = dev(qb), dev(kb), dev(vb)
     n = n_all // ranks
-    packs = _pack_all(q, k, v, G13, start, ranks)
+    packs = _pack_all(q, k, v, g, start, ranks)
     _exchange_on_one_device(packs, n)
-    hg = 12 // ranks
-    full = [tuple(torch.full((ranks * n, hg, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    hg = g.heads // ranks
+    full = [tuple(torch.full((ranks * n, hg, d), float("nan"), dtype=torch.bfloat16, device="cuda")
                   for _ in range(3)) for _ in range(ranks)]
     addrs = [[full[r][x].data_ptr() for r in range(ranks)] for x in range(3)]
     for r in range(ranks):
         sl = slice(r * n, (r + 1) * n)
-        vdit.seq_pack_peers(q[sl], k[sl], v[sl], G13, start, r, ranks, *addrs)
+        vdit.seq_pack_peers(q[sl], k[sl], v[sl], g, start, r, ranks, *addrs)
     torch.cuda.synchronize()
     for r in range(ranks):
         for x in range(3):
