@@ -150,6 +150,31 @@ def test_rope_frequency_ladder_and_direction(g):
         assert np.allclose(ratios, g.theta ** (-2.0 / width), rtol=1e-12, atol=0)
 
 
+@pytest.mark.parametrize("g", [G128, G64])
+def test_rope_each_band_equals_a_library_rotary_embedding(g):
+    # External pin of the pairing and the ladder: each band of the 3-D RoPE is a 1-D rotary
+    # embedding over adjacent channel pairs, which is the convention of the GPT-J rotary in
+    # transformers (rotate_every_two, sinusoids with inverse frequencies 10000^(-2j/width)).
+    # The library computes in fp32, so positions stay small enough for its angles to be exact
+    # to ~1e-5; a rotate-half pairing, a reversed rotation or a shifted band fails by O(1).
+    gptj = pytest.importorskip("transformers.models.gptj.modeling_gptj")
+    assert g.theta == 10000.0
+    n = 2 * g.frame_tokens
+    x = _rand(29, (n, g.heads, g.head_dim))
+    t, h, w = _pos(n, g, 37)
+    y = oracle.rope3d(x, (t, h, w), g)
+    bands = [(0, g.band_t, t), (g.band_t, g.band_t + g.band_h, h),
+             (g.band_t + g.band_h, g.head_dim, w)]
+    for lo, hi, p in bands:
+        width = hi - lo
+        table = gptj.create_sinusoidal_positions(int(p.max()) + 1, width)  # [pos, sin | cos]
+        sincos = table[torch.from_numpy(p.astype(np.int64))]
+        sin, cos = sincos[:, : width // 2], sincos[:, width // 2:]
+        xb = torch.from_numpy(x[None, :, :, lo:hi].astype(np.float32))  # [1, n, heads, width]
+        ref = gptj.apply_rotary_pos_emb(xb, sin[None], cos[None])[0].double().numpy()
+        assert np.max(np.abs(y[:, :, lo:hi] - ref)) < 1e-4
+
+
 # ----------------------------------------------------------------------------- mask
 
 def _golden_mask_cases():
