@@ -285,11 +285,36 @@ def _time_back_to_back(fn, n, stream):
     return a.elapsed_time(b) / n
 
 
-def time_append(vdit, g, capacity_frames, n_frames, start_frame, dev, stream, n=20):
+def _time_graph(fn, n_calls, stream, reps=5):
+    """Mean device time (ms) per call of fn(i), i < n_calls, captured once into one CUDA graph
+    and replayed `reps` times back to back (CUDA events on `stream`): the calls run with no host
+    launch gap between them."""
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(n_calls):
+            fn(i)
+    graph.replay()  # warm-up replay
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * n_calls)
+    del graph
+    return ms
+
+
+def time_append(vdit, g, capacity_frames, n_frames, start_frame, dev, stream, n=20, graph_calls=30):
     """vdit_kv_append of one n_frames chunk, timed back to back over distinct (source, cache)
     sets whose total exceeds L2, so no launch finds its input in L2 and each pays for the
-    write-back its predecessor left there. Returns (ms, algorithmic bytes: read K, V + write K',
-    V)."""
+    write-back its predecessor left there; then the same appends, graph_calls of them (one per
+    DiT block of Wan2.1-1.3B), captured in one CUDA graph, which takes the host's launch gaps
+    out of small appends. Returns (ms, algorithmic bytes: read K, V + write K', V, torch copy ms,
+    graph ms)."""
     ft = g.grid_h * g.grid_w
     shape = (n_frames * ft, g.heads, g.head_dim)
     per_set = 4 * int(np.prod(shape)) * 2
@@ -321,7 +346,9 @@ def time_append(vdit, g, capacity_frames, n_frames, start_frame, dev, stream, n=
     for i in range(n_sets):
         copy(i)
     copy_ms = _time_back_to_back(copy, n, stream)
-    return ms, per_set, copy_ms
+    with _nvtx(f"kv_append graph of {graph_calls}, {n_frames} frames x {g.heads} heads"):
+        graph_ms = _time_graph(one, graph_calls, stream)
+    return ms, per_set, copy_ms, graph_ms
 
 
 def time_workload(vdit, w, dev, stream, burst_peak, n=10):
@@ -564,11 +591,13 @@ def run_gpu(args, w):
     for name, heads, nf, start in (("clip", g.heads, n_last, s_last),
                                    ("chunk_1.3b_h12", 12, 3, 18), ("chunk_14b_h40", 40, 3, 396)):
         ga = vdit.Geometry(g.grid_h, g.grid_w, heads, g.head_dim, g.bands, g.theta)
-        a_ms, a_bytes, c_ms = time_append(vdit, ga, w.capacity_frames if name == "clip" else 21, nf,
-                                          start, dev, stream)
+        a_ms, a_bytes, c_ms, g_ms = time_append(vdit, ga, w.capacity_frames if name == "clip" else 21,
+                                                nf, start, dev, stream)
         gbs = a_bytes / (a_ms * 1e-3) / 1e9
         appends[name] = {"frames": nf, "heads": heads, "ms": a_ms, "bytes": a_bytes, "gbs": gbs,
                          "frac_hbm": gbs / pk0["hbm_gbs"],
+                         "graph_ms": g_ms, "graph_gbs": a_bytes / (g_ms * 1e-3) / 1e9,
+                         "graph_frac_hbm": a_bytes / (g_ms * 1e-3) / 1e9 / pk0["hbm_gbs"],
                          "torch_copy_same_bytes_gbs": a_bytes / (c_ms * 1e-3) / 1e9}
     torch.cuda.synchronize()
 
@@ -709,6 +738,8 @@ def run_gpu(args, w):
                 "kv_append_frac_hbm": appends["clip"]["frac_hbm"],
                 "kv_append": dict(appends, how="vdit_kv_append alone, 20 launches back to back "
                                   "over distinct source and cache buffers (> 400 MB in all); "
+                                  "graph_*: 30 of the same appends (one per DiT block) captured "
+                                  "in one CUDA graph, 5 replays; "
                                   "bytes = read K, V + write K', V; torch_copy_same_bytes_gbs: "
                                   "torch's device copy of K and V (two launches) over the same "
                                   "buffers, for context"),

@@ -36,6 +36,12 @@
  *   - Every call is asynchronous on the caller's CUDA stream (a cudaStream_t passed as void*;
  *     NULL = legacy default stream) except vdit_attn_plan, vdit_plan_info and vdit_plan_export,
  *     which are host-only, and vdit_get_status, which synchronises the device.
+ *   - CUDA graphs: the first call of a launching entry point on a device may set up state there
+ *     (the RoPE tables of a band set, kernel attributes); after one such call has run outside a
+ *     capture, the launching calls (vdit_rope3d_apply, vdit_kv_append, vdit_kv_write,
+ *     vdit_attn_forward and its variants on an uploaded plan, vdit_qkv_rope, the pack and push
+ *     calls) neither allocate nor synchronise, so they may be captured into a CUDA graph on the
+ *     caller's stream. A replay reads the captured pointers' current contents.
  *   - Errors: each call returns VDIT_OK (0) or a negative VDIT_ERR_* code and never throws;
  *     vdit_last_error() gives a thread-local message for the last failure on this thread.
  *     Argument checks happen before any launch, so a rejected call has no effect.
