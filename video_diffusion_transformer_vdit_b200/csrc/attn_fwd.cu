@@ -366,10 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // dynamic-threshold attention pass: a candidate is kept iff s c + (tau_log2 - m c) >= 0
             // (its logit within tau of the row maximum). z = (s c + (tau_log2 - m c)) 2^64 is one
             // packed FMA from s; the power-of-two factor changes no rounding, so z >= 0 exactly
-            // when that fp32 sum is. A kept candidate has z >= 0 >= x = s c - m c, so min(x, z) = x;
-            // a dropped one has a sum below 0 by at least the spacing of the operands' products
-            // (~2^-46 at the magnitudes of the logits), so z < -150 and ex2.approx.ftz of min(x, z)
-            // is exactly 0. Two instructions per pair fewer than a compare and a select per element.
+            // when that fp32 sum is. A kept candidate has z >= 0 >= x = s c - m c, so min(x, z) = x.
+            // A dropped one has z < 0: unless its sum lies within 150 * 2^-64 (~1e-17) of 0, z is
+            // below -150 and ex2.approx.ftz of min(x, z) is exactly 0; inside that band, far inside
+            // the fp32 rounding of the logits themselves, its weight lies between 0 and the kept
+            // one. Two instructions per pair fewer than a compare and a select per element.
             constexpr float kZ = 18446744073709551616.f;  // 2^64
             uint64_t cz2 = 0, bz2 = 0;
             if constexpr (pass1) {
