@@ -230,6 +230,8 @@ VDIT_API int vdit_plan_export_masks(const vdit_plan* p, int* mask_index, unsigne
 VDIT_API int vdit_plan_export_work(const vdit_plan* p, int* row_ptr, int* key_row, int* mask_index,
                                    unsigned int* words);
 
+/* Frees the plan and its device copy (cudaFree). A forward launched on the plan reads that copy
+ * until it completes: synchronise its stream before destroying the plan. NULL is a no-op. */
 VDIT_API void vdit_plan_destroy(vdit_plan* p);
 
 /* Attention forward over an uploaded plan. q: UNROTATED queries, device bf16
